@@ -1,0 +1,44 @@
+"""CPU oracle for the pi0 / pi0.5 joint (prefix-LM) attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this package:
+only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg
+(and its ``--impl reference`` arm) may call it.  It shares no code with the CUDA
+library under ``vla_prefix_lm_b200/csrc`` and imports nothing from the product
+package.
+
+Everything is plain numpy in float64: the visibility mask is built explicitly
+as a boolean matrix from the pages' rule, the scores are a plain matrix
+product, and the softmax is the textbook definition.  See ``attention.py`` for
+the joint prefill / suffix-pass attention, ``brute.py`` for an independent
+per-pair visibility enumerator, and ``counts.py`` for the attention-pair
+counting convention.
+
+Parity status per function (what pins it; tests live in tests/test_oracle.py):
+
+* ``prefill_mask`` / ``suffix_mask`` -- pinned: the Pi0-FAST mask picture
+  (golden file), the pi0.5 five-row permission table (golden file), the
+  all-False / all-True special cases, and exhaustive agreement with the
+  independent ``brute.visible`` if-chain on every ar pattern up to S = 10.
+* ``attention`` / ``prefill`` / ``suffix`` -- pinned: closed forms (q = 0 gives
+  the mean of the visible values; a single visible key returns its value row),
+  invariances (duplicated heads, key permutation inside a bidirectional
+  block), equality with torch's scaled_dot_product_attention in float64, the
+  log-sum-exp against scipy, and suffix-pass == prefill suffix rows.
+* ``counts.control_step_pairs`` -- parity unpinned: the pages quote about
+  1.2e6 pairs per pi0.5 control step without a derivation; the count is only
+  checked to be of that order.
+"""
+
+from .attention import (  # noqa: F401
+    EXPERT,
+    FAST,
+    OTHER,
+    ar_cumsum,
+    attention,
+    prefill,
+    prefill_mask,
+    softmax_probs,
+    suffix,
+    suffix_mask,
+)
+from . import brute, counts  # noqa: F401

@@ -1,0 +1,405 @@
+"""Pins for the CPU oracle against what the pages and the mathematics fix.
+
+None of these checks re-types the oracle's formula: the masks are compared to
+the pages' own pictures and tables (tests/golden, each file cites its page),
+to an independent boundary-walking enumerator over all small ar patterns, and
+the attention values to closed forms, invariances, torch's float64
+scaled_dot_product_attention and scipy's logsumexp.
+"""
+
+import itertools
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+from oracle import brute, counts
+from oracle.attention import EXPERT, FAST, OTHER
+
+from conftest import GOLDEN
+
+
+def _load_rows(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+# ------------------------------------------------------------------ masks
+
+
+def test_fast_mask_picture():
+    """Pi0-FAST 模型架构 2.3: 3 image + 2 language + 3 action tokens."""
+    ar = [0, 0, 0, 0, 0, 1, 1, 1]
+    M = oracle.prefill_mask(ar)[0]
+    seen = set()
+    for label, toks, bits in _load_rows("fast_mask_picture.txt"):
+        want = np.array([c == "1" for c in bits])
+        for t in map(int, toks.split(",")):
+            np.testing.assert_array_equal(M[t], want, err_msg=label)
+            seen.add(t)
+    assert seen == set(range(8))
+
+
+def test_causal_tril_all_true():
+    """VLA论文阅读 Part 3: an all-True ar_mask is the causal (lower-triangular) mask."""
+    want = np.array([[c == "1" for c in r[0]] for r in _load_rows("causal_verify_tril.txt")])
+    np.testing.assert_array_equal(oracle.prefill_mask([1, 1, 1, 1])[0], want)
+    for S in (1, 7, 33):
+        np.testing.assert_array_equal(oracle.prefill_mask(np.ones(S))[0],
+                                      np.tril(np.ones((S, S), bool)))
+
+
+def test_all_false_is_bidirectional():
+    """MM-DiT is fully bidirectional: all-False ar_mask sees every key."""
+    for S in (1, 5, 154):
+        assert oracle.prefill_mask(np.zeros(S))[0].all()
+
+
+def test_pi0_prefix_never_sees_suffix():
+    """OpenPI 1.2: prefix <-> prefix, suffix -> prefix, prefix -/-> suffix."""
+    n_pre = 20
+    ar = [0] * n_pre + [1, 1] + [0] * 9
+    M = oracle.prefill_mask(ar)[0]
+    assert M[:n_pre, :n_pre].all()
+    assert not M[:n_pre, n_pre:].any()
+    assert M[n_pre:, :n_pre].all()
+    # state row sees prefix + itself only; action rows see state and all actions
+    assert M[n_pre, : n_pre + 1].all() and not M[n_pre, n_pre + 1:].any()
+    assert M[n_pre + 1:, :].all()
+
+
+_SEG_NAME = {OTHER: "prefix", FAST: "FAST", EXPERT: "expert"}
+
+
+def _check_permission_table(n_pre, n_fast, n_exp):
+    ar = [0] * n_pre + [1] * n_fast + [1] + [0] * (n_exp - 1)
+    seg = [OTHER] * n_pre + [FAST] * n_fast + [EXPERT] * n_exp
+    M = oracle.prefill_mask(ar, seg)[0]
+    spans = {"prefix": slice(0, n_pre), "FAST": slice(n_pre, n_pre + n_fast),
+             "expert": slice(n_pre + n_fast, n_pre + n_fast + n_exp)}
+    rows = _load_rows("pi05_permission_table.txt")
+    assert len(rows) == 9
+    for qname, kname, rel in rows:
+        blk = M[spans[qname], spans[kname]]
+        if rel == "all":
+            assert blk.all(), (qname, kname)
+        elif rel == "none":
+            assert not blk.any(), (qname, kname)
+        elif rel == "causal":
+            assert blk.shape[0] == blk.shape[1]
+            np.testing.assert_array_equal(blk, np.tril(np.ones(blk.shape, bool)))
+        else:
+            raise AssertionError(rel)
+    return ar, seg
+
+
+def test_pi05_permission_table_small():
+    _check_permission_table(6, 4, 5)
+
+
+def test_pi05_permission_table_full_layout():
+    """The pi0.5 layout of the three-segment workload: 824 | 64 | 50."""
+    ar, seg = _check_permission_table(824, 64, 50)
+    # the cumsum rule alone would let expert queries read FAST keys: the
+    # segment term is what enforces the table's last row
+    M_nosg = oracle.prefill_mask(ar)[0]
+    assert M_nosg[824 + 64:, 824:824 + 64].all()
+
+
+def test_brute_force_all_patterns():
+    """cumsum rule == boundary-walking if-chain on every ar pattern, S <= 10."""
+    for S in range(1, 11):
+        for bits in itertools.product((0, 1), repeat=S):
+            M = oracle.prefill_mask(list(bits))[0]
+            np.testing.assert_array_equal(M, np.array(brute.mask(list(bits))), err_msg=str(bits))
+
+
+def test_brute_force_random_segments():
+    rng = np.random.default_rng(7)
+    for _ in range(400):
+        S = int(rng.integers(1, 13))
+        ar = rng.integers(0, 2, S)
+        seg = rng.integers(0, 3, S)
+        M = oracle.prefill_mask(ar, seg)[0]
+        np.testing.assert_array_equal(M, np.array(brute.mask(list(ar), list(seg))))
+
+
+def test_batched_ar_and_seg():
+    """[B, S] ar / seg give per-batch masks; 1-D ones broadcast."""
+    ar = np.array([[0, 0, 1, 0], [1, 1, 1, 1]])
+    seg = np.array([[0, 1, 2, 2], [0, 0, 0, 0]])
+    M = oracle.prefill_mask(ar, seg)
+    for b in range(2):
+        np.testing.assert_array_equal(M[b], np.array(brute.mask(list(ar[b]), list(seg[b]))))
+    assert oracle.prefill_mask([0, 1], B=3).shape == (3, 2, 2)
+
+
+def test_suffix_mask_construction():
+    """OpenPI 1.6: every suffix row sees every prefix key, then make_attn_mask over the suffix."""
+    ar_suf = [1, 1, 0, 0]
+    M = oracle.suffix_mask(ar_suf, P=5)[0]
+    assert M.shape == (4, 9)
+    assert M[:, :5].all()
+    np.testing.assert_array_equal(M[:, 5:], np.array(brute.mask(ar_suf)))
+
+
+# ------------------------------------------------------------ attention values
+
+
+def _rand(shape, rng, s=1.0):
+    return rng.standard_normal(shape) * s
+
+
+def test_softmax_rows_sum_to_one_and_masked_zero():
+    rng = np.random.default_rng(1)
+    S = 40
+    ar = (rng.random(S) < 0.2).astype(int)
+    M = oracle.prefill_mask(ar)[0]
+    p = oracle.softmax_probs(_rand((S, S), rng, 3.0), M)
+    np.testing.assert_allclose(p.sum(-1), 1.0, rtol=0, atol=1e-12)
+    assert (p[~M] == 0).all()
+    assert (p[M] > 0).all()
+
+
+def test_q_zero_gives_mean_of_visible_values():
+    rng = np.random.default_rng(2)
+    B, S, Hq, d = 2, 17, 4, 8
+    ar = [0] * 6 + [1, 0, 0, 1, 1, 0, 0, 0, 1, 0, 0]
+    q = np.zeros((B, S, Hq, d))
+    k = _rand((B, S, 1, d), rng)
+    v = _rand((B, S, 1, d), rng)
+    out, lse = oracle.prefill(q, k, v, ar)
+    M = np.array(brute.mask(ar))
+    for b in range(B):
+        for i in range(S):
+            want = v[b, M[i], 0, :].mean(0)
+            for h in range(Hq):
+                np.testing.assert_allclose(out[b, i, h], want, atol=1e-13)
+                # all visible logits are 0: lse = log(#visible)
+                assert abs(lse[b, i, h] - np.log(M[i].sum())) < 1e-13
+
+
+def test_single_visible_key_returns_its_value():
+    rng = np.random.default_rng(3)
+    B, S, Hq, d = 1, 9, 2, 16
+    q = _rand((B, S, Hq, d), rng)
+    k = _rand((B, S, 1, d), rng)
+    v = _rand((B, S, 1, d), rng)
+    out, _ = oracle.prefill(q, k, v, [1] * S)
+    for h in range(Hq):
+        np.testing.assert_allclose(out[0, 0, h], v[0, 0, 0], atol=1e-14)
+
+
+def test_duplicated_heads_identical():
+    rng = np.random.default_rng(4)
+    B, S, Hq, d = 2, 21, 8, 32
+    q = _rand((B, S, Hq, d), rng)
+    q[:, :, 5] = q[:, :, 2]
+    k = _rand((B, S, 1, d), rng)
+    v = _rand((B, S, 1, d), rng)
+    ar = [0] * 10 + [1, 1] + [0] * 9
+    out, _ = oracle.prefill(q, k, v, ar)
+    np.testing.assert_array_equal(out[:, :, 5], out[:, :, 2])
+
+
+def test_key_permutation_inside_bidirectional_block():
+    """Keys of one bidirectional block are a set: permuting them (with V) changes nothing."""
+    rng = np.random.default_rng(5)
+    B, S, Hq, d = 1, 30, 4, 16
+    ar = [0] * 20 + [1] + [0] * 9
+    q = _rand((B, S, Hq, d), rng)
+    k = _rand((B, S, 1, d), rng)
+    v = _rand((B, S, 1, d), rng)
+    out, lse = oracle.prefill(q, k, v, ar)
+    perm = np.arange(S)
+    perm[:20] = rng.permutation(20)
+    out2, lse2 = oracle.prefill(q, k[:, perm], v[:, perm], ar)
+    np.testing.assert_allclose(out2, out, atol=1e-13)
+    np.testing.assert_allclose(lse2, lse, atol=1e-13)
+
+
+@pytest.mark.parametrize("Hq,Hkv,scale", [(8, 1, 1.0), (4, 2, 0.37), (2, 1, 1 / 8.0)])
+def test_equals_torch_sdpa_float64(Hq, Hkv, scale):
+    """Library special case: torch SDPA (float64, CPU) with the explicit bool mask."""
+    rng = np.random.default_rng(6)
+    B, S, d = 2, 37, 16
+    ar = [0] * 15 + [1] * 8 + [1] + [0] * 13
+    seg = [OTHER] * 15 + [FAST] * 8 + [EXPERT] * 14
+    q = _rand((B, S, Hq, d), rng)
+    k = _rand((B, S, Hkv, d), rng)
+    v = _rand((B, S, Hkv, d), rng)
+    out, _ = oracle.prefill(q, k, v, ar, seg, scale=scale)
+    M = torch.from_numpy(np.array(brute.mask(ar, seg)))
+    tq, tk, tv = (torch.from_numpy(x).permute(0, 2, 1, 3) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk, tv, attn_mask=M, scale=scale, enable_gqa=True)
+    np.testing.assert_allclose(out, ref.permute(0, 2, 1, 3).numpy(), atol=1e-12)
+
+
+def test_lse_matches_scipy_logsumexp():
+    rng = np.random.default_rng(8)
+    B, S, Hq, d = 1, 25, 2, 8
+    ar = [0] * 12 + [1] + [0] * 12
+    q = _rand((B, S, Hq, d), rng)
+    k = _rand((B, S, 1, d), rng)
+    v = _rand((B, S, 1, d), rng)
+    _, lse = oracle.prefill(q, k, v, ar, scale=0.5)
+    M = np.array(brute.mask(ar))
+    for i in range(S):
+        for h in range(Hq):
+            s = 0.5 * (k[0, :, 0] @ q[0, i, h])
+            assert abs(lse[0, i, h] - scipy.special.logsumexp(s[M[i]])) < 1e-12
+
+
+def test_pure_python_brute_attention():
+    """Pure-Python loops (math.exp) over brute.visible agree with the oracle."""
+    rng = np.random.default_rng(9)
+    B, S, Hq, d = 1, 11, 2, 4
+    ar = [0, 0, 0, 1, 1, 0, 1, 0, 0, 1, 1]
+    seg = [0, 0, 0, 1, 1, 1, 2, 2, 2, 0, 1]
+    q = _rand((B, S, Hq, d), rng)
+    k = _rand((B, S, 1, d), rng)
+    v = _rand((B, S, 1, d), rng)
+    out, _ = oracle.prefill(q, k, v, ar, seg, scale=0.8)
+    for i in range(S):
+        vis = [brute.visible(i, j, ar, seg) for j in range(S)]
+        for h in range(Hq):
+            want = brute.attention_row(list(q[0, i, h]), k[0, :, 0].tolist(),
+                                       v[0, :, 0].tolist(), vis, scale=0.8)
+            np.testing.assert_allclose(out[0, i, h], want, atol=1e-13)
+
+
+def test_suffix_pass_equals_prefill_suffix_rows():
+    """Suffix-only pass == rows [P:] of the joint prefill, for any prefix queries."""
+    rng = np.random.default_rng(10)
+    B, P, Sq, Hq, d = 2, 13, 9, 4, 8
+    ar_suf = [1, 1] + [0] * (Sq - 2)
+    k_c, v_c = _rand((B, P, 1, d), rng), _rand((B, P, 1, d), rng)
+    qs, ks, vs = _rand((B, Sq, Hq, d), rng), _rand((B, Sq, 1, d), rng), _rand((B, Sq, 1, d), rng)
+    out_s, lse_s = oracle.suffix(qs, ks, vs, k_c, v_c, ar_suf, scale=0.7)
+    for trial in range(2):
+        q_pre = _rand((B, P, Hq, d), rng)
+        q = np.concatenate([q_pre, qs], 1)
+        k = np.concatenate([k_c, ks], 1)
+        v = np.concatenate([v_c, vs], 1)
+        out_p, lse_p = oracle.prefill(q, k, v, [0] * P + ar_suf, scale=0.7)
+        np.testing.assert_allclose(out_s, out_p[:, P:], atol=1e-13)
+        np.testing.assert_allclose(lse_s, lse_p[:, P:], atol=1e-13)
+
+
+def test_rows_subset_matches_full():
+    rng = np.random.default_rng(11)
+    B, S, Hq, d = 2, 19, 4, 8
+    ar = [0] * 9 + [1] * 4 + [1] + [0] * 5
+    seg = [0] * 9 + [1] * 4 + [2] * 6
+    q, k, v = _rand((B, S, Hq, d), rng), _rand((B, S, 1, d), rng), _rand((B, S, 1, d), rng)
+    out, lse = oracle.prefill(q, k, v, ar, seg)
+    rows = [(1, 18), (0, 0), (1, 10), (0, 14)]
+    o2, l2 = oracle.prefill(q, k, v, ar, seg, rows=rows)
+    for r, (b, i) in enumerate(rows):
+        np.testing.assert_allclose(o2[r], out[b, i], atol=1e-14)
+        np.testing.assert_allclose(l2[r], lse[b, i], atol=1e-14)
+
+
+# ------------------------------------------------------------------ counts
+
+
+def test_pair_counts():
+    vals = {r[0]: float(r[1]) for r in _load_rows("pair_counts.txt")}
+    assert counts.full_pairs(392 + 48 + 8 + 32) == vals["fused_480_scores"]
+    assert counts.full_pairs(32, 448) == vals["cross_32x448_scores"]
+    mmdit = 28 * counts.full_pairs(4096 + 154)
+    assert float(f"{mmdit:.0e}") == vals["mmdit_28_steps_about"]
+    assert counts.visible_pairs(oracle.prefill_mask(np.zeros(480))) == 230400
+    # parity unpinned: the page's "about 1.2e6" is only matched in order of magnitude
+    c = counts.control_step_pairs(816, 50, 10, suffix_keys=50)
+    assert 0.85 * vals["pi05_control_step_about"] < c < 1.15 * vals["pi05_control_step_about"]
+
+
+# ----------------------------------------------------------- planted mistakes
+
+
+def _pins_pass(mask_fn):
+    """Run the mask pins against a candidate mask builder; True if all hold."""
+    try:
+        M = mask_fn([0, 0, 0, 0, 0, 1, 1, 1], None)
+        for label, toks, bits in _load_rows("fast_mask_picture.txt"):
+            for t in map(int, toks.split(",")):
+                if not (M[t] == np.array([c == "1" for c in bits])).all():
+                    return False
+        ar = [0] * 6 + [1] * 4 + [1] + [0] * 4
+        seg = [0] * 6 + [1] * 4 + [2] * 5
+        M = mask_fn(ar, seg)
+        if not (M == np.array(brute.mask(ar, seg))).all():
+            return False
+        for S in range(1, 7):
+            for bits in itertools.product((0, 1), repeat=S):
+                if not (mask_fn(list(bits), None) == np.array(brute.mask(list(bits)))).all():
+                    return False
+        return True
+    except Exception:
+        return False
+
+
+def test_planted_mask_mistakes_are_caught():
+    def good(ar, seg):
+        return oracle.prefill_mask(ar, seg)[0]
+
+    def transposed(ar, seg):
+        return oracle.prefill_mask(ar, seg)[0].T
+
+    def strict(ar, seg):
+        cs = oracle.ar_cumsum(np.asarray(ar))
+        return cs[None, :] < cs[:, None]
+
+    def no_seg_rule(ar, seg):
+        return oracle.prefill_mask(ar, None)[0]
+
+    def seg_rule_reversed(ar, seg):
+        M = oracle.prefill_mask(ar, None)[0]
+        if seg is not None:
+            s = np.asarray(seg)
+            M &= ~((s[:, None] == FAST) & (s[None, :] == EXPERT))
+        return M
+
+    def exclusive_cumsum(ar, seg):
+        a = (np.asarray(ar) != 0).astype(int)
+        cs = np.cumsum(a) - a
+        return cs[None, :] <= cs[:, None]
+
+    assert _pins_pass(good)
+    for bad in (transposed, strict, no_seg_rule, seg_rule_reversed, exclusive_cumsum):
+        assert not _pins_pass(bad), bad.__name__
+
+
+def test_planted_value_mistakes_are_caught():
+    """Dropping the scale, swapping q/k roles or mis-grouping heads breaks the SDPA pin."""
+    rng = np.random.default_rng(12)
+    B, S, Hq, Hkv, d = 1, 12, 4, 2, 8
+    ar = [0] * 6 + [1] + [0] * 5
+    q, k, v = _rand((B, S, Hq, d), rng), _rand((B, S, Hkv, d), rng), _rand((B, S, Hkv, d), rng)
+    M = oracle.prefill_mask(ar, B=B)
+    tq, tk, tv = (torch.from_numpy(x).permute(0, 2, 1, 3) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk, tv, attn_mask=torch.from_numpy(M[0]), scale=0.5, enable_gqa=True
+    ).permute(0, 2, 1, 3).numpy()
+
+    good, _ = oracle.attention(q, k, v, M, 0.5)
+    assert np.abs(good - ref).max() < 1e-12
+    no_scale, _ = oracle.attention(q, k, v, M, 1.0)
+    assert np.abs(no_scale - ref).max() > 1e-3
+    # modulo head grouping instead of contiguous groups
+    q_regroup = q[:, :, [0, 2, 1, 3], :]
+    bad_group, _ = oracle.attention(q_regroup, k, v, M, 0.5)
+    assert np.abs(bad_group[:, :, [0, 2, 1, 3]] - ref).max() > 1e-3
+    # transposed mask
+    bad_t, _ = oracle.attention(q, k, v, np.swapaxes(M, 1, 2), 0.5)
+    assert np.abs(bad_t - ref).max() > 1e-3
