@@ -1,0 +1,189 @@
+/*
+ * pi_attn.h -- C ABI of libpiattn.so: the pi0 / pi0.5 joint (prefix-LM)
+ * attention on one NVIDIA B200 (sm_100a).
+ *
+ * What is computed (sources: page title, section):
+ *
+ *  - "π0.5 vs MM-DiT joint attention", "joint attention 只管算子,mask 才管权限":
+ *    each expert's q, k, v are concatenated along the token axis into one
+ *    shared KV pool and a single softmax runs over it.  The experts share the
+ *    head geometry: 8 query heads, 1 KV head, head_dim 256 (also "Pi0-FAST
+ *    模型架构", 6 关键超参数: num_heads 8, num_kv_heads 1, head_dim 256).
+ *  - same page, "π0.5:三段,两处看不到": key j is visible to query i iff
+ *    cumsum(ar_mask)[j] <= cumsum(ar_mask)[i]; pi0.5 additionally forbids
+ *    expert queries from reading FAST keys (last row of the permission table).
+ *  - "VLA 代码精读 - OpenPI & StarVLA", 1.2 (Prefix-Suffix 注意力掩码): ar_mask
+ *    False = shares attention with the preceding tokens, True = the preceding
+ *    tokens cannot see this token.
+ *  - same page, 1.6 Pi0.sample_actions: the prefix is run once and its K/V
+ *    kept; each of the 10 Euler steps runs only the suffix tokens, whose
+ *    queries see every cached prefix key plus the suffix keys allowed by the
+ *    cumsum rule over the suffix alone.  The cache is read, never appended.
+ *
+ *   out[b,i,h,:] = sum_j softmax_j( scale * <q[b,i,h,:], k[b,j,g(h),:]> | visible(i,j) ) v[b,j,g(h),:]
+ *   g(h) = h / (Hq / Hkv)
+ *
+ * Memory layout (all entry points): every tensor is a dense, contiguous,
+ * caller-owned DEVICE buffer in token-major order [B, S, H, d] (d innermost,
+ * then heads, then tokens, then batch).  ar_mask is uint8 (0 = False,
+ * nonzero = True); segment_ids is int32 (PI_SEG_*; any other value is treated
+ * as PI_SEG_OTHER).  Both are [S] rows, one per batch element at a distance of
+ * desc->mask_batch_stride elements (0 = one row shared by the whole batch).
+ *
+ * Ownership and threading: the library never allocates, frees or retains a
+ * caller buffer; all work is enqueued on the caller's stream and the calls
+ * return before it runs.  Buffers must stay valid until the stream reaches the
+ * work.  Calls on different streams may run concurrently; the only global
+ * state is the device status word read by pi_attn_read_status.
+ *
+ * Errors: every entry point returns PI_OK or a PI_ERR_* code.  Argument
+ * errors are detected on the host before anything is enqueued (nothing is
+ * launched).  PI_ERR_CUDA reports a failed launch (the CUDA error is left in
+ * the runtime's sticky/last-error state).  Device-side failures (a bounded
+ * wait that ran out) do not trap: the kernel records PI_ERR_TIMEOUT in the
+ * status word, abandons its tile and returns, and the host reads it with
+ * pi_attn_read_status.  No exception crosses this boundary.
+ */
+#ifndef PI_ATTN_H_
+#define PI_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (NULL = the legacy default stream), kept opaque here so that
+ * C callers need no CUDA headers. */
+typedef void* pi_stream_t;
+
+enum pi_dtype {
+  PI_BF16 = 0, /* bf16 in/out, fp32 accumulation (tcgen05 tensor cores)   */
+  PI_F32 = 1   /* fp32 in/out, fp32 FFMA arithmetic (CUDA cores)         */
+};
+
+enum pi_status {
+  PI_OK = 0,
+  PI_ERR_ARG = 1,         /* NULL pointer, bad shape, stride or size      */
+  PI_ERR_ALIGN = 2,       /* a pointer is not 16-byte aligned             */
+  PI_ERR_UNSUPPORTED = 3, /* dtype / head geometry this build lacks       */
+  PI_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed         */
+  PI_ERR_TIMEOUT = 5      /* a device-side bounded wait ran out           */
+};
+
+enum pi_segment {
+  PI_SEG_OTHER = 0,  /* prefix: image patches, text, discrete state      */
+  PI_SEG_FAST = 1,   /* FAST discrete action tokens                      */
+  PI_SEG_EXPERT = 2  /* the action expert's continuous chunk             */
+};
+
+typedef struct pi_attn_desc {
+  int32_t B;    /* batch size (B == 0 is a no-op)                            */
+  int32_t Sq;   /* query tokens: prefill = S; suffix = suffix tokens          */
+  int32_t P;    /* suffix mode: cached prefix tokens; prefill: must be 0      */
+  int32_t Hq;   /* query heads                                                */
+  int32_t Hkv;  /* key/value heads; Hq % Hkv == 0                             */
+  int32_t d;    /* head dimension                                             */
+  int32_t dtype;          /* enum pi_dtype                                    */
+  float softmax_scale;    /* multiplies q.k before the softmax (finite)       */
+  int64_t mask_batch_stride; /* elements between batch rows of ar_mask and
+                                segment_ids; 0 = shared by the batch, else >= Sq */
+} pi_attn_desc;
+
+/*
+ * Supported geometry in this build:
+ *   PI_BF16: Hkv == 1, d == 256, Hq in {1, 2, 4, 8, 16}; tokens Sq <= 16383
+ *            (the in-kernel block index is 14 bits), P < 2^31 / Hq.
+ *   PI_F32 : Hq % Hkv == 0, d in {32, 64, 128, 256}, Sq <= 16383.
+ * Anything else returns PI_ERR_UNSUPPORTED.  Sq == 0 or B == 0 is a no-op.
+ */
+
+/*
+ * pi_attn_prefill -- joint prefill over [prefix, suffix] tokens (mode 1).
+ * Source: "VLA 代码精读 - OpenPI & StarVLA", 1.5 Pi0.compute_loss (one forward
+ * over the concatenated tokens under make_attn_mask), with the mask rule of
+ * "π0.5 vs MM-DiT joint attention", π0.5:三段.
+ *
+ *   q    [B, S, Hq, d]     (S = desc->Sq, desc->P must be 0)
+ *   k, v [B, S, Hkv, d]
+ *   ar_mask     [B or 1, S] uint8            (required)
+ *   segment_ids [B or 1, S] int32 or NULL    (NULL: no expert<-FAST rule)
+ *   out  [B, S, Hq, d]  same dtype as q      (written)
+ *   lse  [B, S, Hq] fp32 or NULL             (natural-log log-sum-exp of the
+ *                                             scaled visible scores; written)
+ * Every query sees at least itself, so no row is empty.
+ */
+int pi_attn_prefill(const pi_attn_desc* desc, const void* q, const void* k, const void* v,
+                    const uint8_t* ar_mask, const int32_t* segment_ids, void* out, float* lse,
+                    pi_stream_t stream);
+
+/*
+ * pi_attn_suffix -- suffix-only pass against a prefix KV cache (mode 2), the
+ * call each Euler flow-matching step makes.
+ * Source: "VLA 代码精读 - OpenPI & StarVLA", 1.6 Pi0.sample_actions: the key
+ * mask is [every prefix key | make_attn_mask(suffix ar_mask)], the cache is
+ * not extended.
+ *
+ *   q_suf [B, Sq, Hq, d];  k_suf, v_suf [B, Sq, Hkv, d]
+ *   k_cache, v_cache [B, P, Hkv, d]  (read only; P = desc->P >= 0)
+ *   ar_mask_suf [B or 1, Sq] uint8
+ *   out [B, Sq, Hq, d]
+ *   workspace / ws_bytes: caller-provided device scratch of at least
+ *   pi_attn_suffix_workspace_bytes(desc) bytes (may be NULL when that is 0);
+ *   its contents need no initialisation and are garbage afterwards.  Calls
+ *   that may overlap on the GPU need distinct workspaces.
+ */
+int pi_attn_suffix(const pi_attn_desc* desc, const void* q_suf, const void* k_suf,
+                   const void* v_suf, const void* k_cache, const void* v_cache,
+                   const uint8_t* ar_mask_suf, void* out, void* workspace, size_t ws_bytes,
+                   pi_stream_t stream);
+
+/* Bytes of workspace pi_attn_suffix needs for this descriptor (0 if none);
+ * returns 0 for a descriptor that pi_attn_suffix would reject. */
+size_t pi_attn_suffix_workspace_bytes(const pi_attn_desc* desc);
+
+/*
+ * pi_attn_debug_mask -- writes the visibility matrix the kernels evaluate, as
+ * uint8 0/1, for bit-exact comparison with an explicitly built mask.
+ * Uses the same in-kernel predicate (cumsum of ar_mask, the expert<-FAST
+ * rule, and the suffix-pass prefix columns) as the attention kernels.
+ *   mode 0 (prefill): mask_out [B, Sq, Sq];      seg may be NULL
+ *   mode 1 (suffix) : mask_out [B, Sq, P + Sq];  seg must be NULL
+ * Only desc->B, Sq, P and mask_batch_stride are read.
+ */
+int pi_attn_debug_mask(const pi_attn_desc* desc, int mode, const uint8_t* ar_mask,
+                       const int32_t* segment_ids, uint8_t* mask_out, pi_stream_t stream);
+
+/*
+ * pi_attn_read_status -- synchronises `stream`, returns the device status word
+ * (PI_OK or the first PI_ERR_TIMEOUT recorded by any kernel since the last
+ * read) and clears it.  Returns PI_ERR_CUDA if the synchronisation fails.
+ */
+int pi_attn_read_status(pi_stream_t stream);
+
+/* Human-readable name of a pi_status code (static storage). */
+const char* pi_attn_status_string(int status);
+
+/*
+ * pi_attn_set_wait_limit -- bound, in SM clock cycles, on every device-side
+ * spin wait (mbarrier phase waits) in kernels launched after this call.
+ * 0 restores the default (2^31 cycles, about a second).  Returns the previous
+ * value.  Process-wide.
+ */
+uint64_t pi_attn_set_wait_limit(uint64_t cycles);
+
+/*
+ * pi_attn_selftest_wait -- launches one CTA that waits on an mbarrier that
+ * nothing ever arrives at, bounded by the current wait limit; the wait runs
+ * out and records PI_ERR_TIMEOUT in the status word.  Exercises the timeout
+ * path of the same bounded-wait routine the attention kernels use, without
+ * faulting or hanging the GPU.
+ */
+int pi_attn_selftest_wait(pi_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PI_ATTN_H_ */

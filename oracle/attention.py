@@ -59,7 +59,7 @@ def ar_cumsum(ar):
     return np.cumsum(ar != 0, axis=-1, dtype=np.int64)
 
 
-def prefill_mask(ar, seg=None, B=None):
+def prefill_mask(ar, seg=None, B=None, rows=None):
     """Explicit [B, S, S] boolean visibility matrix of the joint prefill.
 
     M[b, i, j] = cumsum(ar)[j] <= cumsum(ar)[i]            (the cumsum rule)
@@ -67,17 +67,20 @@ def prefill_mask(ar, seg=None, B=None):
                                                    (pi0.5's 'expert <- FAST' row)
 
     ``ar`` and ``seg`` are [S] (shared by the batch) or [B, S].  ``B`` sets the
-    batch when both are 1-D (default 1).
+    batch when both are 1-D (default 1).  ``rows`` (a list of query indices)
+    returns only those rows, [B, len(rows), S], for sequences too long to hold
+    the full matrix.
     """
     ar = np.asarray(ar)
     if B is None:
         B = ar.shape[0] if ar.ndim == 2 else 1
     ar = _as_batched(ar, B, "ar")
     cs = ar_cumsum(ar)                                   # [B, S]
-    M = cs[:, None, :] <= cs[:, :, None]                 # [B, i, j]
+    qi = np.arange(cs.shape[1]) if rows is None else np.asarray(rows)
+    M = cs[:, None, :] <= cs[:, qi, None]                # [B, i, j]
     if seg is not None:
         seg = _as_batched(seg, B, "seg")
-        forbid = (seg[:, :, None] == EXPERT) & (seg[:, None, :] == FAST)
+        forbid = (seg[:, qi, None] == EXPERT) & (seg[:, None, :] == FAST)
         M = M & ~forbid
     return M
 

@@ -1,0 +1,137 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching the GPU.
+
+Nothing here launches a kernel; each call below fails validation (or is a
+B == 0 no-op) before any CUDA runtime call is made.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+
+def _lib():
+    from vla_prefix_lm_b200 import binding, build
+    build.build()
+    return binding, binding.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "pi_attn.h")).read()
+    return sorted(set(re.findall(r"\b(pi_attn_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_two_calls():
+    names = _declared()
+    assert "pi_attn_prefill" in names and "pi_attn_suffix" in names
+
+
+def test_library_exports_every_declared_symbol():
+    binding, L = _lib()
+    for name in _declared():
+        assert hasattr(L, name), name
+    assert set(binding.EXPORTED) <= set(_declared())
+
+
+def _desc(binding, **kw):
+    d = dict(B=2, Sq=16, P=0, Hq=8, Hkv=1, d=256, dtype=binding.PI_BF16, softmax_scale=1.0,
+             mask_batch_stride=0)
+    d.update(kw)
+    return binding.PiAttnDesc(**d)
+
+
+FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
+FAKE_MIS = ctypes.c_void_p(0x10008)  # misaligned
+
+
+def _prefill(L, desc, q=FAKE, k=FAKE, v=FAKE, ar=FAKE, seg=None, out=FAKE, lse=None):
+    return L.pi_attn_prefill(ctypes.byref(desc) if desc is not None else None,
+                             q, k, v, ar, seg, out, lse, None)
+
+
+def test_prefill_argument_errors():
+    b, L = _lib()
+    assert _prefill(L, None) == b.PI_ERR_ARG
+    assert _prefill(L, _desc(b, Hq=0)) == b.PI_ERR_ARG
+    assert _prefill(L, _desc(b, P=3)) == b.PI_ERR_ARG          # prefill has no cache
+    assert _prefill(L, _desc(b, Hq=6, Hkv=4)) == b.PI_ERR_ARG
+    assert _prefill(L, _desc(b, softmax_scale=float("nan"))) == b.PI_ERR_ARG
+    assert _prefill(L, _desc(b, mask_batch_stride=5)) == b.PI_ERR_ARG
+    assert _prefill(L, _desc(b), q=None) == b.PI_ERR_ARG
+    assert _prefill(L, _desc(b), ar=None) == b.PI_ERR_ARG
+    assert _prefill(L, _desc(b), k=FAKE_MIS) == b.PI_ERR_ALIGN
+    assert _prefill(L, _desc(b), out=FAKE_MIS) == b.PI_ERR_ALIGN
+
+
+def test_prefill_unsupported_geometry():
+    b, L = _lib()
+    assert _prefill(L, _desc(b, d=128)) == b.PI_ERR_UNSUPPORTED
+    assert _prefill(L, _desc(b, Hkv=2)) == b.PI_ERR_UNSUPPORTED
+    assert _prefill(L, _desc(b, Hq=3, Hkv=1)) == b.PI_ERR_UNSUPPORTED
+    assert _prefill(L, _desc(b, dtype=7)) == b.PI_ERR_UNSUPPORTED
+    assert _prefill(L, _desc(b, Sq=16384)) == b.PI_ERR_UNSUPPORTED
+    assert _prefill(L, _desc(b, dtype=b.PI_F32, d=48)) == b.PI_ERR_UNSUPPORTED
+
+
+def test_empty_inputs_are_noops():
+    b, L = _lib()
+    assert _prefill(L, _desc(b, B=0), q=None, k=None, v=None, ar=None, out=None) == b.PI_OK
+    assert _prefill(L, _desc(b, Sq=0), q=None, k=None, v=None, ar=None, out=None) == b.PI_OK
+    d = _desc(b, Sq=0, P=10)
+    assert L.pi_attn_suffix(ctypes.byref(d), None, None, None, None, None, None, None, None, 0,
+                            None) == b.PI_OK
+
+
+def test_suffix_argument_errors():
+    b, L = _lib()
+    d = _desc(b, P=816, Sq=51)
+    args = [FAKE] * 7
+    rc = L.pi_attn_suffix(ctypes.byref(d), *args[:3], None, None, args[5], args[6], None, 0,
+                          None)
+    assert rc == b.PI_ERR_ARG                                   # P > 0 needs a cache
+    rc = L.pi_attn_suffix(ctypes.byref(d), *args[:3], FAKE_MIS, FAKE, FAKE, FAKE, None, 0, None)
+    assert rc == b.PI_ERR_ALIGN
+    d2 = _desc(b, P=-1)
+    rc = L.pi_attn_suffix(ctypes.byref(d2), *args, None, 0, None)
+    assert rc == b.PI_ERR_ARG
+
+
+def test_workspace_query_is_host_only():
+    b, L = _lib()
+    d = _desc(b, B=32, Sq=51, P=816)
+    n = L.pi_attn_suffix_workspace_bytes(ctypes.byref(d))
+    assert n >= 0
+    assert L.pi_attn_suffix_workspace_bytes(ctypes.byref(_desc(b, Hq=0))) == 0
+    assert L.pi_attn_suffix_workspace_bytes(None) == 0
+
+
+def test_status_strings_and_wait_limit():
+    b, L = _lib()
+    for code in range(6):
+        assert b.status_string(code).startswith("PI_")
+    prev = b.pi_attn_set_wait_limit(12345)
+    assert b.pi_attn_set_wait_limit(0) == 12345
+    assert b.pi_attn_set_wait_limit(prev) == 1 << 31
+
+
+def test_debug_mask_argument_errors():
+    b, L = _lib()
+    d = _desc(b)
+    assert L.pi_attn_debug_mask(ctypes.byref(d), 2, FAKE, None, FAKE, None) == b.PI_ERR_ARG
+    assert L.pi_attn_debug_mask(ctypes.byref(d), 0, None, None, FAKE, None) == b.PI_ERR_ARG
+    d1 = _desc(b, P=4)
+    assert L.pi_attn_debug_mask(ctypes.byref(d1), 1, FAKE, FAKE, FAKE, None) == b.PI_ERR_ARG
+
+
+def test_product_path_has_no_oracle_import():
+    """The package never imports the oracle (test infrastructure only)."""
+    pkg = os.path.join(ROOT, "vla_prefix_lm_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f

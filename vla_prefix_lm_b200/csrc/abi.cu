@@ -1,0 +1,281 @@
+// abi.cu -- the extern "C" entry points of libpiattn.so (declared in
+// include/pi_attn.h): argument validation, TMA tensor-map encoding, dispatch
+// to the kernels, and the device status word.
+//
+// Validation happens entirely on the host, before anything is enqueued: an
+// entry point that returns an error has launched nothing.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/pi_attn.h"
+#include "launch.h"
+#include "mask.cuh"
+
+namespace {
+
+using namespace piattn;
+
+constexpr unsigned long long kDefaultWaitLimit = 1ull << 31;
+std::atomic<unsigned long long> g_wait_limit{kDefaultWaitLimit};
+
+// The device status word (one per device the library runs on).
+__device__ int g_status;
+
+int* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  static std::mutex mu;
+  static int* ptrs[64] = {nullptr};
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+bool make_ctl(DevCtl* ctl) {
+  ctl->status = status_ptr();
+  ctl->wait_limit = g_wait_limit.load();
+  return ctl->status != nullptr;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// A [batch][rows][256] bf16 tensor viewed as 3-D (256, rows, batch), 128-byte
+// swizzle, box (64, box_rows, 1).  Rows past `rows` read as zero.
+bool encode_rows(CUtensorMap* map, const void* base, uint64_t rows, uint64_t batch,
+                 uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {256, rows, batch};
+  cuuint64_t strides[2] = {256 * 2, 256 * 2 * rows};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_desc(const pi_attn_desc* d, bool suffix) {
+  if (!d) return PI_ERR_ARG;
+  if (d->B < 0 || d->Sq < 0 || d->P < 0 || d->Hq <= 0 || d->Hkv <= 0 || d->d <= 0)
+    return PI_ERR_ARG;
+  if (!suffix && d->P != 0) return PI_ERR_ARG;
+  if (d->Hq % d->Hkv != 0) return PI_ERR_ARG;
+  if (!std::isfinite(d->softmax_scale)) return PI_ERR_ARG;
+  if (d->mask_batch_stride < 0 || (d->mask_batch_stride != 0 && d->mask_batch_stride < d->Sq))
+    return PI_ERR_ARG;
+  if (d->Sq > kMaxTokens) return PI_ERR_UNSUPPORTED;
+  if (d->dtype == PI_BF16) {
+    if (d->Hkv != 1 || d->d != 256) return PI_ERR_UNSUPPORTED;
+    if (!(d->Hq == 1 || d->Hq == 2 || d->Hq == 4 || d->Hq == 8 || d->Hq == 16))
+      return PI_ERR_UNSUPPORTED;
+    if ((long long)d->P * d->Hq >= (1ll << 31)) return PI_ERR_UNSUPPORTED;
+  } else if (d->dtype == PI_F32) {
+    if (!(d->d == 32 || d->d == 64 || d->d == 128 || d->d == 256)) return PI_ERR_UNSUPPORTED;
+  } else {
+    return PI_ERR_UNSUPPORTED;
+  }
+  return PI_OK;
+}
+
+int launched(cudaError_t e) { return e == cudaSuccess ? PI_OK : PI_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int pi_attn_prefill(const pi_attn_desc* d, const void* q, const void* k, const void* v,
+                    const uint8_t* ar_mask, const int32_t* segment_ids, void* out, float* lse,
+                    pi_stream_t stream) {
+  int rc = check_desc(d, false);
+  if (rc != PI_OK) return rc;
+  if (d->B == 0 || d->Sq == 0) return PI_OK;
+  if (!q || !k || !v || !ar_mask || !out) return PI_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return PI_ERR_ALIGN;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return PI_ERR_ALIGN;
+  if (segment_ids && (reinterpret_cast<uintptr_t>(segment_ids) & 3u)) return PI_ERR_ALIGN;
+  DevCtl ctl;
+  if (!make_ctl(&ctl)) return PI_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->dtype == PI_F32) {
+    SimtParams p{};
+    p.q = static_cast<const float*>(q);
+    p.k = static_cast<const float*>(k);
+    p.v = static_cast<const float*>(v);
+    p.ar = ar_mask;
+    p.seg = segment_ids;
+    p.mask_bs = d->mask_batch_stride;
+    p.out = static_cast<float*>(out);
+    p.lse = lse;
+    p.B = d->B; p.Sq = d->Sq; p.P = 0; p.Hq = d->Hq; p.Hkv = d->Hkv; p.d = d->d;
+    p.scale = d->softmax_scale;
+    return launched(launch_simt_f32(p, ctl, st));
+  }
+  TcParams p;
+  std::memset(&p, 0, sizeof(p));
+  const uint64_t rows = (uint64_t)d->Sq * d->Hq;
+  if (!encode_rows(&p.map_q, q, rows, d->B, 128) ||
+      !encode_rows(&p.map_k, k, d->Sq, d->B, 128) ||
+      !encode_rows(&p.map_v, v, d->Sq, d->B, 128) ||
+      !encode_rows(&p.map_o, out, rows, d->B, 32))
+    return PI_ERR_CUDA;
+  p.map_kc = p.map_k;
+  p.map_vc = p.map_v;
+  p.ar = ar_mask;
+  p.seg = segment_ids;
+  p.mask_bs = d->mask_batch_stride;
+  p.lse = lse;
+  p.ws = nullptr;
+  p.out_ptr = out;
+  p.B = d->B; p.Sq = d->Sq; p.P = 0; p.Hq = d->Hq;
+  p.n_splits = 1;
+  p.scale = d->softmax_scale;
+  p.scale_log2 = d->softmax_scale * 1.4426950408889634f;
+  return launched(launch_tc_attention(p, false, ctl, st));
+}
+
+size_t pi_attn_suffix_workspace_bytes(const pi_attn_desc* d) {
+  if (check_desc(d, true) != PI_OK) return 0;
+  if (d->dtype != PI_BF16 || d->B == 0 || d->Sq == 0) return 0;
+  return tc_suffix_workspace_bytes(d->B, d->Sq, d->P, d->Hq);
+}
+
+int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
+                   const void* v_suf, const void* k_cache, const void* v_cache,
+                   const uint8_t* ar_mask_suf, void* out, void* workspace, size_t ws_bytes,
+                   pi_stream_t stream) {
+  int rc = check_desc(d, true);
+  if (rc != PI_OK) return rc;
+  if (d->B == 0 || d->Sq == 0) return PI_OK;
+  if (!q_suf || !k_suf || !v_suf || !ar_mask_suf || !out) return PI_ERR_ARG;
+  if (d->P > 0 && (!k_cache || !v_cache)) return PI_ERR_ARG;
+  if (!aligned16(q_suf) || !aligned16(k_suf) || !aligned16(v_suf) || !aligned16(out) ||
+      (d->P > 0 && (!aligned16(k_cache) || !aligned16(v_cache))))
+    return PI_ERR_ALIGN;
+  DevCtl ctl;
+  if (!make_ctl(&ctl)) return PI_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d->dtype == PI_F32) {
+    SimtParams p{};
+    p.q = static_cast<const float*>(q_suf);
+    p.k = static_cast<const float*>(k_suf);
+    p.v = static_cast<const float*>(v_suf);
+    p.kc = static_cast<const float*>(k_cache);
+    p.vc = static_cast<const float*>(v_cache);
+    p.ar = ar_mask_suf;
+    p.seg = nullptr;
+    p.mask_bs = d->mask_batch_stride;
+    p.out = static_cast<float*>(out);
+    p.lse = nullptr;
+    p.B = d->B; p.Sq = d->Sq; p.P = d->P; p.Hq = d->Hq; p.Hkv = d->Hkv; p.d = d->d;
+    p.scale = d->softmax_scale;
+    return launched(launch_simt_f32(p, ctl, st));
+  }
+  const int splits = tc_suffix_splits(d->B, d->Sq, d->P, d->Hq);
+  const size_t need = tc_suffix_workspace_bytes(d->B, d->Sq, d->P, d->Hq);
+  if (need > 0) {
+    if (!workspace || ws_bytes < need) return PI_ERR_ARG;
+    if (!aligned16(workspace)) return PI_ERR_ALIGN;
+  }
+  TcParams p;
+  std::memset(&p, 0, sizeof(p));
+  const uint64_t rows = (uint64_t)d->Sq * d->Hq;
+  if (!encode_rows(&p.map_q, q_suf, rows, d->B, 128) ||
+      !encode_rows(&p.map_k, k_suf, d->Sq, d->B, 128) ||
+      !encode_rows(&p.map_v, v_suf, d->Sq, d->B, 128) ||
+      !encode_rows(&p.map_o, out, rows, d->B, 32))
+    return PI_ERR_CUDA;
+  if (d->P > 0) {
+    if (!encode_rows(&p.map_kc, k_cache, d->P, d->B, 128) ||
+        !encode_rows(&p.map_vc, v_cache, d->P, d->B, 128))
+      return PI_ERR_CUDA;
+  } else {
+    p.map_kc = p.map_k;
+    p.map_vc = p.map_v;
+  }
+  p.ar = ar_mask_suf;
+  p.seg = nullptr;
+  p.mask_bs = d->mask_batch_stride;
+  p.lse = nullptr;
+  p.ws = static_cast<float*>(workspace);
+  p.out_ptr = out;
+  p.B = d->B; p.Sq = d->Sq; p.P = d->P; p.Hq = d->Hq;
+  p.n_splits = splits;
+  p.scale = d->softmax_scale;
+  p.scale_log2 = d->softmax_scale * 1.4426950408889634f;
+  return launched(launch_tc_attention(p, true, ctl, st));
+}
+
+int pi_attn_debug_mask(const pi_attn_desc* d, int mode, const uint8_t* ar_mask,
+                       const int32_t* segment_ids, uint8_t* mask_out, pi_stream_t stream) {
+  if (!d || !ar_mask || !mask_out) return PI_ERR_ARG;
+  if (mode != 0 && mode != 1) return PI_ERR_ARG;
+  if (d->B < 0 || d->Sq < 0 || d->P < 0) return PI_ERR_ARG;
+  if (mode == 0 && d->P != 0) return PI_ERR_ARG;
+  if (mode == 1 && segment_ids) return PI_ERR_ARG;
+  if (d->mask_batch_stride < 0 || (d->mask_batch_stride != 0 && d->mask_batch_stride < d->Sq))
+    return PI_ERR_ARG;
+  if (d->Sq > kMaxTokens) return PI_ERR_UNSUPPORTED;
+  if (d->B == 0 || d->Sq == 0) return PI_OK;
+  return launched(launch_debug_mask(mode, d->B, d->Sq, d->P, ar_mask, segment_ids,
+                                    d->mask_batch_stride, mask_out,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int pi_attn_read_status(pi_stream_t stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PI_ERR_CUDA;
+  int* p = status_ptr();
+  if (!p) return PI_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return PI_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return PI_ERR_CUDA;
+  return v;
+}
+
+const char* pi_attn_status_string(int s) {
+  switch (s) {
+    case PI_OK: return "PI_OK";
+    case PI_ERR_ARG: return "PI_ERR_ARG: invalid argument";
+    case PI_ERR_ALIGN: return "PI_ERR_ALIGN: pointer not 16-byte aligned";
+    case PI_ERR_UNSUPPORTED: return "PI_ERR_UNSUPPORTED: dtype or geometry not supported";
+    case PI_ERR_CUDA: return "PI_ERR_CUDA: CUDA launch or runtime call failed";
+    case PI_ERR_TIMEOUT: return "PI_ERR_TIMEOUT: a device-side bounded wait ran out";
+    default: return "unknown pi_attn status";
+  }
+}
+
+uint64_t pi_attn_set_wait_limit(uint64_t cycles) {
+  return g_wait_limit.exchange(cycles ? cycles : kDefaultWaitLimit);
+}
+
+int pi_attn_selftest_wait(pi_stream_t stream) {
+  DevCtl ctl;
+  if (!make_ctl(&ctl)) return PI_ERR_CUDA;
+  return launched(launch_selftest_wait(ctl, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

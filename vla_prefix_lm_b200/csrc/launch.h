@@ -1,0 +1,64 @@
+// launch.h -- internal launchers behind the C ABI (host side, not exported).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace piattn {
+
+// Inputs of the fp32 SIMT path (both modes).  Prefill: k/v hold the S keys,
+// kc/vc are null and P = 0.  Suffix: k/v hold the Sq suffix keys and kc/vc the
+// P cached prefix keys.
+struct SimtParams {
+  const float* q;
+  const float* k;
+  const float* v;
+  const float* kc;
+  const float* vc;
+  const uint8_t* ar;
+  const int32_t* seg;
+  long long mask_bs;
+  float* out;
+  float* lse;
+  int B, Sq, P, Hq, Hkv, d;
+  float scale;
+};
+
+cudaError_t launch_simt_f32(const SimtParams& p, const DevCtl& ctl, cudaStream_t st);
+
+cudaError_t launch_debug_mask(int mode, int B, int Sq, int P, const uint8_t* ar,
+                              const int32_t* seg, long long mask_bs, uint8_t* out,
+                              cudaStream_t st);
+
+cudaError_t launch_selftest_wait(const DevCtl& ctl, cudaStream_t st);
+
+// bf16 tcgen05 path.  All tensors are [B, tokens, heads, 256] bf16; maps are
+// encoded by the ABI layer.
+struct TcParams {
+  CUtensorMap map_q;    // q rows    : dims (256, Sq*Hq, B), box (64, 128, 1)
+  CUtensorMap map_k;    // keys      : dims (256, Sk_src, B), box (64, 128, 1)
+  CUtensorMap map_v;
+  CUtensorMap map_kc;   // suffix mode: cached keys (dims (256, P, B)); unused in prefill
+  CUtensorMap map_vc;
+  CUtensorMap map_o;    // out rows  : dims (256, Sq*Hq, B), box (64, 32, 1)
+  const uint8_t* ar;
+  const int32_t* seg;
+  long long mask_bs;
+  float* lse;           // prefill only; may be null
+  float* ws;            // split-K partials (suffix mode); may be null
+  void* out_ptr;        // bf16 output rows (written by the combine kernel under split-K)
+  int B, Sq, P, Hq;
+  int n_splits;         // KV splits per query tile (1 = write final output)
+  float scale_log2;     // softmax_scale * log2(e)
+  float scale;          // softmax_scale
+};
+
+cudaError_t launch_tc_attention(const TcParams& p, bool suffix_mode, const DevCtl& ctl,
+                                cudaStream_t st);
+
+size_t tc_suffix_workspace_bytes(int B, int Sq, int P, int Hq);
+int tc_suffix_splits(int B, int Sq, int P, int Hq);
+
+}  // namespace piattn
