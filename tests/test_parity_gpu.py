@@ -35,7 +35,7 @@ def _err(got, want):
 
 
 def _prefill_case(B, ar, seg, Hq, d, dtype, seed, scale=1.0, lse=False, std=None):
-    S = len(ar)
+    S = np.asarray(ar).shape[-1]
     s = d ** -0.25 if std is None else std
     q, q64 = W.draw((B, S, Hq, d), seed * 4, d, dtype, s)
     k, k64 = W.draw((B, S, 1, d), seed * 4 + 1, d, dtype, s)

@@ -575,19 +575,24 @@ cudaError_t launch_tc_attention(const TcParams& p, bool suffix_mode, const DevCt
   const int n_qtiles = (rows + kBM - 1) / kBM;
   dim3 grid(n_qtiles * p.n_splits, p.B);
   const size_t smem = smem_bytes(p.Sq);
-  cudaError_t e;
+  // The opt-in shared-memory size is raised once per process to the largest
+  // this kernel can ask for, so later launches (and stream captures) make no
+  // attribute calls.
+  static const cudaError_t attr_err = [] {
+    const int most = (int)smem_bytes(kMaxTokens);
+    cudaError_t a = cudaFuncSetAttribute(tc_attention_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+    cudaError_t b = cudaFuncSetAttribute(tc_attention_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+    return a != cudaSuccess ? a : b;
+  }();
+  if (attr_err != cudaSuccess) return attr_err;
   if (suffix_mode) {
-    e = cudaFuncSetAttribute(tc_attention_kernel<true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     tc_attention_kernel<true><<<grid, kThreads, smem, st>>>(p, ctl);
   } else {
-    e = cudaFuncSetAttribute(tc_attention_kernel<false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     tc_attention_kernel<false><<<grid, kThreads, smem, st>>>(p, ctl);
   }
-  e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || p.n_splits <= 1) return e;
   const long long n_rows = (long long)p.B * rows;
   // The combine writes the bf16 output rows directly (same [B, Sq, Hq, 256] layout).
