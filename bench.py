@@ -210,8 +210,11 @@ def run_ours(args, rank, ws, local):
         return graphs[n]
 
     plan = [chunk] * (args.steps // chunk) + ([args.steps % chunk] if args.steps % chunk else [])
-    for n in set(plan):
-        graph_for(n).replay()
+    # CUDAGraph.replay() launches on torch's current stream: make it `stream`,
+    # the stream the timing events are recorded on.
+    with torch.cuda.stream(stream):
+        for n in set(plan):
+            graph_for(n).replay()
     torch.cuda.synchronize()
 
     sampler = ClockSampler(gpu_id(dev)) if rank == 0 else None
@@ -220,10 +223,11 @@ def run_ours(args, rank, ws, local):
     dist.barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
-    e0.record(stream)
-    for n in plan:
-        graph_for(n).replay()
-    e1.record(stream)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for n in plan:
+            graph_for(n).replay()
+        e1.record(stream)
     torch.cuda.synchronize()
     t_wall1 = time.time()
     dist.barrier()
@@ -356,15 +360,17 @@ def suffix_control(args, dev, stream, rank):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         ctrl()
-    g.replay()
+    with torch.cuda.stream(stream):
+        g.replay()
     torch.cuda.synchronize()
     reps = max(5, min(200, args.steps // 10))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
-    e0.record(stream)
-    for _ in range(reps):
-        g.replay()
-    e1.record(stream)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
     torch.cuda.synchronize()
     us_ctrl = dist.max_over_ranks(e0.elapsed_time(e1) * 1e3 / reps)
 
@@ -378,9 +384,9 @@ def suffix_control(args, dev, stream, rank):
     for _ in range(20):
         with torch.cuda.stream(stream):
             flush.fill_(1.0)
-        e0.record(stream)
-        g1.replay()
-        e1.record(stream)
+            e0.record(stream)
+            g1.replay()
+            e1.record(stream)
         torch.cuda.synchronize()
         cold.append(e0.elapsed_time(e1) * 1e3)
     us_cold = dist.max_over_ranks(float(np.median(cold)))

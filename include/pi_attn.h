@@ -86,7 +86,7 @@ typedef struct pi_attn_desc {
   int32_t Hkv;  /* key/value heads; Hq % Hkv == 0                             */
   int32_t d;    /* head dimension                                             */
   int32_t dtype;          /* enum pi_dtype                                    */
-  float softmax_scale;    /* multiplies q.k before the softmax (finite)       */
+  float softmax_scale;    /* multiplies q.k before the softmax (finite, > 0)  */
   int64_t mask_batch_stride; /* elements between batch rows of ar_mask and
                                 segment_ids; 0 = shared by the batch, else >= Sq */
 } pi_attn_desc;

@@ -60,6 +60,8 @@ def test_prefill_argument_errors():
     assert _prefill(L, _desc(b, P=3)) == b.PI_ERR_ARG          # prefill has no cache
     assert _prefill(L, _desc(b, Hq=6, Hkv=4)) == b.PI_ERR_ARG
     assert _prefill(L, _desc(b, softmax_scale=float("nan"))) == b.PI_ERR_ARG
+    assert _prefill(L, _desc(b, softmax_scale=0.0)) == b.PI_ERR_ARG
+    assert _prefill(L, _desc(b, softmax_scale=-1.0)) == b.PI_ERR_ARG
     assert _prefill(L, _desc(b, mask_batch_stride=5)) == b.PI_ERR_ARG
     assert _prefill(L, _desc(b), q=None) == b.PI_ERR_ARG
     assert _prefill(L, _desc(b), ar=None) == b.PI_ERR_ARG

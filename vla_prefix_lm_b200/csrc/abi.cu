@@ -59,17 +59,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// A [batch][rows][256] bf16 tensor viewed as 3-D (256, rows, batch), 128-byte
-// swizzle, box (64, box_rows, 1).  Rows past `rows` read as zero.
+// A [batch][rows][256] bf16 tensor viewed as 4-D (64, rows, 4, batch): the
+// row stride is 512 B and dimension 2 walks the four 64-column blocks of a
+// row (stride 128 B), so one box (64, box_rows, 4, 1) lands in shared memory
+// as 4 blocks of [box_rows x 64] with the 128-byte swizzle -- the operand
+// layout of the tensor-core kernel.  Rows past `rows` read as zero and are
+// clipped on stores.
 bool encode_rows(CUtensorMap* map, const void* base, uint64_t rows, uint64_t batch,
                  uint32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[3] = {256, rows, batch};
-  cuuint64_t strides[2] = {256 * 2, 256 * 2 * rows};
-  cuuint32_t box[3] = {64, box_rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+  cuuint64_t dims[4] = {64, rows, 4, batch};
+  cuuint64_t strides[3] = {256 * 2, 64 * 2, 256 * 2 * rows};
+  cuuint32_t box[4] = {64, box_rows, 4, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -83,7 +87,7 @@ int check_desc(const pi_attn_desc* d, bool suffix) {
     return PI_ERR_ARG;
   if (!suffix && d->P != 0) return PI_ERR_ARG;
   if (d->Hq % d->Hkv != 0) return PI_ERR_ARG;
-  if (!std::isfinite(d->softmax_scale)) return PI_ERR_ARG;
+  if (!std::isfinite(d->softmax_scale) || !(d->softmax_scale > 0.f)) return PI_ERR_ARG;
   if (d->mask_batch_stride < 0 || (d->mask_batch_stride != 0 && d->mask_batch_stride < d->Sq))
     return PI_ERR_ARG;
   if (d->Sq > kMaxTokens) return PI_ERR_UNSUPPORTED;
@@ -137,8 +141,8 @@ int pi_attn_prefill(const pi_attn_desc* d, const void* q, const void* k, const v
   std::memset(&p, 0, sizeof(p));
   const uint64_t rows = (uint64_t)d->Sq * d->Hq;
   if (!encode_rows(&p.map_q, q, rows, d->B, 128) ||
-      !encode_rows(&p.map_k, k, d->Sq, d->B, 128) ||
-      !encode_rows(&p.map_v, v, d->Sq, d->B, 128) ||
+      !encode_rows(&p.map_k, k, d->Sq, d->B, 64) ||
+      !encode_rows(&p.map_v, v, d->Sq, d->B, 64) ||
       !encode_rows(&p.map_o, out, rows, d->B, 32))
     return PI_ERR_CUDA;
   p.map_kc = p.map_k;
@@ -203,13 +207,13 @@ int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
   std::memset(&p, 0, sizeof(p));
   const uint64_t rows = (uint64_t)d->Sq * d->Hq;
   if (!encode_rows(&p.map_q, q_suf, rows, d->B, 128) ||
-      !encode_rows(&p.map_k, k_suf, d->Sq, d->B, 128) ||
-      !encode_rows(&p.map_v, v_suf, d->Sq, d->B, 128) ||
+      !encode_rows(&p.map_k, k_suf, d->Sq, d->B, 64) ||
+      !encode_rows(&p.map_v, v_suf, d->Sq, d->B, 64) ||
       !encode_rows(&p.map_o, out, rows, d->B, 32))
     return PI_ERR_CUDA;
   if (d->P > 0) {
-    if (!encode_rows(&p.map_kc, k_cache, d->P, d->B, 128) ||
-        !encode_rows(&p.map_vc, v_cache, d->P, d->B, 128))
+    if (!encode_rows(&p.map_kc, k_cache, d->P, d->B, 64) ||
+        !encode_rows(&p.map_vc, v_cache, d->P, d->B, 64))
       return PI_ERR_CUDA;
   } else {
     p.map_kc = p.map_k;

@@ -37,12 +37,13 @@ cudaError_t launch_selftest_wait(const DevCtl& ctl, cudaStream_t st);
 // bf16 tcgen05 path.  All tensors are [B, tokens, heads, 256] bf16; maps are
 // encoded by the ABI layer.
 struct TcParams {
-  CUtensorMap map_q;    // q rows    : dims (256, Sq*Hq, B), box (64, 128, 1)
-  CUtensorMap map_k;    // keys      : dims (256, Sk_src, B), box (64, 128, 1)
+  // 4-D views (64, rows, 4 column blocks, B) of [B, rows, 256] bf16 tensors
+  CUtensorMap map_q;    // q rows (Sq*Hq per batch), box (64, 128, 4, 1)
+  CUtensorMap map_k;    // keys (prefill: S; suffix: Sq), box (64, 64, 4, 1)
   CUtensorMap map_v;
-  CUtensorMap map_kc;   // suffix mode: cached keys (dims (256, P, B)); unused in prefill
+  CUtensorMap map_kc;   // suffix mode: cached keys (P per batch); unused in prefill
   CUtensorMap map_vc;
-  CUtensorMap map_o;    // out rows  : dims (256, Sq*Hq, B), box (64, 32, 1)
+  CUtensorMap map_o;    // out rows, box (64, 32, 4, 1)
   const uint8_t* ar;
   const int32_t* seg;
   long long mask_bs;

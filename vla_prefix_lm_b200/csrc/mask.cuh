@@ -73,4 +73,102 @@ __device__ void build_codes(const uint8_t* __restrict__ ar, const int32_t* __res
   }
 }
 
+// Same result as build_codes, for the tensor-core kernel.  Each thread owns
+// 32 consecutive tokens per round: their ar_mask bytes (and segment ids) are
+// all loaded up front -- 16-byte vectors when aligned -- and reduced to
+// 32-bit masks; one shuffle scan across the warp and a short scan over the
+// kThreads/32 warp totals give each thread its starting block index.  Codes
+// past S up to S_pad (a multiple of 32) are 0xFFFF.  `scratch` is shared
+// memory for kThreads/32 ints.  Every thread of the block must call it; it
+// ends with a block barrier.
+__device__ __forceinline__ uint32_t nonzero_byte_bits(uint32_t w) {
+  return ((w & 0xFFu) ? 1u : 0u) | ((w & 0xFF00u) ? 2u : 0u) | ((w & 0xFF0000u) ? 4u : 0u) |
+         ((w & 0xFF000000u) ? 8u : 0u);
+}
+
+template <int kThreads>
+__device__ void build_codes_x32(const uint8_t* __restrict__ ar, const int32_t* __restrict__ seg,
+                                int S, int S_pad, uint16_t* codes, int* scratch) {
+  constexpr int kWarps = kThreads / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int carry = 0;
+  for (int base = 0; base < S_pad; base += kThreads * 32) {
+    const int t0 = base + (int)threadIdx.x * 32;
+    uint32_t bits = 0, fast = 0, expert = 0;
+    if (t0 + 32 <= S && (reinterpret_cast<uintptr_t>(ar + t0) & 15u) == 0) {
+      const uint4 a = *reinterpret_cast<const uint4*>(ar + t0);
+      const uint4 c = *reinterpret_cast<const uint4*>(ar + t0 + 16);
+      bits = nonzero_byte_bits(a.x) | (nonzero_byte_bits(a.y) << 4) |
+             (nonzero_byte_bits(a.z) << 8) | (nonzero_byte_bits(a.w) << 12) |
+             (nonzero_byte_bits(c.x) << 16) | (nonzero_byte_bits(c.y) << 20) |
+             (nonzero_byte_bits(c.z) << 24) | (nonzero_byte_bits(c.w) << 28);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (t0 + i < S && ar[t0 + i] != 0) bits |= 1u << i;
+    }
+    if (seg != nullptr) {
+      if (t0 + 32 <= S && (reinterpret_cast<uintptr_t>(seg + t0) & 15u) == 0) {
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const int4 v = reinterpret_cast<const int4*>(seg + t0)[g];
+          const int sv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            fast |= (sv[h] == kSegFast ? 1u : 0u) << (4 * g + h);
+            expert |= (sv[h] == kSegExpert ? 1u : 0u) << (4 * g + h);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int sv = t0 + i < S ? seg[t0 + i] : 0;
+          fast |= (sv == kSegFast ? 1u : 0u) << i;
+          expert |= (sv == kSegExpert ? 1u : 0u) << i;
+        }
+      }
+    }
+    const int cnt = __popc(bits);
+    int x = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int v = scratch[w];
+      before += (w < warp) ? v : 0;
+      total += v;
+    }
+    const int excl = carry + before + x - cnt;  // tokens before t0 that are True
+    if (t0 < S_pad) {
+      uint32_t packed[16];
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        uint32_t c2[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int k = i + h;
+          const uint32_t upto = k == 31 ? 0xFFFFFFFFu : ((2u << k) - 1u);
+          const uint32_t cs = (uint32_t)excl + (uint32_t)__popc(bits & upto);
+          c2[h] = t0 + k < S
+                      ? ((cs << 2) | (((expert >> k) & 1u) << 1) | ((fast >> k) & 1u))
+                      : 0xFFFFu;
+        }
+        packed[i / 2] = c2[0] | (c2[1] << 16);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(codes + t0);   // t0 is a multiple of 32
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+        dst[g] = make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+    }
+    carry += total;
+    __syncthreads();
+  }
+}
+
 }  // namespace piattn
