@@ -63,15 +63,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // row stride is 512 B and dimension 2 walks the four 64-column blocks of a
 // row (stride 128 B), so one box (64, box_rows, 4, 1) lands in shared memory
 // as 4 blocks of [box_rows x 64] with the 128-byte swizzle -- the operand
-// layout of the tensor-core kernel.  Rows past `rows` read as zero and are
+// layout of the tensor-core kernels.  A box of 2 blocks brings half the
+// columns (the CTA-pair kernel's V halves).  Rows past `rows` read as zero and are
 // clipped on stores.
 bool encode_rows(CUtensorMap* map, const void* base, uint64_t rows, uint64_t batch,
-                 uint32_t box_rows) {
+                 uint32_t box_rows, uint32_t box_blocks = 4) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {64, rows, 4, batch};
   cuuint64_t strides[3] = {256 * 2, 64 * 2, 256 * 2 * rows};
-  cuuint32_t box[4] = {64, box_rows, 4, 1};
+  cuuint32_t box[4] = {64, box_rows, box_blocks, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -143,10 +144,12 @@ int pi_attn_prefill(const pi_attn_desc* d, const void* q, const void* k, const v
   if (!encode_rows(&p.map_q, q, rows, d->B, 128) ||
       !encode_rows(&p.map_k, k, d->Sq, d->B, 64) ||
       !encode_rows(&p.map_v, v, d->Sq, d->B, 64) ||
+      !encode_rows(&p.map_vh, v, d->Sq, d->B, 128, 2) ||
       !encode_rows(&p.map_o, out, rows, d->B, 32))
     return PI_ERR_CUDA;
   p.map_kc = p.map_k;
   p.map_vc = p.map_v;
+  p.map_vch = p.map_vh;
   p.ar = ar_mask;
   p.seg = segment_ids;
   p.mask_bs = d->mask_batch_stride;
@@ -157,7 +160,7 @@ int pi_attn_prefill(const pi_attn_desc* d, const void* q, const void* k, const v
   p.n_splits = 1;
   p.scale = d->softmax_scale;
   p.scale_log2 = d->softmax_scale * 1.4426950408889634f;
-  return launched(launch_tc_attention(p, false, ctl, st));
+  return launched(launch_tc_pair(p, false, ctl, st));
 }
 
 size_t pi_attn_suffix_workspace_bytes(const pi_attn_desc* d) {
@@ -209,15 +212,18 @@ int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
   if (!encode_rows(&p.map_q, q_suf, rows, d->B, 128) ||
       !encode_rows(&p.map_k, k_suf, d->Sq, d->B, 64) ||
       !encode_rows(&p.map_v, v_suf, d->Sq, d->B, 64) ||
+      !encode_rows(&p.map_vh, v_suf, d->Sq, d->B, 128, 2) ||
       !encode_rows(&p.map_o, out, rows, d->B, 32))
     return PI_ERR_CUDA;
   if (d->P > 0) {
     if (!encode_rows(&p.map_kc, k_cache, d->P, d->B, 64) ||
-        !encode_rows(&p.map_vc, v_cache, d->P, d->B, 64))
+        !encode_rows(&p.map_vc, v_cache, d->P, d->B, 64) ||
+        !encode_rows(&p.map_vch, v_cache, d->P, d->B, 128, 2))
       return PI_ERR_CUDA;
   } else {
     p.map_kc = p.map_k;
     p.map_vc = p.map_v;
+    p.map_vch = p.map_vh;
   }
   p.ar = ar_mask_suf;
   p.seg = nullptr;
@@ -229,7 +235,8 @@ int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
   p.n_splits = splits;
   p.scale = d->softmax_scale;
   p.scale_log2 = d->softmax_scale * 1.4426950408889634f;
-  return launched(launch_tc_attention(p, true, ctl, st));
+  if (splits > 1) return launched(launch_tc_attention(p, true, ctl, st));
+  return launched(launch_tc_pair(p, true, ctl, st));
 }
 
 int pi_attn_debug_mask(const pi_attn_desc* d, int mode, const uint8_t* ar_mask,

@@ -44,6 +44,8 @@ struct TcParams {
   CUtensorMap map_kc;   // suffix mode: cached keys (P per batch); unused in prefill
   CUtensorMap map_vc;
   CUtensorMap map_o;    // out rows, box (64, 32, 4, 1)
+  CUtensorMap map_vh;   // values, half width: box (64, 128, 2, 1) (CTA-pair kernel)
+  CUtensorMap map_vch;  // cached values, half width
   const uint8_t* ar;
   const int32_t* seg;
   long long mask_bs;
@@ -58,6 +60,10 @@ struct TcParams {
 
 cudaError_t launch_tc_attention(const TcParams& p, bool suffix_mode, const DevCtl& ctl,
                                 cudaStream_t st);
+
+// CTA-pair (2-SM) form: 256 query rows per cluster of 2, 128-key tiles.
+cudaError_t launch_tc_pair(const TcParams& p, bool suffix_mode, const DevCtl& ctl,
+                           cudaStream_t st);
 
 size_t tc_suffix_workspace_bytes(int B, int Sq, int P, int Hq);
 int tc_suffix_splits(int B, int Sq, int P, int Hq);
