@@ -48,7 +48,7 @@ L2_BYTES = 126 * 2**20
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the
 # kernel sources whose digest is recorded beside it.
 TRAFFIC = {"bytes": None, "src_sha": None}
-KERNEL_SOURCES = ("vla_prefix_lm_b200/csrc/tc_attention.cu", "vla_prefix_lm_b200/csrc/common.cuh",
+KERNEL_SOURCES = ("vla_prefix_lm_b200/csrc/tc_pair.cu", "vla_prefix_lm_b200/csrc/common.cuh",
                   "vla_prefix_lm_b200/csrc/mask.cuh")
 
 
@@ -309,7 +309,7 @@ def run_ours(args, rank, ws, local):
         "gb_per_s_algorithmic": bytes_step / (ms_step / 1e3) / 1e9,
         "roofline": {
             "bound": "tensor",
-            "kernel": "tc_attention_kernel<prefill>",
+            "kernel": "tc_pair_kernel<prefill>",
             "achieved": achieved_tflops,
             "peak": P["bf16_tflops"],
             "unit": "TFLOP/s",

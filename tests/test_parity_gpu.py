@@ -224,6 +224,28 @@ def test_bf16_suffix_edge_sizes(P, Sq):
     assert _err(out, ref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("B,P", [(1, 816), (2, 816), (4, 2000), (1, 3000)])
+def test_bf16_suffix_split_k(B, P):
+    """Small-batch suffix passes split the key tiles over several CTA pairs
+    (caller-provided workspace, partials merged by the combine kernel)."""
+    Sq, Hq, d = 51, 8, 256
+    ar = W.pi0_suffix_ar(Sq - 1)
+    qs, q64 = W.draw((B, Sq, Hq, d), 61, d, "bf16")
+    ks, k64 = W.draw((B, Sq, 1, d), 62, d, "bf16")
+    vs, v64 = W.draw((B, Sq, 1, d), 63, d, "bf16")
+    kc, kc64 = W.draw((B, P, 1, d), 64, d, "bf16")
+    vc, vc64 = W.draw((B, P, 1, d), 65, d, "bf16")
+    args = (qs.cuda(), ks.cuda(), vs.cuda(), kc.cuda(), vc.cuda(), torch.from_numpy(ar).cuda())
+    need = _b().pi_attn_suffix_workspace_bytes(args[0], args[1], args[3], args[5])
+    assert need > 0
+    ws = torch.full((need,), 0xAB, dtype=torch.uint8, device="cuda")  # garbage in: no init needed
+    out = _b().pi_attn_suffix(*args, workspace=ws)
+    ref, _ = oracle.suffix(q64, k64, v64, kc64, vc64, ar)
+    assert _err(out, ref) <= TOL_BF16
+    with pytest.raises(Exception):
+        _b().pi_attn_suffix(*args, workspace=ws[: need - 16])
+
+
 def test_suffix_equals_prefill_suffix_rows_on_gpu():
     """Suffix pass == rows [P:] of a joint prefill over [prefix, suffix] (any prefix q)."""
     B, P, Sq, Hq, d = 2, 260, 51, 8, 256

@@ -143,12 +143,10 @@ int pi_attn_prefill(const pi_attn_desc* d, const void* q, const void* k, const v
   const uint64_t rows = (uint64_t)d->Sq * d->Hq;
   if (!encode_rows(&p.map_q, q, rows, d->B, 128) ||
       !encode_rows(&p.map_k, k, d->Sq, d->B, 64) ||
-      !encode_rows(&p.map_v, v, d->Sq, d->B, 64) ||
       !encode_rows(&p.map_vh, v, d->Sq, d->B, 128, 2) ||
       !encode_rows(&p.map_o, out, rows, d->B, 32))
     return PI_ERR_CUDA;
   p.map_kc = p.map_k;
-  p.map_vc = p.map_v;
   p.map_vch = p.map_vh;
   p.ar = ar_mask;
   p.seg = segment_ids;
@@ -211,18 +209,15 @@ int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
   const uint64_t rows = (uint64_t)d->Sq * d->Hq;
   if (!encode_rows(&p.map_q, q_suf, rows, d->B, 128) ||
       !encode_rows(&p.map_k, k_suf, d->Sq, d->B, 64) ||
-      !encode_rows(&p.map_v, v_suf, d->Sq, d->B, 64) ||
       !encode_rows(&p.map_vh, v_suf, d->Sq, d->B, 128, 2) ||
       !encode_rows(&p.map_o, out, rows, d->B, 32))
     return PI_ERR_CUDA;
   if (d->P > 0) {
     if (!encode_rows(&p.map_kc, k_cache, d->P, d->B, 64) ||
-        !encode_rows(&p.map_vc, v_cache, d->P, d->B, 64) ||
         !encode_rows(&p.map_vch, v_cache, d->P, d->B, 128, 2))
       return PI_ERR_CUDA;
   } else {
     p.map_kc = p.map_k;
-    p.map_vc = p.map_v;
     p.map_vch = p.map_vh;
   }
   p.ar = ar_mask_suf;
@@ -235,7 +230,6 @@ int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
   p.n_splits = splits;
   p.scale = d->softmax_scale;
   p.scale_log2 = d->softmax_scale * 1.4426950408889634f;
-  if (splits > 1) return launched(launch_tc_attention(p, true, ctl, st));
   return launched(launch_tc_pair(p, true, ctl, st));
 }
 

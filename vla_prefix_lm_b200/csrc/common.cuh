@@ -266,10 +266,13 @@ __device__ __forceinline__ void cluster_sync() {
                ::: "memory");
 }
 
-// Arrive on an mbarrier given by a shared::cluster address (possibly the peer's).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
+// Arrive on an mbarrier given by a shared::cluster address (possibly the
+// peer CTA's), with the default release semantics.  A cluster-scope release
+// here costs ~1000 cycles per arrival; the data this signal publishes (TMEM
+// written by tcgen05.st) is ordered by tcgen05.wait::st and
+// tcgen05.fence::before_thread_sync, not by this arrive.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // 4-D tiled load into this CTA's shared memory whose completion is counted on
@@ -357,6 +360,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
          | ((b_mn ? 1u : 0u) << 16)      // B major
          | ((uint32_t)(N >> 3) << 17)    // N / 8
          | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// Two non-negative finite floats to bf16x2, rounding half away from zero, on
+// the integer pipes (the conversion unit is busy with exp2 in the softmax).
+__device__ __forceinline__ uint32_t pack_bf16x2_rna(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo) + 0x8000u;
+  const uint32_t b = __float_as_uint(hi) + 0x8000u;
+  return __byte_perm(a, b, 0x7632);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -39,13 +39,11 @@ cudaError_t launch_selftest_wait(const DevCtl& ctl, cudaStream_t st);
 struct TcParams {
   // 4-D views (64, rows, 4 column blocks, B) of [B, rows, 256] bf16 tensors
   CUtensorMap map_q;    // q rows (Sq*Hq per batch), box (64, 128, 4, 1)
-  CUtensorMap map_k;    // keys (prefill: S; suffix: Sq), box (64, 64, 4, 1)
-  CUtensorMap map_v;
+  CUtensorMap map_k;    // keys (prefill: S; suffix: Sq), 64 keys x 256: box (64, 64, 4, 1)
   CUtensorMap map_kc;   // suffix mode: cached keys (P per batch); unused in prefill
-  CUtensorMap map_vc;
   CUtensorMap map_o;    // out rows, box (64, 32, 4, 1)
-  CUtensorMap map_vh;   // values, half width: box (64, 128, 2, 1) (CTA-pair kernel)
-  CUtensorMap map_vch;  // cached values, half width
+  CUtensorMap map_vh;   // values, 128 keys x 128 columns: box (64, 128, 2, 1)
+  CUtensorMap map_vch;  // cached values, same box
   const uint8_t* ar;
   const int32_t* seg;
   long long mask_bs;
@@ -58,10 +56,9 @@ struct TcParams {
   float scale;          // softmax_scale
 };
 
-cudaError_t launch_tc_attention(const TcParams& p, bool suffix_mode, const DevCtl& ctl,
-                                cudaStream_t st);
-
-// CTA-pair (2-SM) form: 256 query rows per cluster of 2, 128-key tiles.
+// CTA-pair (2-SM) form: 256 query rows per cluster of 2, 128-key tiles.  With
+// p.n_splits > 1 the key tiles are split over that many pairs per query tile,
+// partials go to p.ws and a combine kernel writes the output.
 cudaError_t launch_tc_pair(const TcParams& p, bool suffix_mode, const DevCtl& ctl,
                            cudaStream_t st);
 

@@ -86,49 +86,79 @@ __device__ __forceinline__ uint32_t nonzero_byte_bits(uint32_t w) {
          ((w & 0xFF000000u) ? 8u : 0u);
 }
 
+// The ar_mask bits and segment flags of 32 consecutive tokens starting at t0
+// (16-byte vector loads when aligned).  Tokens at or past S read as False / 0.
+struct Flags32 {
+  uint32_t bits, fast, expert;
+};
+
+__device__ __forceinline__ Flags32 load_flags32(const uint8_t* __restrict__ ar,
+                                                const int32_t* __restrict__ seg, int S, int t0) {
+  Flags32 f{0u, 0u, 0u};
+  if (t0 >= S) return f;
+  if (t0 + 32 <= S && (reinterpret_cast<uintptr_t>(ar + t0) & 15u) == 0) {
+    const uint4 a = *reinterpret_cast<const uint4*>(ar + t0);
+    const uint4 c = *reinterpret_cast<const uint4*>(ar + t0 + 16);
+    f.bits = nonzero_byte_bits(a.x) | (nonzero_byte_bits(a.y) << 4) |
+             (nonzero_byte_bits(a.z) << 8) | (nonzero_byte_bits(a.w) << 12) |
+             (nonzero_byte_bits(c.x) << 16) | (nonzero_byte_bits(c.y) << 20) |
+             (nonzero_byte_bits(c.z) << 24) | (nonzero_byte_bits(c.w) << 28);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (t0 + i < S && ar[t0 + i] != 0) f.bits |= 1u << i;
+  }
+  if (seg != nullptr) {
+    if (t0 + 32 <= S && (reinterpret_cast<uintptr_t>(seg + t0) & 15u) == 0) {
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const int4 v = reinterpret_cast<const int4*>(seg + t0)[g];
+        const int sv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          f.fast |= (sv[h] == kSegFast ? 1u : 0u) << (4 * g + h);
+          f.expert |= (sv[h] == kSegExpert ? 1u : 0u) << (4 * g + h);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int sv = t0 + i < S ? seg[t0 + i] : 0;
+        f.fast |= (sv == kSegFast ? 1u : 0u) << i;
+        f.expert |= (sv == kSegExpert ? 1u : 0u) << i;
+      }
+    }
+  }
+  return f;
+}
+
+// Same result as build_codes, for the tensor-core kernels.  Each thread owns
+// 32 consecutive tokens per round (their flags come from load_flags32; the
+// first round's may be loaded early by the caller and passed in `first`); one
+// shuffle scan across the warp and a short scan over the kThreads/32 warp
+// totals give each thread its starting block index.  Codes past S up to S_pad
+// (a multiple of 32) are 0xFFFF.  `scratch` is shared memory for kThreads/32
+// ints.  Every thread of the block must call it; it ends with a block barrier.
+// Per-128-token summaries the tile classifier needs: the block index (cs) of
+// the tile's first token, the largest cs in it, and whether it holds any /
+// only FAST tokens.
+struct TileSums {
+  uint16_t* cs_first;
+  uint16_t* cs_last;
+  uint8_t* fast;   // bit 0: any FAST token, bit 1: all tokens FAST
+};
+
 template <int kThreads>
 __device__ void build_codes_x32(const uint8_t* __restrict__ ar, const int32_t* __restrict__ seg,
-                                int S, int S_pad, uint16_t* codes, int* scratch) {
+                                int S, int S_pad, uint16_t* codes, int* scratch,
+                                Flags32 first, TileSums sums) {
   constexpr int kWarps = kThreads / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int carry = 0;
   for (int base = 0; base < S_pad; base += kThreads * 32) {
     const int t0 = base + (int)threadIdx.x * 32;
-    uint32_t bits = 0, fast = 0, expert = 0;
-    if (t0 + 32 <= S && (reinterpret_cast<uintptr_t>(ar + t0) & 15u) == 0) {
-      const uint4 a = *reinterpret_cast<const uint4*>(ar + t0);
-      const uint4 c = *reinterpret_cast<const uint4*>(ar + t0 + 16);
-      bits = nonzero_byte_bits(a.x) | (nonzero_byte_bits(a.y) << 4) |
-             (nonzero_byte_bits(a.z) << 8) | (nonzero_byte_bits(a.w) << 12) |
-             (nonzero_byte_bits(c.x) << 16) | (nonzero_byte_bits(c.y) << 20) |
-             (nonzero_byte_bits(c.z) << 24) | (nonzero_byte_bits(c.w) << 28);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (t0 + i < S && ar[t0 + i] != 0) bits |= 1u << i;
-    }
-    if (seg != nullptr) {
-      if (t0 + 32 <= S && (reinterpret_cast<uintptr_t>(seg + t0) & 15u) == 0) {
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const int4 v = reinterpret_cast<const int4*>(seg + t0)[g];
-          const int sv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            fast |= (sv[h] == kSegFast ? 1u : 0u) << (4 * g + h);
-            expert |= (sv[h] == kSegExpert ? 1u : 0u) << (4 * g + h);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int sv = t0 + i < S ? seg[t0 + i] : 0;
-          fast |= (sv == kSegFast ? 1u : 0u) << i;
-          expert |= (sv == kSegExpert ? 1u : 0u) << i;
-        }
-      }
-    }
-    const int cnt = __popc(bits);
+    const Flags32 f = base == 0 ? first : load_flags32(ar, seg, S, t0);
+    const int cnt = __popc(f.bits);
     int x = cnt;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -154,9 +184,9 @@ __device__ void build_codes_x32(const uint8_t* __restrict__ ar, const int32_t* _
         for (int h = 0; h < 2; ++h) {
           const int k = i + h;
           const uint32_t upto = k == 31 ? 0xFFFFFFFFu : ((2u << k) - 1u);
-          const uint32_t cs = (uint32_t)excl + (uint32_t)__popc(bits & upto);
+          const uint32_t cs = (uint32_t)excl + (uint32_t)__popc(f.bits & upto);
           c2[h] = t0 + k < S
-                      ? ((cs << 2) | (((expert >> k) & 1u) << 1) | ((fast >> k) & 1u))
+                      ? ((cs << 2) | (((f.expert >> k) & 1u) << 1) | ((f.fast >> k) & 1u))
                       : 0xFFFFu;
         }
         packed[i / 2] = c2[0] | (c2[1] << 16);
@@ -165,6 +195,26 @@ __device__ void build_codes_x32(const uint8_t* __restrict__ ar, const int32_t* _
 #pragma unroll
       for (int g = 0; g < 4; ++g)
         dst[g] = make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+    }
+    if (sums.cs_first != nullptr) {
+      // Four consecutive lanes own one 128-token tile: combine their parts.
+      const int nv = min(max(S - t0, 0), 32);                 // valid tokens here
+      const uint32_t vmask = nv >= 32 ? 0xFFFFFFFFu : ((1u << nv) - 1u);
+      uint32_t any_f = (f.fast & vmask) != 0u ? 1u : 0u;
+      uint32_t all_f = (f.fast & vmask) == vmask ? 1u : 0u;   // vacuous when nv == 0
+      uint32_t cs_hi = nv > 0 ? (uint32_t)excl + (uint32_t)__popc(f.bits & vmask) : 0u;
+#pragma unroll
+      for (int off = 1; off < 4; off <<= 1) {
+        any_f |= __shfl_xor_sync(0xffffffffu, any_f, off);
+        all_f &= __shfl_xor_sync(0xffffffffu, all_f, off);
+        cs_hi = max(cs_hi, __shfl_xor_sync(0xffffffffu, cs_hi, off));
+      }
+      if ((lane & 3) == 0 && t0 < S) {
+        const int tile = t0 >> 7;
+        sums.cs_first[tile] = (uint16_t)((uint32_t)excl + (f.bits & 1u));
+        sums.cs_last[tile] = (uint16_t)cs_hi;
+        sums.fast[tile] = (uint8_t)(any_f | (all_f << 1));
+      }
     }
     carry += total;
     __syncthreads();

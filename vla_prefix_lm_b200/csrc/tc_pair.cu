@@ -15,10 +15,11 @@
 // tensor rate instead of 64), and every MMA instruction and every barrier
 // round trip covers twice the work of a one-CTA, 64-key design.
 //
-// Mask: as in tc_attention.cu -- packed per-token codes (mask.cuh), key tiles
-// classified for the whole 256-row pair tile (skip / full / partial), partial
-// tiles masked per row by a visible-prefix length plus, for expert rows, the
-// FAST keys.
+// Mask: every CTA scans ar_mask / segment_ids into packed per-token codes
+// (mask.cuh), classifies each key tile for the whole 256-row pair tile (skip /
+// full / partial; both CTAs reach the same list), and masks a partial tile per
+// row by its visible-prefix length plus, for expert rows, the FAST keys.  No
+// mask is materialised.
 //
 // Warp roles per CTA (192 threads):
 //   warp 0      TMA producer for this CTA's halves (both CTAs)
@@ -79,11 +80,11 @@ struct __align__(8) Smem {
   uint32_t tmem_base;
   int abort;
   int n_list;
-  int q_any_exp, q_all_exp;
-  uint32_t cq_first, cq_last;
   int scan[kThreads / 32];
   uint16_t list[kMaxKeyTiles];
-  uint8_t cls[kMaxKeyTiles];
+  uint16_t tile_cs_first[kMaxKeyTiles];
+  uint16_t tile_cs_last[kMaxKeyTiles];
+  uint8_t tile_fast[kMaxKeyTiles];
 };
 
 constexpr int kOffCodes = kOffCtl + ((int)sizeof(Smem) + 127) / 128 * 128;
@@ -151,6 +152,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int n_key_tok = p.Sq;
   const int n_cache = kSuffix ? (p.P + kBN - 1) / kBN : 0;
 
+  // The mask bytes are the first global reads: issue them before anything
+  // else so their latency hides behind the barrier and TMEM set-up.
+  const uint8_t* ar_b = p.ar + (long long)b * p.mask_bs;
+  const int32_t* seg_b = (!kSuffix && p.seg) ? p.seg + (long long)b * p.mask_bs : nullptr;
+  const Flags32 flags0 = load_flags32(ar_b, seg_b, n_key_tok, (int)threadIdx.x * 32);
+
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
@@ -186,12 +193,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tmem_alloc_pair(&sm.tmem_base, 512);
     tmem_relinquish_pair();
   }
-  {
-    const uint8_t* ar = p.ar + (long long)b * p.mask_bs;
-    const int32_t* seg = (!kSuffix && p.seg) ? p.seg + (long long)b * p.mask_bs : nullptr;
-    build_codes_x32<kThreads>(ar, seg, n_key_tok, pad_tokens(n_key_tok), codes, sm.scan);
-  }
-  // Pair-tile summary, then per-key-tile classification (identical in both CTAs).
+  build_codes_x32<kThreads>(ar_b, seg_b, n_key_tok, pad_tokens(n_key_tok), codes, sm.scan,
+                            flags0, TileSums{sm.tile_cs_first, sm.tile_cs_last, sm.tile_fast});
+  // Warp 0 classifies every key tile for the whole 256-row pair tile (the
+  // list must be identical in both CTAs) and compacts the visited ones:
+  //   skip    no query of the pair sees any key of the tile
+  //   full    every query sees every key (no per-element predicate)
+  //   partial per-row visible prefix, FAST hole for expert rows
+  const int n_ktiles = (n_key_tok + kBN - 1) / kBN;
   if (warp == 0) {
     int any_e = 0, all_e = 1;
     for (int t = tq0 + lane; t <= tq1; t += 32) {
@@ -201,54 +210,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     any_e = __any_sync(0xffffffffu, any_e);
     all_e = __all_sync(0xffffffffu, all_e);
-    if (lane == 0) {
-      sm.q_any_exp = any_e;
-      sm.q_all_exp = all_e;
-      sm.cq_first = codes[tq0];
-      sm.cq_last = codes[tq1];
-    }
-  }
-  __syncthreads();
-  const int n_ktiles = (n_key_tok + kBN - 1) / kBN;
-  {
-    const uint32_t csq0 = sm.cq_first >> 2, csq1 = sm.cq_last >> 2;
-    const int q_any_exp = sm.q_any_exp, q_all_exp = sm.q_all_exp;
-    for (int t = warp; t < n_ktiles; t += kThreads / 32) {
-      const int k0 = t * kBN;
-      const int k1 = min(k0 + kBN, n_key_tok) - 1;
-      int any_f = 0, all_f = 1;
-      for (int j = k0 + lane; j <= k1; j += 32) {
-        const int f = codes[j] & 1;
-        any_f |= f;
-        all_f &= f;
-      }
-      any_f = __any_sync(0xffffffffu, any_f);
-      all_f = __all_sync(0xffffffffu, all_f);
-      if (lane == 0) {
-        const uint32_t csk0 = codes[k0] >> 2, csk1 = codes[k1] >> 2;
-        uint8_t c;
-        if (csk0 > csq1 || (q_all_exp && all_f)) {
-          c = 0;
-        } else if (csk1 <= csq0 && !(q_any_exp && any_f) && k1 - k0 + 1 == kBN) {
-          c = 1;
-        } else {
-          c = 2;
-        }
-        sm.cls[t] = c | (any_f ? 4 : 0);
-      }
-    }
-  }
-  __syncthreads();
-  if (warp == 0) {
+    const uint32_t csq0 = codes[tq0] >> 2, csq1 = codes[tq1] >> 2;
     int base = 0;
     for (int t0 = 0; t0 < n_ktiles; t0 += 32) {
       const int t = t0 + lane;
-      const uint8_t c = t < n_ktiles ? sm.cls[t] : 0;
-      const unsigned m = __ballot_sync(0xffffffffu, (c & 3) != 0);
-      if (c & 3) {
+      int c = 0;
+      bool any_f = false;
+      if (t < n_ktiles) {
+        const uint32_t csk0 = sm.tile_cs_first[t], csk1 = sm.tile_cs_last[t];
+        any_f = (sm.tile_fast[t] & 1) != 0;
+        const bool all_f = (sm.tile_fast[t] & 2) != 0;
+        const bool complete = (t + 1) * kBN <= n_key_tok;
+        if (csk0 > csq1 || (all_e && all_f)) c = 0;
+        else if (csk1 <= csq0 && !(any_e && any_f) && complete) c = 1;
+        else c = 2;
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, c != 0);
+      if (c != 0) {
         const int pos = base + __popc(m & ((1u << lane) - 1));
-        sm.list[pos] = (uint16_t)(t | ((c & 3) == 2 ? kTilePartial : 0) |
-                                  ((c & 4) ? kTileAnyFast : 0));
+        sm.list[pos] = (uint16_t)(t | (c == 2 ? kTilePartial : 0) | (any_f ? kTileAnyFast : 0));
       }
       base += __popc(m);
     }
@@ -481,7 +461,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const float p0 = ex2(fmaf(x[2 * e], c, nm));
         const float p1 = ex2(fmaf(x[2 * e + 1], c, nm));
         ls[e & 7] += p0 + p1;
-        pk[e] = pack_bf16x2(p0, p1);
+        pk[e] = pack_bf16x2_rna(p0, p1);
       }
       l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
 
@@ -517,7 +497,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(bs ? p_full_l1 : p_full_l0);
+      if (lane == 0) mbar_arrive_remote(bs ? p_full_l1 : p_full_l0);
     }
 
     if (ok && n_it > 0) {
@@ -560,7 +540,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (!kSuffix && p.lse && row_valid)
           p.lse[grow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
-      } else if (row_valid) {
+      } else {
+        // Split-K partial: unnormalised O and (m, l) for the combine kernel.
+        // tcgen05.ld is warp-collective (.sync.aligned): every lane loads,
+        // only lanes holding a real row store.
         const long long slot = ((long long)split * p.B + b) * rows_per_b + row0 + r;
         float* wo = p.ws + slot * kD;
 #pragma unroll 1
@@ -569,15 +552,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tmem_ld32(tO + lane_off + 32 * cc, o);
           tmem_ld_wait();
           reg_fence(o);
+          if (row_valid) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(wo + 32 * cc + e) =
-                make_float4(__uint_as_float(o[e]), __uint_as_float(o[e + 1]),
-                            __uint_as_float(o[e + 2]), __uint_as_float(o[e + 3]));
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(wo + 32 * cc + e) =
+                  make_float4(__uint_as_float(o[e]), __uint_as_float(o[e + 1]),
+                              __uint_as_float(o[e + 2]), __uint_as_float(o[e + 3]));
+          }
         }
-        float* wml = p.ws + (long long)p.n_splits * p.B * rows_per_b * kD + slot * 2;
-        wml[0] = m_run;
-        wml[1] = l_run;
+        if (row_valid) {
+          float* wml = p.ws + (long long)p.n_splits * p.B * rows_per_b * kD + slot * 2;
+          wml[0] = m_run;
+          wml[1] = l_run;
+        }
       }
     }
     if (n_it == 0 && p.n_splits > 1 && row0 + r < rows_per_b) {
@@ -588,6 +575,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   }
 
+  // The Q load was issued before the key tiles were counted: a split with no
+  // tiles (or one that gave up) must still let both halves land before the
+  // CTAs leave.  Completed already in every other case, so this returns at once.
+  if (leader && threadIdx.x == 0) (void)mbar_wait(&sm.q_full, 0, ctl);
   // Neither CTA may leave while its partner can still signal its barriers or
   // read its shared memory; then both free their TMEM.
   __syncwarp();
@@ -598,6 +589,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem, 512);
   }
+}
+
+// Merges split-K partials: out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s
+// with M = max_s m_s (the log-sum-exp rule).  One warp per output row; each
+// lane handles 8 of the 256 columns.  HBM-bound: it reads the fp32 partials
+// once and writes the bf16 row once.
+__global__ void __launch_bounds__(256)
+    combine_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ out, int n_splits,
+                   long long n_rows) {
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= n_rows) return;
+  const float* ml = ws + (long long)n_splits * n_rows * kD;
+  float M = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, ml[(s * n_rows + row) * 2]);
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  float L = 0.f;
+  for (int s = 0; s < n_splits; ++s) {
+    const float m = ml[(s * n_rows + row) * 2];
+    const float l = ml[(s * n_rows + row) * 2 + 1];
+    if (l == 0.f) continue;
+    const float w = ex2(m - M);
+    L += w * l;
+    const float4* src = reinterpret_cast<const float4*>(ws + (s * n_rows + row) * kD + lane * 8);
+    const float4 a = src[0], c = src[1];
+    acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
+    acc[4] += w * c.x; acc[5] += w * c.y; acc[6] += w * c.z; acc[7] += w * c.w;
+  }
+  const float inv = 1.f / L;
+  uint4 pk;
+  pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  pk.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  pk.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  *reinterpret_cast<uint4*>(out + row * kD + lane * 8) = pk;
 }
 
 size_t pair_smem_bytes(int n_code_tokens) {
@@ -626,7 +652,38 @@ cudaError_t launch_tc_pair(const TcParams& p, bool suffix_mode, const DevCtl& ct
   } else {
     tc_pair_kernel<false><<<grid, kThreads, smem, st>>>(p, ctl);
   }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || p.n_splits <= 1) return e;
+  const long long n_rows = (long long)p.B * rows;
+  combine_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, st>>>(
+      p.ws, reinterpret_cast<__nv_bfloat16*>(p.out_ptr), p.n_splits, n_rows);
   return cudaGetLastError();
+}
+
+int tc_suffix_splits(int B, int Sq, int P, int Hq) {
+  // Split the key tiles over several CTA pairs only when the pairs of one
+  // split would leave SMs idle: enough splits to fill the SMs once, each
+  // keeping at least two key tiles, at most 8.
+  static int n_sm = [] {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+  }();
+  const int rows = Sq * Hq;
+  const int n_ctas = 2 * ((rows + 2 * kBM - 1) / (2 * kBM)) * B;
+  const int tiles = (P + kBN - 1) / kBN + (Sq + kBN - 1) / kBN;
+  int s = n_sm / max(n_ctas, 1);
+  s = min(s, tiles / 2);
+  s = min(s, 8);
+  return max(s, 1);
+}
+
+size_t tc_suffix_workspace_bytes(int B, int Sq, int P, int Hq) {
+  const int s = tc_suffix_splits(B, Sq, P, Hq);
+  if (s <= 1) return 0;
+  const size_t rows = (size_t)B * Sq * Hq;
+  return (size_t)s * rows * (kD + 2) * sizeof(float);
 }
 
 }  // namespace piattn
