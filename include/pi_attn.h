@@ -182,6 +182,34 @@ uint64_t pi_attn_set_wait_limit(uint64_t cycles);
  */
 int pi_attn_selftest_wait(pi_stream_t stream);
 
+/*
+ * pi_attn_suffix_noalloc -- pi_attn_suffix for callers that cannot allocate
+ * device memory.  The pages have no counterpart: this is plumbing, not part of
+ * the method.  Same arguments, layout, result and errors as pi_attn_suffix,
+ * minus the workspace: the split-K partials go to a fixed buffer inside the
+ * library (a file-scope __device__ array, one per device, of
+ * pi_attn_suffix_noalloc_capacity() = 16 MiB).
+ *
+ *  - Allocates nothing: no cudaMalloc/cudaFree, no allocating library call.
+ *  - The first call on each device looks up the buffer's address
+ *    (cudaGetSymbolAddress) and caches it; make that first call before any
+ *    stream capture begins.
+ *  - Nothing in the buffer needs to start at zero: every call writes each
+ *    partial it later reads.
+ *  - Two calls that may overlap on the GPU (different streams of one device)
+ *    race on the shared buffer and give wrong results; calls on one stream are
+ *    ordered and safe.  Different devices have separate buffers.
+ *  - PI_ERR_UNSUPPORTED, before anything is enqueued, when the descriptor
+ *    needs more than the capacity (pi_attn_suffix_workspace_bytes(desc) >
+ *    16 MiB; that happens only for small-batch shapes with many query rows).
+ */
+int pi_attn_suffix_noalloc(const pi_attn_desc* desc, const void* q_suf, const void* k_suf,
+                           const void* v_suf, const void* k_cache, const void* v_cache,
+                           const uint8_t* ar_mask_suf, void* out, pi_stream_t stream);
+
+/* Size in bytes of the fixed buffer pi_attn_suffix_noalloc uses. */
+size_t pi_attn_suffix_noalloc_capacity(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -32,6 +32,8 @@ EXPORTED = (
     "pi_attn_status_string",
     "pi_attn_set_wait_limit",
     "pi_attn_selftest_wait",
+    "pi_attn_suffix_noalloc",
+    "pi_attn_suffix_noalloc_capacity",
 )
 
 
@@ -84,6 +86,10 @@ def lib() -> ctypes.CDLL:
         L.pi_attn_set_wait_limit.restype = ctypes.c_uint64
         L.pi_attn_selftest_wait.argtypes = [vp]
         L.pi_attn_selftest_wait.restype = i32
+        L.pi_attn_suffix_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.pi_attn_suffix_noalloc.restype = i32
+        L.pi_attn_suffix_noalloc_capacity.argtypes = []
+        L.pi_attn_suffix_noalloc_capacity.restype = sz
         _lib = L
     return _lib
 
@@ -204,6 +210,34 @@ def pi_attn_suffix(q_suf, k_suf, v_suf, k_cache, v_cache, ar_mask_suf, out=None,
                               _ptr(workspace), ws_bytes, ctypes.c_void_p(_stream(stream)))
     if rc != PI_OK:
         raise PiAttnError(rc, "pi_attn_suffix")
+    return out
+
+
+def pi_attn_suffix_noalloc(q_suf, k_suf, v_suf, k_cache, v_cache, ar_mask_suf, out,
+                           softmax_scale=1.0, stream=None):
+    """pi_attn_suffix with the split-K scratch in the library's fixed device
+    buffer: allocates nothing, so ``out`` must be given."""
+    _need(q_suf, "q_suf", dims=4)
+    _need(k_suf, "k_suf", q_suf.dtype, 4)
+    _need(v_suf, "v_suf", q_suf.dtype, 4)
+    _need(ar_mask_suf, "ar_mask_suf", torch.uint8)
+    if k_cache is not None:
+        _need(k_cache, "k_cache", q_suf.dtype, 4)
+        _need(v_cache, "v_cache", q_suf.dtype, 4)
+        if k_cache.shape != v_cache.shape or k_cache.shape[0] != q_suf.shape[0]:
+            raise ValueError("cache shape mismatch")
+    _need(out, "out", q_suf.dtype, 4)
+    desc = _suffix_desc(q_suf, k_suf, k_cache, ar_mask_suf, softmax_scale)
+    rc = lib().pi_attn_suffix_noalloc(ctypes.byref(desc), _ptr(q_suf), _ptr(k_suf),
+                                      _ptr(v_suf), _ptr(k_cache), _ptr(v_cache),
+                                      _ptr(ar_mask_suf), _ptr(out),
+                                      ctypes.c_void_p(_stream(stream)))
+    if rc != PI_OK:
+        need = int(lib().pi_attn_suffix_workspace_bytes(ctypes.byref(desc)))
+        cap = int(lib().pi_attn_suffix_noalloc_capacity())
+        extra = (f": needs {need} bytes of scratch, the fixed buffer holds {cap}"
+                 if rc == PI_ERR_UNSUPPORTED and need > cap else "")
+        raise PiAttnError(rc, "pi_attn_suffix_noalloc" + extra)
     return out
 
 
