@@ -144,7 +144,7 @@ int pi_attn_prefill(const pi_attn_desc* d, const void* q, const void* k, const v
   if (!encode_rows(&p.map_q, q, rows, d->B, 128) ||
       !encode_rows(&p.map_k, k, d->Sq, d->B, 64) ||
       !encode_rows(&p.map_vh, v, d->Sq, d->B, 128, 2) ||
-      !encode_rows(&p.map_o, out, rows, d->B, 32))
+      !encode_rows(&p.map_o, out, rows, d->B, 32, 1))
     return PI_ERR_CUDA;
   p.map_kc = p.map_k;
   p.map_vch = p.map_vh;
@@ -210,7 +210,7 @@ int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
   if (!encode_rows(&p.map_q, q_suf, rows, d->B, 128) ||
       !encode_rows(&p.map_k, k_suf, d->Sq, d->B, 64) ||
       !encode_rows(&p.map_vh, v_suf, d->Sq, d->B, 128, 2) ||
-      !encode_rows(&p.map_o, out, rows, d->B, 32))
+      !encode_rows(&p.map_o, out, rows, d->B, 32, 1))
     return PI_ERR_CUDA;
   if (d->P > 0) {
     if (!encode_rows(&p.map_kc, k_cache, d->P, d->B, 64) ||

@@ -1,41 +1,52 @@
 // tc_pair.cu -- bf16 joint (prefix-LM) attention on tcgen05, CTA-pair (2-SM) form.
 //
-// A cluster of two CTAs computes one 256-row query tile: 256 / Hq query
-// tokens x Hq heads, 128 rows per CTA.  With a single KV head all rows read
-// the same K/V rows ("π0.5 vs MM-DiT joint attention", "joint attention 只管
-// 算子": 8 query heads, 1 KV head, head_dim 256, one shared KV pool).
+// A cluster of two CTAs computes 256-row query tiles: 256 / Hq query tokens x
+// Hq heads, 128 rows per CTA.  With a single KV head all rows read the same
+// K/V rows ("π0.5 vs MM-DiT joint attention", "joint attention 只管算子": 8
+// query heads, 1 KV head, head_dim 256, one shared KV pool).
 //
 // Per key tile of 128 keys, issued by ONE thread of the even CTA for the pair:
 //   S = Q K^T   tcgen05.mma.cta_group::2, M = 256: A = Q rows of each CTA
 //               (its shared memory), B = K split by keys (64 per CTA)
-//   P           fp32 online softmax in each CTA, one thread per row
-//   O += P V    tcgen05.mma.cta_group::2: A = P (each CTA's TMEM, bf16),
+//   P           fp32 online softmax in each CTA, one thread per row; P is
+//               written to shared memory as bf16 and S's TMEM is released as
+//               soon as it has been read, so QK of the next tiles never waits
+//               for a PV
+//   O += P V    tcgen05.mma.cta_group::2: A = P (each CTA's shared memory),
 //               B = V split by columns (128 of the 256 per CTA)
-// Each SM therefore streams half of every K/V tile (32 B/clk at the full
-// tensor rate instead of 64), and every MMA instruction and every barrier
-// round trip covers twice the work of a one-CTA, 64-key design.
+// Each SM streams half of every K/V tile, and every MMA instruction and every
+// barrier round trip covers twice the work of a one-CTA, 64-key design.
+//
+// Work units.  A unit is one (batch, 256-row query tile, key split).  When
+// ar_mask / segment_ids are shared by the batch, one cluster per SM pair runs
+// and walks units c, c + C, c + 2C, ...: the next unit's Q is loaded as soon
+// as the last QK of the current one has read Q, its first QKs run while the
+// softmax warps write the current unit's output, and the mask scan runs once
+// per cluster.  With per-batch masks every unit gets its own cluster.
 //
 // Mask: every CTA scans ar_mask / segment_ids into packed per-token codes
-// (mask.cuh), classifies each key tile for the whole 256-row pair tile (skip /
-// full / partial; both CTAs reach the same list), and masks a partial tile per
-// row by its visible-prefix length plus, for expert rows, the FAST keys.  No
-// mask is materialised.
+// (mask.cuh).  Per unit, each warp classifies every key tile for the unit's
+// 256 query rows (skip / full / partial) into its own list -- all lists are
+// equal, and private lists need no cross-warp synchronisation -- and a
+// partial tile is masked per row by its visible-prefix length plus, for
+// expert rows, the FAST keys.  No mask is materialised.
 //
 // Warp roles per CTA (192 threads):
 //   warp 0      TMA producer for this CTA's halves (both CTAs)
 //   warp 1      TMEM allocation (both CTAs, cta_group::2); MMA issue (even CTA)
 //   warps 2..5  softmax, O correction, epilogue (both CTAs, own rows)
 //
-// TMEM per CTA (512 columns): O fp32 [0,256) | S0 [256,384) | S1 [384,512);
-// P of tile t is packed bf16 over the first 64 columns of S[t%2].
-// Shared memory per CTA: Q 64 KB | ring 4 x 32 KB (K halves [64 x 256], V
-// halves [128 x 128]) | control | per-token codes.  The epilogue stages the
-// bf16 output in the Q area (dead after the last QK).
+// TMEM per CTA (512 columns): O fp32 [0,256) | S0 [256,384) | S1 [384,512).
+// Shared memory per CTA: Q 64 KB | ring 3 x 32 KB (K halves [64 x 256], V
+// halves [128 x 128]) | P 32 KB ([128 rows x 128 keys] bf16, two 128-byte-
+// swizzled [128 x 64] blocks; also the output staging area) | control |
+// per-token codes.
 //
-// Synchronisation across the pair: the even CTA owns q_full, kv_full and
-// p_full (the odd CTA's TMA loads and softmax warps arrive there through
-// cluster addresses); the MMA thread's commits arrive on the s_full, o_done
-// and kv_empty barriers of both CTAs.  Every wait is bounded (DevCtl).
+// Synchronisation across the pair: the even CTA owns q_full, kv_full, s_free,
+// p_full and o_free (the odd CTA's TMA loads and softmax warps arrive there
+// through cluster addresses); the MMA thread's commits arrive on the q_empty,
+// kv_empty, s_full and o_done barriers of both CTAs.  Every wait is bounded
+// (DevCtl).  Counters that index barriers and ring slots run across units.
 #include <cfloat>
 
 #include "launch.h"
@@ -54,12 +65,18 @@ constexpr int kQBytes = 4 * kQBlk;          // 64 KB
 constexpr int kKBlk = 64 * 128;             // K half block: [64 keys x 64 d] = 8 KB
 constexpr int kVBlk = kBN * 128;            // V half block: [128 keys x 64 d] = 16 KB
 constexpr int kItemBytes = 32768;           // K half (4 x 8 KB) or V half (2 x 16 KB)
-constexpr int kStages = 4;
+constexpr int kStages = 3;
+constexpr int kPBlk = kBM * 128;            // P block: [128 rows x 64 keys] = 16 KB
+constexpr int kPBytes = 2 * kPBlk;          // 32 KB
+constexpr int kStageRows = 32;              // output rows staged per softmax warp
 constexpr int kOffQ = 0;
 constexpr int kOffRing = kQBytes;
-constexpr int kOffCtl = kOffRing + kStages * kItemBytes;
+constexpr int kOffP = kOffRing + kStages * kItemBytes;
+constexpr int kOffCtl = kOffP + kPBytes;
 constexpr int kMaxKeyTiles = (kMaxTokens + kBN - 1) / kBN + 2;
+constexpr int kLists = kThreads / 32;       // one private tile list per warp
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 256
+constexpr int kSmemLimit = 232448;          // 227 KB per CTA on sm_100
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(2 * kBM, kBN, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(2 * kBM, kD, false, true);
@@ -70,18 +87,20 @@ constexpr uint16_t kTileAnyFast = 0x4000;
 constexpr uint16_t kTileIndex = 0x3FFF;
 
 struct __align__(8) Smem {
-  uint64_t q_full;               // even CTA: both Q halves landed
+  uint64_t q_full;               // even CTA: both Q halves landed (one phase per unit)
+  uint64_t q_empty;              // each CTA: the unit's last QK has read Q
   uint64_t kv_full[kStages];     // even CTA: both halves of a K or V item landed
   uint64_t kv_empty[kStages];    // each CTA: its ring stage may be refilled
   uint64_t s_full[2];            // each CTA: S tile in its TMEM
-  uint64_t p_full[2];            // even CTA: P written by the pair's 8 softmax warps
+  uint64_t s_free[2];            // even CTA: the pair's 8 softmax warps have read S
+  uint64_t p_full;               // even CTA: P written by the pair's 8 softmax warps
   uint64_t o_done;               // each CTA: PV finished
+  uint64_t o_free;               // even CTA: the pair's softmax warps have read O
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  int n_list;
   int scan[kThreads / 32];
-  uint16_t list[kMaxKeyTiles];
+  uint16_t list[kLists][kMaxKeyTiles];
   uint16_t tile_cs_first[kMaxKeyTiles];
   uint16_t tile_cs_last[kMaxKeyTiles];
   uint8_t tile_fast[kMaxKeyTiles];
@@ -90,6 +109,12 @@ struct __align__(8) Smem {
 constexpr int kOffCodes = kOffCtl + ((int)sizeof(Smem) + 127) / 128 * 128;
 
 __host__ __device__ constexpr int pad_tokens(int n) { return (n + 127) / 128 * 128; }
+
+// Bytes the kernel's layout needs past a 1024-byte aligned base.
+__host__ __device__ constexpr int layout_bytes(int n_code_tokens) {
+  return kOffCodes + pad_tokens(n_code_tokens) * 2;
+}
+static_assert(layout_bytes(kMaxTokens) <= kSmemLimit, "shared-memory layout too large");
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -112,6 +137,12 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Sm
   return true;
 }
 
+// Warp-uniform bounded wait: every lane polls, all lanes get the same answer.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Smem& sm,
+                                          const DevCtl& ctl) {
+  return __all_sync(0xffffffffu, wait_or_abort(bar, parity, sm, ctl));
+}
+
 struct KvTile {
   int src;       // 0: k/v (prefill keys or suffix keys), 1: cached prefix
   int tile;
@@ -120,62 +151,141 @@ struct KvTile {
 };
 
 template <bool kSuffix>
-__device__ __forceinline__ KvTile kv_tile_at(const Smem& sm, int idx, int n_cache, int P) {
+__device__ __forceinline__ KvTile kv_tile_at(const uint16_t* list, int idx, int n_cache, int P) {
   if (kSuffix && idx < n_cache) return KvTile{1, idx, (idx + 1) * kBN > P, false};
-  const uint16_t e = sm.list[kSuffix ? idx - n_cache : idx];
+  const uint16_t e = list[kSuffix ? idx - n_cache : idx];
   return KvTile{0, (int)(e & kTileIndex), (e & kTilePartial) != 0, (e & kTileAnyFast) != 0};
+}
+
+// One work unit: a (batch, pair tile, key split) triple, plus its key range.
+struct Unit {
+  int b, pair, split;
+  int tq0, tq1;        // first / last valid query token of the pair tile
+  int it_begin, n_it;  // this split's slice of the visited key tiles
+};
+
+// Warp-collective: classifies every key tile for the unit's query tokens
+// [tq0, tq1] and writes the visited ones, in order, to `list`:
+//   skip    no query of the unit sees any key of the tile
+//   full    every query sees every key (no per-element predicate)
+//   partial per-row visible prefix, FAST hole for expert rows
+// Returns the number of entries (the same in every lane).
+__device__ int build_tile_list(const Smem& sm, const uint16_t* codes, int tq0, int tq1,
+                               int n_key_tok, uint16_t* list, int lane) {
+  const int n_ktiles = (n_key_tok + kBN - 1) / kBN;
+  int any_e = 0, all_e = 1;
+  for (int t = tq0 + lane; t <= tq1; t += 32) {
+    const int e = (codes[t] >> 1) & 1;
+    any_e |= e;
+    all_e &= e;
+  }
+  any_e = __any_sync(0xffffffffu, any_e);
+  all_e = __all_sync(0xffffffffu, all_e);
+  const uint32_t csq0 = codes[tq0] >> 2, csq1 = codes[tq1] >> 2;
+  int base = 0;
+  for (int t0 = 0; t0 < n_ktiles; t0 += 32) {
+    const int t = t0 + lane;
+    int c = 0;
+    bool any_f = false;
+    if (t < n_ktiles) {
+      const uint32_t csk0 = sm.tile_cs_first[t], csk1 = sm.tile_cs_last[t];
+      any_f = (sm.tile_fast[t] & 1) != 0;
+      const bool all_f = (sm.tile_fast[t] & 2) != 0;
+      const bool complete = (t + 1) * kBN <= n_key_tok;
+      if (csk0 > csq1 || (all_e && all_f)) c = 0;
+      else if (csk1 <= csq0 && !(any_e && any_f) && complete) c = 1;
+      else c = 2;
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, c != 0);
+    if (c != 0) {
+      const int pos = base + __popc(m & ((1u << lane) - 1));
+      list[pos] = (uint16_t)(t | (c == 2 ? kTilePartial : 0) | (any_f ? kTileAnyFast : 0));
+    }
+    base += __popc(m);
+  }
+  __syncwarp();
+  return base;
+}
+
+// Warp-collective: the unit with index u and this warp's tile list for it.
+template <bool kSuffix>
+__device__ __forceinline__ Unit make_unit(int u, const TcParams& p, int n_pairs, int n_cache,
+                                          const Smem& sm, const uint16_t* codes, uint16_t* list,
+                                          int lane) {
+  Unit x;
+  x.split = u % p.n_splits;
+  const int t = u / p.n_splits;
+  x.pair = t % n_pairs;
+  x.b = t / n_pairs;
+  const int tok_per_pair = 2 * kBM / p.Hq;
+  x.tq0 = x.pair * tok_per_pair;
+  x.tq1 = min(x.tq0 + tok_per_pair, p.Sq) - 1;
+  const int n_list = build_tile_list(sm, codes, x.tq0, x.tq1, p.Sq, list, lane);
+  const int n_total = n_cache + n_list;
+  const int per = (n_total + p.n_splits - 1) / p.n_splits;
+  x.it_begin = min(x.split * per, n_total);
+  x.n_it = min(x.it_begin + per, n_total) - x.it_begin;
+  return x;
 }
 
 template <bool kSuffix>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    tc_pair_kernel(const __grid_constant__ TcParams p, const DevCtl ctl) {
+    tc_pair_kernel(const __grid_constant__ TcParams p, const DevCtl ctl, int smem_bytes) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // Both CTAs see the same base offset, so both leave here or neither does.
+  if ((int)(smem - smem_raw) + layout_bytes(p.Sq) > smem_bytes) {
+    if (threadIdx.x == 0) record_status(ctl, kStatusUnsupported);
+    return;
+  }
   Smem& sm = *reinterpret_cast<Smem*>(smem + kOffCtl);
   uint16_t* codes = reinterpret_cast<uint16_t*>(smem + kOffCodes);
   uint8_t* sQ = smem + kOffQ;
   uint8_t* ring = smem + kOffRing;
+  uint8_t* sP = smem + kOffP;
 
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows_per_b = p.Sq * p.Hq;
   const int n_pairs = (rows_per_b + 2 * kBM - 1) / (2 * kBM);
-  const int pair = (blockIdx.x >> 1) % n_pairs;
-  const int split = (blockIdx.x >> 1) / n_pairs;
-  const int b = blockIdx.y;
-  const int row0 = pair * 2 * kBM + (int)rank * kBM;   // first row of this CTA
-  const int tok_per_pair = 2 * kBM / p.Hq;
-  const int tq0 = pair * tok_per_pair;                  // first token of the pair
-  const int tq1 = min(tq0 + tok_per_pair, p.Sq) - 1;    // last valid token of the pair
+  const int n_units = p.B * n_pairs * p.n_splits;
+  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
   const int n_key_tok = p.Sq;
   const int n_cache = kSuffix ? (p.P + kBN - 1) / kBN : 0;
 
   // The mask bytes are the first global reads: issue them before anything
-  // else so their latency hides behind the barrier and TMEM set-up.
-  const uint8_t* ar_b = p.ar + (long long)b * p.mask_bs;
-  const int32_t* seg_b = (!kSuffix && p.seg) ? p.seg + (long long)b * p.mask_bs : nullptr;
+  // else so their latency hides behind the barrier and TMEM set-up.  With a
+  // batch-shared mask (the persistent case) every unit uses row 0; otherwise
+  // this cluster runs exactly one unit and scans that unit's batch row.
+  const int b_codes = (cluster / p.n_splits) / n_pairs;
+  const uint8_t* ar_b = p.ar + (long long)b_codes * p.mask_bs;
+  const int32_t* seg_b = (!kSuffix && p.seg) ? p.seg + (long long)b_codes * p.mask_bs : nullptr;
   const Flags32 flags0 = load_flags32(ar_b, seg_b, n_key_tok, (int)threadIdx.x * 32);
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_empty, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.p_full[s], 8);
+      mbar_init(&sm.s_free[s], 8);
     }
+    mbar_init(&sm.p_full, 8);
     mbar_init(&sm.o_done, 1);
+    mbar_init(&sm.o_free, 8);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&p.map_q);
     tma_prefetch_desc(&p.map_k);
     tma_prefetch_desc(&p.map_vh);
+    tma_prefetch_desc(&p.map_o);
     if (kSuffix) {
       tma_prefetch_desc(&p.map_kc);
       tma_prefetch_desc(&p.map_vch);
@@ -183,57 +293,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   // Both CTAs' barriers must exist before either side signals the other.
   cluster_sync();
-  const uint32_t q_full_l = mapa_shared(smem_u32(&sm.q_full), 0);
-  if (threadIdx.x == 0) {
-    // Q does not depend on the mask: start it before the scan.
-    if (leader) mbar_arrive_expect_tx(&sm.q_full, 2 * kQBytes);
-    tma_load_4d_pair(sQ, &p.map_q, q_full_l, 0, row0, 0, b);
-  }
   if (warp == 1) {
     tmem_alloc_pair(&sm.tmem_base, 512);
     tmem_relinquish_pair();
   }
   build_codes_x32<kThreads>(ar_b, seg_b, n_key_tok, pad_tokens(n_key_tok), codes, sm.scan,
                             flags0, TileSums{sm.tile_cs_first, sm.tile_cs_last, sm.tile_fast});
-  // Warp 0 classifies every key tile for the whole 256-row pair tile (the
-  // list must be identical in both CTAs) and compacts the visited ones:
-  //   skip    no query of the pair sees any key of the tile
-  //   full    every query sees every key (no per-element predicate)
-  //   partial per-row visible prefix, FAST hole for expert rows
-  const int n_ktiles = (n_key_tok + kBN - 1) / kBN;
-  if (warp == 0) {
-    int any_e = 0, all_e = 1;
-    for (int t = tq0 + lane; t <= tq1; t += 32) {
-      const int e = (codes[t] >> 1) & 1;
-      any_e |= e;
-      all_e &= e;
-    }
-    any_e = __any_sync(0xffffffffu, any_e);
-    all_e = __all_sync(0xffffffffu, all_e);
-    const uint32_t csq0 = codes[tq0] >> 2, csq1 = codes[tq1] >> 2;
-    int base = 0;
-    for (int t0 = 0; t0 < n_ktiles; t0 += 32) {
-      const int t = t0 + lane;
-      int c = 0;
-      bool any_f = false;
-      if (t < n_ktiles) {
-        const uint32_t csk0 = sm.tile_cs_first[t], csk1 = sm.tile_cs_last[t];
-        any_f = (sm.tile_fast[t] & 1) != 0;
-        const bool all_f = (sm.tile_fast[t] & 2) != 0;
-        const bool complete = (t + 1) * kBN <= n_key_tok;
-        if (csk0 > csq1 || (all_e && all_f)) c = 0;
-        else if (csk1 <= csq0 && !(any_e && any_f) && complete) c = 1;
-        else c = 2;
-      }
-      const unsigned m = __ballot_sync(0xffffffffu, c != 0);
-      if (c != 0) {
-        const int pos = base + __popc(m & ((1u << lane) - 1));
-        sm.list[pos] = (uint16_t)(t | (c == 2 ? kTilePartial : 0) | (any_f ? kTileAnyFast : 0));
-      }
-      base += __popc(m);
-    }
-    if (lane == 0) sm.n_list = base;
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -241,79 +306,100 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   const uint32_t tO = tmem + kColO;
   const uint32_t tS = tmem + kColS;      // S[b] at +128*b
-
-  const int n_total = n_cache + sm.n_list;
-  const int per = (n_total + p.n_splits - 1) / p.n_splits;
-  const int it_begin = min(split * per, n_total);
-  const int it_end = min(it_begin + per, n_total);
-  const int n_it = it_end - it_begin;
+  uint16_t* list = sm.list[warp];
 
   if (warp == 0) {
     // ------------------------------------------------- producer (both CTAs)
-    if (n_it > 0) {
-      uint32_t u = 0;
+    const uint32_t q_full_l = mapa_shared(smem_u32(&sm.q_full), 0);
+    uint32_t u = 0;                 // ring items issued
+    uint32_t nq = 0;                // Q loads issued
+    bool ok = true;
+    for (int unit = cluster; unit < n_units && ok; unit += n_clusters) {
+      const Unit x = make_unit<kSuffix>(unit, p, n_pairs, n_cache, sm, codes, list, lane);
+      if (x.n_it == 0) continue;
+      const int row0 = x.pair * 2 * kBM + (int)rank * kBM;
+      if (nq > 0 && !warp_wait(&sm.q_empty, (nq - 1) & 1, sm, ctl)) break;
+      if (lane == 0) {
+        if (leader) mbar_arrive_expect_tx(&sm.q_full, 2 * kQBytes);
+        tma_load_4d_pair(sQ, &p.map_q, q_full_l, 0, row0, 0, x.b);
+      }
+      __syncwarp();
+      ++nq;
       auto load = [&](int idx, bool is_v) -> bool {
-        const KvTile kt = kv_tile_at<kSuffix>(sm, idx, n_cache, p.P);
+        const KvTile kt = kv_tile_at<kSuffix>(list, idx, n_cache, p.P);
         const int s = (int)(u % kStages);
         const uint32_t rel = u / kStages;
-        if (rel > 0) {
-          const bool ok = wait_or_abort(&sm.kv_empty[s], (rel - 1) & 1, sm, ctl);
-          if (!__all_sync(0xffffffffu, ok)) return false;
-        }
+        if (rel > 0 && !warp_wait(&sm.kv_empty[s], (rel - 1) & 1, sm, ctl)) return false;
         if (lane == 0) {
           const uint32_t full_l = mapa_shared(smem_u32(&sm.kv_full[s]), 0);
           if (leader) mbar_arrive_expect_tx(&sm.kv_full[s], 2 * kItemBytes);
           uint8_t* dst = ring + s * kItemBytes;
           if (!is_v) {   // this CTA's 64 keys of the tile, all 256 columns
             const CUtensorMap* map = kt.src ? &p.map_kc : &p.map_k;
-            tma_load_4d_pair(dst, map, full_l, 0, kt.tile * kBN + 64 * (int)rank, 0, b);
+            tma_load_4d_pair(dst, map, full_l, 0, kt.tile * kBN + 64 * (int)rank, 0, x.b);
           } else {       // all 128 keys of the tile, this CTA's 128 columns
             const CUtensorMap* map = kt.src ? &p.map_vch : &p.map_vh;
-            tma_load_4d_pair(dst, map, full_l, 0, kt.tile * kBN, 2 * (int)rank, b);
+            tma_load_4d_pair(dst, map, full_l, 0, kt.tile * kBN, 2 * (int)rank, x.b);
           }
         }
         __syncwarp();
         ++u;
         return true;
       };
-      bool ok = true;
-      for (int i = it_begin; i < it_end && ok; ++i) {
+      const int it_end = x.it_begin + x.n_it;
+      for (int i = x.it_begin; i < it_end && ok; ++i) {
         ok = load(i, false);
-        if (ok && i > it_begin) ok = load(i - 1, true);
+        if (ok && i > x.it_begin) ok = load(i - 1, true);
       }
       if (ok) ok = load(it_end - 1, true);
-      // On failure, loads already issued land on their own (bounded by the TMA);
-      // the cluster barrier at the end keeps both CTAs alive until then.
     }
+    // Every load completes on the even CTA's barriers: there, wait (bounded)
+    // for the last phase of each, so no copy into either CTA is still in
+    // flight when the cluster leaves.  Phases the consumer already waited for
+    // return at once.
+    if (leader && lane == 0) {
+      if (nq > 0) (void)mbar_wait(&sm.q_full, (nq - 1) & 1, ctl);
+      for (int s = 0; s < kStages; ++s) {
+        const uint32_t n_s = u > (uint32_t)s ? (u - (uint32_t)s + kStages - 1) / kStages : 0;
+        if (n_s > 0) (void)mbar_wait(&sm.kv_full[s], (n_s - 1) & 1, ctl);
+      }
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------- MMA issuer (even CTA only)
-    if (leader && n_it > 0) {
-      bool ok = __all_sync(0xffffffffu, wait_or_abort(&sm.q_full, 0, sm, ctl));
-      tc_fence_after();
+    if (leader) {
       const uint64_t qdesc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t kdesc0 = sdesc_sw128(smem_u32(ring), 16, 1024);
       const uint64_t vdesc0 = sdesc_sw128(smem_u32(ring), kVBlk, 1024);
+      const uint64_t pdesc0 = sdesc_sw128(smem_u32(sP), 16, 1024);
       auto commit_both = [&](uint64_t* bar) {
         umma_commit_pair(mapa_shared(smem_u32(bar), 0));
         umma_commit_pair(mapa_shared(smem_u32(bar), 1));
       };
-      uint32_t u = 0;
-      auto pv = [&](int x) -> bool {
-        const int bp = x & 1;
-        if (!__all_sync(0xffffffffu, wait_or_abort(&sm.p_full[bp], (x >> 1) & 1, sm, ctl)))
-          return false;
+      uint32_t u = 0;     // ring items consumed
+      uint32_t nq = 0;    // units started (Q loads consumed)
+      uint32_t g = 0;     // key tiles processed, across units
+      bool ok = true;
+      auto pv = [&](uint32_t x, bool first) -> bool {
+        if (!warp_wait(&sm.p_full, x & 1, sm, ctl)) return false;
+        // The unit's first PV overwrites O: the previous unit's epilogue must
+        // have read it.
+        if (first && nq > 1 && !warp_wait(&sm.o_free, (nq - 2) & 1, sm, ctl)) return false;
         const int s = (int)(u % kStages);
-        if (!__all_sync(0xffffffffu, wait_or_abort(&sm.kv_full[s], (u / kStages) & 1, sm, ctl)))
-          return false;
+        if (!warp_wait(&sm.kv_full[s], (u / kStages) & 1, sm, ctl)) return false;
         tc_fence_after();
         if (lane == 0) {
           const uint64_t vd = vdesc0 + (uint64_t)((s * kItemBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
-            // B = V[16 keys x (128 columns per CTA)], MN-major: 8-key groups
-            // 1024 B apart, 64-column blocks 16 KB apart; a K step is 16 rows.
-            umma_pair_ts(tO, tS + 128 * bp + kk * 8, vd + (uint64_t)((kk * 2048) >> 4),
-                         kIdescPV, (x > 0 || kk > 0) ? 1u : 0u);
+            // A = P[128 rows per CTA x 16 keys], K-major: 8-row groups 1024 B
+            // apart; a K step walks 32 B inside a 64-key block, then the next
+            // block.  B = V[16 keys x (128 columns per CTA)], MN-major: 8-key
+            // groups 1024 B apart, 64-column blocks 16 KB apart; a K step is
+            // 16 rows.
+            const uint32_t poff = (uint32_t)((kk >> 2) * kPBlk + (kk & 3) * 32);
+            umma_pair_ss(tO, pdesc0 + (uint64_t)(poff >> 4), vd + (uint64_t)((kk * 2048) >> 4),
+                         kIdescPV, (!first || kk > 0) ? 1u : 0u);
           }
           commit_both(&sm.kv_empty[s]);
           commit_both(&sm.o_done);
@@ -322,38 +408,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ++u;
         return true;
       };
-      for (int i = it_begin; i < it_end && ok; ++i) {
-        const int li = i - it_begin;
-        const int s = (int)(u % kStages);
-        ok = __all_sync(0xffffffffu, wait_or_abort(&sm.kv_full[s], (u / kStages) & 1, sm, ctl));
-        if (!ok) break;
-        if (li >= 2) {
-          // S[li%2] still holds P of tile li-2, the A operand of PV(li-2):
-          // this QK may only overwrite it once that PV has finished.
-          ok = __all_sync(0xffffffffu, wait_or_abort(&sm.o_done, (li - 2) & 1, sm, ctl));
-          if (!ok) break;
-        }
-        tc_fence_after();
-        if (lane == 0) {
-          const uint64_t kd = kdesc0 + (uint64_t)((s * kItemBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            // A = Q[128 rows per CTA x 16 d], B = K[64 keys per CTA x 16 d],
-            // both K-major: 8-row groups 1024 B apart; the K step walks 32 B
-            // inside a 64-column block, then the next block.
-            const uint32_t qoff = (uint32_t)((kk >> 2) * kQBlk + (kk & 3) * 32);
-            const uint32_t koff = (uint32_t)((kk >> 2) * kKBlk + (kk & 3) * 32);
-            umma_pair_ss(tS + 128 * (li & 1), qdesc0 + (uint64_t)(qoff >> 4),
-                         kd + (uint64_t)(koff >> 4), kIdescQK, kk > 0 ? 1u : 0u);
+      for (int unit = cluster; unit < n_units && ok; unit += n_clusters) {
+        const Unit x = make_unit<kSuffix>(unit, p, n_pairs, n_cache, sm, codes, list, lane);
+        if (x.n_it == 0) continue;
+        if (!warp_wait(&sm.q_full, nq & 1, sm, ctl)) break;
+        ++nq;
+        for (int li = 0; li < x.n_it && ok; ++li) {
+          const uint32_t gi = g + (uint32_t)li;
+          const int s = (int)(u % kStages);
+          if (!warp_wait(&sm.kv_full[s], (u / kStages) & 1, sm, ctl)) { ok = false; break; }
+          // S[gi%2] was last read by the softmax of tile gi-2.
+          if (gi >= 2 && !warp_wait(&sm.s_free[gi & 1], ((gi - 2) >> 1) & 1, sm, ctl)) {
+            ok = false;
+            break;
           }
-          commit_both(&sm.kv_empty[s]);
-          commit_both(&sm.s_full[li & 1]);
+          tc_fence_after();
+          if (lane == 0) {
+            const uint64_t kd = kdesc0 + (uint64_t)((s * kItemBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              // A = Q[128 rows per CTA x 16 d], B = K[64 keys per CTA x 16 d],
+              // both K-major: 8-row groups 1024 B apart; the K step walks 32 B
+              // inside a 64-column block, then the next block.
+              const uint32_t qoff = (uint32_t)((kk >> 2) * kQBlk + (kk & 3) * 32);
+              const uint32_t koff = (uint32_t)((kk >> 2) * kKBlk + (kk & 3) * 32);
+              umma_pair_ss(tS + 128 * (gi & 1), qdesc0 + (uint64_t)(qoff >> 4),
+                           kd + (uint64_t)(koff >> 4), kIdescQK, kk > 0 ? 1u : 0u);
+            }
+            commit_both(&sm.kv_empty[s]);
+            commit_both(&sm.s_full[gi & 1]);
+            if (li == x.n_it - 1) commit_both(&sm.q_empty);
+          }
+          __syncwarp();
+          ++u;
+          if (li >= 1) ok = pv(gi - 1, li == 1);
         }
-        __syncwarp();
-        ++u;
-        if (li >= 1) ok = pv(li - 1);
+        if (ok) ok = pv(g + (uint32_t)x.n_it - 1, x.n_it == 1);
+        g += (uint32_t)x.n_it;
       }
-      if (ok) ok = pv(n_it - 1);
       if (lane == 0) umma_commit_pair(smem_u32(&sm.drain));
       __syncwarp();
       (void)mbar_wait(&sm.drain, 0, ctl);
@@ -363,188 +455,245 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;             // row of this thread in the CTA
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const int tok = min(tq0 + ((int)rank * kBM + r) / p.Hq, tq1);
-    const uint32_t cq = codes[tok];
-    const uint32_t csq = cq >> 2;
-    const bool row_expert = (cq & 2u) != 0;
     const float c = p.scale_log2;                  // > 0
-    const uint32_t p_full_l0 = mapa_shared(smem_u32(&sm.p_full[0]), 0);
-    const uint32_t p_full_l1 = mapa_shared(smem_u32(&sm.p_full[1]), 0);
-    float m_run = -INFINITY;
-    float l_run = 0.f;
+    const uint32_t s_free_l0 = mapa_shared(smem_u32(&sm.s_free[0]), 0);
+    const uint32_t s_free_l1 = mapa_shared(smem_u32(&sm.s_free[1]), 0);
+    const uint32_t p_full_l = mapa_shared(smem_u32(&sm.p_full), 0);
+    const uint32_t o_free_l = mapa_shared(smem_u32(&sm.o_free), 0);
+    // This row's 128-byte lines in the two P blocks (K-major, 128-byte swizzle).
+    uint8_t* const p_row0 = sP + r * 128;
+    uint8_t* const p_row1 = sP + kPBlk + r * 128;
+    uint32_t g = 0;
+    bool store_pending = false;    // this warp's output stores may still read P
     bool ok = true;
 
-    for (int i = it_begin; i < it_end && ok; ++i) {
-      const int li = i - it_begin;
-      const int bs = li & 1;
-      if (!wait_or_abort(&sm.s_full[bs], (li >> 1) & 1, sm, ctl)) ok = false;
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      const KvTile kt = kv_tile_at<kSuffix>(sm, i, n_cache, p.P);
-      float x[kBN];
-      {
-        // all four 32-column loads in flight, one wait
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        tmem_ld32(tS + lane_off + 128 * bs, r0);
-        tmem_ld32(tS + lane_off + 128 * bs + 32, r1);
-        tmem_ld32(tS + lane_off + 128 * bs + 64, r2);
-        tmem_ld32(tS + lane_off + 128 * bs + 96, r3);
-        tmem_ld_wait();
-        reg_fence(r0);
-        reg_fence(r1);
-        reg_fence(r2);
-        reg_fence(r3);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          x[e] = __uint_as_float(r0[e]);
-          x[32 + e] = __uint_as_float(r1[e]);
-          x[64 + e] = __uint_as_float(r2[e]);
-          x[96 + e] = __uint_as_float(r3[e]);
-        }
-      }
-      if (kt.partial) {
-        const int k0 = kt.tile * kBN;
-        int e;
-        bool hole = false;
-        if (kSuffix && kt.src == 1) {
-          e = min(kBN, p.P - k0);
-        } else {
-          e = 0;
-#pragma unroll
-          for (int step = kBN; step >= 1; step >>= 1) {
-            const int probe = e + step;
-            if (probe <= kBN && (uint32_t)(codes[k0 + probe - 1] >> 2) <= csq) e = probe;
-          }
-          e = min(e, n_key_tok - k0);
-          hole = row_expert && kt.any_fast;
-        }
-        if (hole) {
-          const uint4* kc = reinterpret_cast<const uint4*>(codes + k0);
-#pragma unroll
-          for (int g = 0; g < kBN / 8; ++g) {
-            const uint4 v4 = kc[g];
-            const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-            for (int h = 0; h < 8; ++h) {
-              const int j = 8 * g + h;
-              const bool fast = ((wv[h >> 1] >> (16 * (h & 1))) & 1u) != 0;
-              x[j] = (j < e && !fast) ? x[j] : -INFINITY;
-            }
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < kBN; ++j) x[j] = j < e ? x[j] : -INFINITY;
-        }
-      }
-      float mt[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) mt[j] = fmaxf(fmaxf(x[j], x[j + 32]), fmaxf(x[j + 64], x[j + 96]));
-#pragma unroll
-      for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-        for (int j = 0; j < w; ++j) mt[j] = fmaxf(mt[j], mt[j + w]);
-      const float mx = mt[0] * c;
-
-      // Lazy rescaling (exact: O and l always share the reference max).
-      const bool upd = mx > m_run + kRescaleThreshold;
-      const float m_new = upd ? mx : m_run;
-      const float alpha = ex2(m_run - m_new);
-      const bool need_o = upd && (m_run != -INFINITY);
-      l_run *= (m_run == -INFINITY) ? 0.f : alpha;
-      m_run = m_new;
-      const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
-      float ls[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      uint32_t pk[64];
-#pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        const float p0 = ex2(fmaf(x[2 * e], c, nm));
-        const float p1 = ex2(fmaf(x[2 * e + 1], c, nm));
-        ls[e & 7] += p0 + p1;
-        pk[e] = pack_bf16x2_rna(p0, p1);
-      }
-      l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-
-      // No TMEM write of this tile (O rescale or P) may overlap PV of the
-      // previous tile: in the CTA-pair form a P store racing the running pair
-      // MMA corrupted results.  PV(li-1) has normally finished long before the
-      // exponentials above are done, so this wait is free in steady state.
-      if (li >= 1) {
-        if (!wait_or_abort(&sm.o_done, (li - 1) & 1, sm, ctl)) ok = false;
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, need_o)) {
-        const float a = need_o ? alpha : 1.f;
-#pragma unroll 1
-        for (int cc = 0; cc < kD / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tO + lane_off + 32 * cc, o);
-          tmem_ld_wait();
-          reg_fence(o);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a);
-          tmem_st32(tO + lane_off + 32 * cc, o);
-        }
-      }
-      {
-        uint32_t (&pk0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
-        uint32_t (&pk1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-        tmem_st32(tS + lane_off + 128 * bs, pk0);
-        tmem_st32(tS + lane_off + 128 * bs + 32, pk1);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(bs ? p_full_l1 : p_full_l0);
-    }
-
-    if (ok && n_it > 0) {
-      if (!wait_or_abort(&sm.o_done, (n_it - 1) & 1, sm, ctl)) ok = false;
-    }
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok && n_it > 0) {
-      tc_fence_after();
-      const long long grow = (long long)b * rows_per_b + row0 + r;
+    for (int unit = cluster; unit < n_units && ok; unit += n_clusters) {
+      const Unit x = make_unit<kSuffix>(unit, p, n_pairs, n_cache, sm, codes, list, lane);
+      const int row0 = x.pair * 2 * kBM + (int)rank * kBM;
       const bool row_valid = row0 + r < rows_per_b;
-      if (p.n_splits == 1) {
-        const float inv = 1.f / l_run;
-        // Q is dead once the last PV has finished: stage the bf16 rows there.
-        uint8_t* stage = sQ + quarter * 16384;
-#pragma unroll 1
-        for (int cc = 0; cc < kD / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tO + lane_off + 32 * cc, o);
+      const long long slot = ((long long)x.split * p.B + x.b) * rows_per_b + row0 + r;
+      if (x.n_it == 0) {
+        if (p.n_splits > 1 && row_valid) {
+          float* wml = p.ws + (long long)p.n_splits * p.B * rows_per_b * kD + slot * 2;
+          wml[0] = -INFINITY;
+          wml[1] = 0.f;
+        }
+        continue;
+      }
+      const int tok = min(x.tq0 + ((int)rank * kBM + r) / p.Hq, x.tq1);
+      const uint32_t cq = codes[tok];
+      const uint32_t csq = cq >> 2;
+      const bool row_expert = (cq & 2u) != 0;
+      float m_run = -INFINITY;
+      float l_run = 0.f;
+
+      for (int li = 0; li < x.n_it; ++li) {
+        const uint32_t gi = g + (uint32_t)li;
+        const int bs = (int)(gi & 1);
+        if (!warp_wait(&sm.s_full[bs], (gi >> 1) & 1, sm, ctl)) { ok = false; break; }
+        tc_fence_after();
+        const KvTile kt = kv_tile_at<kSuffix>(list, x.it_begin + li, n_cache, p.P);
+        float xs[kBN];
+        {
+          // all four 32-column loads in flight, one wait
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          tmem_ld32(tS + lane_off + 128 * bs, r0);
+          tmem_ld32(tS + lane_off + 128 * bs + 32, r1);
+          tmem_ld32(tS + lane_off + 128 * bs + 64, r2);
+          tmem_ld32(tS + lane_off + 128 * bs + 96, r3);
           tmem_ld_wait();
-          reg_fence(o);
-          uint32_t ob[16];
+          reg_fence(r0);
+          reg_fence(r1);
+          reg_fence(r2);
+          reg_fence(r3);
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            ob[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
-                                __uint_as_float(o[2 * e + 1]) * inv);
-          uint8_t* blk = stage + (cc >> 1) * 4096 + lane * 128;
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int unit = (cc & 1) * 4 + q4;
-            *reinterpret_cast<uint4*>(blk + ((unit ^ (lane & 7)) << 4)) =
-                make_uint4(ob[4 * q4], ob[4 * q4 + 1], ob[4 * q4 + 2], ob[4 * q4 + 3]);
+          for (int e = 0; e < 32; ++e) {
+            xs[e] = __uint_as_float(r0[e]);
+            xs[32 + e] = __uint_as_float(r1[e]);
+            xs[64 + e] = __uint_as_float(r2[e]);
+            xs[96 + e] = __uint_as_float(r3[e]);
           }
+        }
+        // S is in registers: the next QK into this buffer may start.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(bs ? s_free_l1 : s_free_l0);
+        if (kt.partial) {
+          const int k0 = kt.tile * kBN;
+          int e;
+          bool hole = false;
+          if (kSuffix && kt.src == 1) {
+            e = min(kBN, p.P - k0);
+          } else {
+            e = 0;
+#pragma unroll
+            for (int step = kBN; step >= 1; step >>= 1) {
+              const int probe = e + step;
+              if (probe <= kBN && (uint32_t)(codes[k0 + probe - 1] >> 2) <= csq) e = probe;
+            }
+            e = min(e, n_key_tok - k0);
+            hole = row_expert && kt.any_fast;
+          }
+          if (hole) {
+            const uint4* kc = reinterpret_cast<const uint4*>(codes + k0);
+#pragma unroll
+            for (int q8 = 0; q8 < kBN / 8; ++q8) {
+              const uint4 v4 = kc[q8];
+              const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+              for (int h = 0; h < 8; ++h) {
+                const int j = 8 * q8 + h;
+                const bool fast = ((wv[h >> 1] >> (16 * (h & 1))) & 1u) != 0;
+                xs[j] = (j < e && !fast) ? xs[j] : -INFINITY;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < kBN; ++j) xs[j] = j < e ? xs[j] : -INFINITY;
+          }
+        }
+        // Row maximum: eight independent chains of three-input max.
+        float m8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float a = fmax3(xs[k], xs[k + 8], xs[k + 16]);
+#pragma unroll
+          for (int i = 3; i < 15; i += 2) a = fmax3(a, xs[k + 8 * i], xs[k + 8 * i + 8]);
+          m8[k] = fmaxf(a, xs[k + 120]);
+        }
+        const float mx =
+            fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], fmax3(m8[4], m8[5], m8[6]), m8[7])) * c;
+
+        // Lazy rescaling (exact: O and l always share the reference max).
+        const bool upd = mx > m_run + kRescaleThreshold;
+        const float m_new = upd ? mx : m_run;
+        const float alpha = ex2(m_run - m_new);
+        const bool need_o = upd && (m_run != -INFINITY);
+        l_run *= (m_run == -INFINITY) ? 0.f : alpha;
+        m_run = m_new;
+        const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+        const float2 c2 = make_float2(c, c), n2 = make_float2(nm, nm);
+        float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+        uint32_t pk[64];
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          const float2 t = ffma2(make_float2(xs[2 * e], xs[2 * e + 1]), c2, n2);
+          const float2 pp = make_float2(ex2(t.x), ex2(t.y));
+          ls[e & 3] = fadd2(ls[e & 3], pp);
+          pk[e] = cvt_bf16x2(pp.x, pp.y);
+        }
+        const float2 lsum = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
+        l_run += lsum.x + lsum.y;
+
+        // PV of the previous tile reads the P buffer and accumulates into O:
+        // both must be finished before either is written again.  It has
+        // normally finished long before the exponentials above are done.
+        if (gi >= 1) {
+          if (!warp_wait(&sm.o_done, (gi - 1) & 1, sm, ctl)) { ok = false; break; }
+          tc_fence_after();
+        }
+        if (store_pending) {     // the previous unit's output stores read P
+          if (lane == 0) tma_store_wait_read();
+          __syncwarp();
+          store_pending = false;
+        }
+        const bool rescale = __any_sync(0xffffffffu, need_o);
+        if (rescale) {
+          const float a = need_o ? alpha : 1.f;
+#pragma unroll 1
+          for (int cc = 0; cc < kD / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + lane_off + 32 * cc, o);
+            tmem_ld_wait();
+            reg_fence(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a);
+            tmem_st32(tO + lane_off + 32 * cc, o);
+          }
+        }
+        // P row -> shared memory: 16-byte chunk j of the row's 128-byte line
+        // goes to chunk j ^ (row % 8) (128-byte swizzle, conflict-free).
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int sw = (j ^ (r & 7)) << 4;
+          *reinterpret_cast<uint4*>(p_row0 + sw) =
+              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          *reinterpret_cast<uint4*>(p_row1 + sw) =
+              make_uint4(pk[32 + 4 * j], pk[33 + 4 * j], pk[34 + 4 * j], pk[35 + 4 * j]);
         }
         fence_proxy_async_smem();
+        if (rescale) tmem_st_wait();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          tma_store_4d(&p.map_o, stage, 0, row0 + quarter * 32, 0, b);
-          tma_store_commit();
-          tma_store_wait_all();
+        if (lane == 0) mbar_arrive_remote(p_full_l);
+      }
+      if (!ok) break;
+
+      // ------------------------------------------------------- epilogue
+      const uint32_t g_last = g + (uint32_t)x.n_it - 1;
+      g += (uint32_t)x.n_it;
+      if (!warp_wait(&sm.o_done, g_last & 1, sm, ctl)) { ok = false; break; }
+      tc_fence_after();
+      const long long grow = (long long)x.b * rows_per_b + row0 + r;
+      if (p.n_splits == 1) {
+        const float inv = 1.f / l_run;
+        // The P buffer is free once the last PV has finished: each warp stages
+        // its own 32 rows there, 64 columns per 4 KB swizzled box, in two
+        // rounds of two boxes.
+        uint8_t* const st0 = sP + quarter * 4096;
+        uint8_t* const st1 = sP + kPBlk + quarter * 4096;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          if (half == 1) {
+            if (lane == 0) tma_store_wait_read();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int sub = 0; sub < 2; ++sub) {
+            const int col = 128 * half + 64 * sub;
+            uint32_t o0[32], o1[32];
+            tmem_ld32(tO + lane_off + col, o0);
+            tmem_ld32(tO + lane_off + col + 32, o1);
+            tmem_ld_wait();
+            reg_fence(o0);
+            reg_fence(o1);
+            uint32_t ob[32];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              ob[e] = cvt_bf16x2(__uint_as_float(o0[2 * e]) * inv,
+                                 __uint_as_float(o0[2 * e + 1]) * inv);
+              ob[16 + e] = cvt_bf16x2(__uint_as_float(o1[2 * e]) * inv,
+                                      __uint_as_float(o1[2 * e + 1]) * inv);
+            }
+            uint8_t* line = (sub ? st1 : st0) + lane * 128;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4*>(line + ((j ^ (lane & 7)) << 4)) =
+                  make_uint4(ob[4 * j], ob[4 * j + 1], ob[4 * j + 2], ob[4 * j + 3]);
+          }
+          if (half == 1) {
+            // All of O has been read: the next unit's first PV may overwrite it.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(o_free_l);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_4d(&p.map_o, st0, 0, row0 + quarter * kStageRows, 2 * half, x.b);
+            tma_store_4d(&p.map_o, st1, 0, row0 + quarter * kStageRows, 2 * half + 1, x.b);
+            tma_store_commit();
+          }
+          __syncwarp();
         }
+        store_pending = true;
         if (!kSuffix && p.lse && row_valid)
           p.lse[grow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
       } else {
         // Split-K partial: unnormalised O and (m, l) for the combine kernel.
         // tcgen05.ld is warp-collective (.sync.aligned): every lane loads,
         // only lanes holding a real row store.
-        const long long slot = ((long long)split * p.B + b) * rows_per_b + row0 + r;
         float* wo = p.ws + slot * kD;
 #pragma unroll 1
         for (int cc = 0; cc < kD / 32; ++cc) {
@@ -560,6 +709,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                               __uint_as_float(o[e + 2]), __uint_as_float(o[e + 3]));
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(o_free_l);
         if (row_valid) {
           float* wml = p.ws + (long long)p.n_splits * p.B * rows_per_b * kD + slot * 2;
           wml[0] = m_run;
@@ -567,18 +719,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (n_it == 0 && p.n_splits > 1 && row0 + r < rows_per_b) {
-      const long long slot = ((long long)split * p.B + b) * rows_per_b + row0 + r;
-      float* wml = p.ws + (long long)p.n_splits * p.B * rows_per_b * kD + slot * 2;
-      wml[0] = -INFINITY;
-      wml[1] = 0.f;
-    }
+    if (store_pending && lane == 0) tma_store_wait_read();
+    __syncwarp();
   }
 
-  // The Q load was issued before the key tiles were counted: a split with no
-  // tiles (or one that gave up) must still let both halves land before the
-  // CTAs leave.  Completed already in every other case, so this returns at once.
-  if (leader && threadIdx.x == 0) (void)mbar_wait(&sm.q_full, 0, ctl);
   // Neither CTA may leave while its partner can still signal its barriers or
   // read its shared memory; then both free their TMEM.
   __syncwarp();
@@ -626,8 +770,21 @@ __global__ void __launch_bounds__(256)
   *reinterpret_cast<uint4*>(out + row * kD + lane * 8) = pk;
 }
 
-size_t pair_smem_bytes(int n_code_tokens) {
-  return 1024 /* alignment slack */ + kOffCodes + (size_t)pad_tokens(n_code_tokens) * 2;
+// Dynamic shared memory for S code tokens: the layout plus up to 1 KB to
+// align its base, capped at the per-CTA limit (the kernel checks that its
+// aligned layout fits what it was given).
+int pair_smem_bytes(int n_code_tokens) {
+  return min(layout_bytes(n_code_tokens) + 1024, kSmemLimit);
+}
+
+int sm_count() {
+  static const int n = [] {
+    int dev = 0, v = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    return v > 0 ? v : 148;
+  }();
+  return n;
 }
 
 }  // namespace
@@ -636,21 +793,24 @@ cudaError_t launch_tc_pair(const TcParams& p, bool suffix_mode, const DevCtl& ct
                            cudaStream_t st) {
   const int rows = p.Sq * p.Hq;
   const int n_pairs = (rows + 2 * kBM - 1) / (2 * kBM);
-  dim3 grid(2 * n_pairs * p.n_splits, p.B);
-  const size_t smem = pair_smem_bytes(p.Sq);
+  const int n_units = p.B * n_pairs * p.n_splits;
+  // A batch-shared mask lets one cluster per SM pair walk many units;
+  // per-batch masks get one cluster per unit (each scans its own row).
+  const int n_clusters = p.mask_bs == 0 ? min(n_units, max(sm_count() / 2, 1)) : n_units;
+  dim3 grid(2 * n_clusters, 1);
+  const int smem = pair_smem_bytes(p.Sq);
   static const cudaError_t attr_err = [] {
-    const int most = (int)pair_smem_bytes(kMaxTokens);
     cudaError_t a = cudaFuncSetAttribute(tc_pair_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     cudaError_t b = cudaFuncSetAttribute(tc_pair_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     return a != cudaSuccess ? a : b;
   }();
   if (attr_err != cudaSuccess) return attr_err;
   if (suffix_mode) {
-    tc_pair_kernel<true><<<grid, kThreads, smem, st>>>(p, ctl);
+    tc_pair_kernel<true><<<grid, kThreads, smem, st>>>(p, ctl, smem);
   } else {
-    tc_pair_kernel<false><<<grid, kThreads, smem, st>>>(p, ctl);
+    tc_pair_kernel<false><<<grid, kThreads, smem, st>>>(p, ctl, smem);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || p.n_splits <= 1) return e;
@@ -664,16 +824,10 @@ int tc_suffix_splits(int B, int Sq, int P, int Hq) {
   // Split the key tiles over several CTA pairs only when the pairs of one
   // split would leave SMs idle: enough splits to fill the SMs once, each
   // keeping at least two key tiles, at most 8.
-  static int n_sm = [] {
-    int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
-  }();
   const int rows = Sq * Hq;
   const int n_ctas = 2 * ((rows + 2 * kBM - 1) / (2 * kBM)) * B;
   const int tiles = (P + kBN - 1) / kBN + (Sq + kBN - 1) / kBN;
-  int s = n_sm / max(n_ctas, 1);
+  int s = sm_count() / max(n_ctas, 1);
   s = min(s, tiles / 2);
   s = min(s, 8);
   return max(s, 1);
