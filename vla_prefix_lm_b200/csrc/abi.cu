@@ -64,7 +64,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // row (stride 128 B), so one box (64, box_rows, 4, 1) lands in shared memory
 // as 4 blocks of [box_rows x 64] with the 128-byte swizzle -- the operand
 // layout of the tensor-core kernels.  A box of 2 blocks brings half the
-// columns (the CTA-pair kernel's V halves).  Rows past `rows` read as zero and are
+// columns (the CTA-pair kernel's V quarters).  Rows past `rows` read as zero and are
 // clipped on stores.
 bool encode_rows(CUtensorMap* map, const void* base, uint64_t rows, uint64_t batch,
                  uint32_t box_rows, uint32_t box_blocks = 4) {
@@ -143,7 +143,7 @@ int pi_attn_prefill(const pi_attn_desc* d, const void* q, const void* k, const v
   const uint64_t rows = (uint64_t)d->Sq * d->Hq;
   if (!encode_rows(&p.map_q, q, rows, d->B, 128) ||
       !encode_rows(&p.map_k, k, d->Sq, d->B, 64) ||
-      !encode_rows(&p.map_vh, v, d->Sq, d->B, 128, 2) ||
+      !encode_rows(&p.map_vh, v, d->Sq, d->B, 64, 2) ||
       !encode_rows(&p.map_o, out, rows, d->B, 32, 1))
     return PI_ERR_CUDA;
   p.map_kc = p.map_k;
@@ -209,12 +209,12 @@ int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
   const uint64_t rows = (uint64_t)d->Sq * d->Hq;
   if (!encode_rows(&p.map_q, q_suf, rows, d->B, 128) ||
       !encode_rows(&p.map_k, k_suf, d->Sq, d->B, 64) ||
-      !encode_rows(&p.map_vh, v_suf, d->Sq, d->B, 128, 2) ||
+      !encode_rows(&p.map_vh, v_suf, d->Sq, d->B, 64, 2) ||
       !encode_rows(&p.map_o, out, rows, d->B, 32, 1))
     return PI_ERR_CUDA;
   if (d->P > 0) {
     if (!encode_rows(&p.map_kc, k_cache, d->P, d->B, 64) ||
-        !encode_rows(&p.map_vch, v_cache, d->P, d->B, 128, 2))
+        !encode_rows(&p.map_vch, v_cache, d->P, d->B, 64, 2))
       return PI_ERR_CUDA;
   } else {
     p.map_kc = p.map_k;

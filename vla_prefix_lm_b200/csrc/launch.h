@@ -42,7 +42,7 @@ struct TcParams {
   CUtensorMap map_k;    // keys (prefill: S; suffix: Sq), 64 keys x 256: box (64, 64, 4, 1)
   CUtensorMap map_kc;   // suffix mode: cached keys (P per batch); unused in prefill
   CUtensorMap map_o;    // out rows, box (64, 32, 1, 1): one 64-column block
-  CUtensorMap map_vh;   // values, 128 keys x 128 columns: box (64, 128, 2, 1)
+  CUtensorMap map_vh;   // values, 64 keys x 128 columns: box (64, 64, 2, 1)
   CUtensorMap map_vch;  // cached values, same box
   const uint8_t* ar;
   const int32_t* seg;

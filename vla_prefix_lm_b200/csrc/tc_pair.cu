@@ -5,7 +5,8 @@
 // K/V rows ("π0.5 vs MM-DiT joint attention", "joint attention 只管算子": 8
 // query heads, 1 KV head, head_dim 256, one shared KV pool).
 //
-// Per key tile of 128 keys, issued by ONE thread of the even CTA for the pair:
+// Per key tile of 128 keys, issued for the pair by two threads of the even CTA
+// (one for QK, one for PV):
 //   S = Q K^T   tcgen05.mma.cta_group::2, M = 256: A = Q rows of each CTA
 //               (its shared memory), B = K split by keys (64 per CTA)
 //   P           fp32 online softmax in each CTA, one thread per row; P is
@@ -31,22 +32,25 @@
 // partial tile is masked per row by its visible-prefix length plus, for
 // expert rows, the FAST keys.  No mask is materialised.
 //
-// Warp roles per CTA (192 threads):
+// Warp roles per CTA (224 threads):
 //   warp 0      TMA producer for this CTA's halves (both CTAs)
-//   warp 1      TMEM allocation (both CTAs, cta_group::2); MMA issue (even CTA)
+//   warp 1      TMEM allocation (both CTAs, cta_group::2); QK issue (even CTA)
 //   warps 2..5  softmax, O correction, epilogue (both CTAs, own rows)
+//   warp 6      PV issue (even CTA)
 //
 // TMEM per CTA (512 columns): O fp32 [0,256) | S0 [256,384) | S1 [384,512).
-// Shared memory per CTA: Q 64 KB | ring 3 x 32 KB (K halves [64 x 256], V
-// halves [128 x 128]) | P 32 KB ([128 rows x 128 keys] bf16, two 128-byte-
-// swizzled [128 x 64] blocks; also the output staging area) | control |
-// per-token codes.
+// Shared memory per CTA: Q 64 KB | K ring 2 x 32 KB (this CTA's 64 keys x
+// 256) | V ring 2 or 4 x 16 KB (64 keys x this CTA's 128 columns) | P 32 KB
+// ([128 rows x 128 keys] bf16, two 128-byte-swizzled [128 x 64] blocks; also
+// the output staging area) | control | per-token codes.
 //
-// Synchronisation across the pair: the even CTA owns q_full, kv_full, s_free,
-// p_full and o_free (the odd CTA's TMA loads and softmax warps arrive there
-// through cluster addresses); the MMA thread's commits arrive on the q_empty,
-// kv_empty, s_full and o_done barriers of both CTAs.  Every wait is bounded
-// (DevCtl).  Counters that index barriers and ring slots run across units.
+// Synchronisation across the pair: the even CTA owns q_full, k_full, v_full,
+// s_free, p_full and o_free (the odd CTA's TMA loads and softmax warps arrive
+// there through cluster addresses); the issuing threads' commits arrive on
+// the q_empty, k_empty, v_empty, s_full and o_done barriers of both CTAs.
+// Every wait is bounded (DevCtl).  Counters that index barriers and ring
+// slots run across units; each ring has a single consumer thread, which
+// waits on its slots in fill order.
 #include <cfloat>
 
 #include "launch.h"
@@ -56,25 +60,22 @@ namespace piattn {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr int kBM = 128;                    // query rows per CTA (256 per pair)
 constexpr int kBN = 128;                    // keys per key tile
 constexpr int kD = 256;
 constexpr int kQBlk = kBM * 128;            // [128 rows x 64 bf16] = 16 KB
 constexpr int kQBytes = 4 * kQBlk;          // 64 KB
-constexpr int kKBlk = 64 * 128;             // K half block: [64 keys x 64 d] = 8 KB
-constexpr int kVBlk = kBN * 128;            // V half block: [128 keys x 64 d] = 16 KB
-constexpr int kItemBytes = 32768;           // K half (4 x 8 KB) or V half (2 x 16 KB)
-constexpr int kStages = 3;
+constexpr int kKBlk = 64 * 128;             // K item block: [64 keys x 64 d] = 8 KB
+constexpr int kKItem = 4 * kKBlk;           // K item: this CTA's 64 keys x 256 d = 32 KB
+constexpr int kVBlk = 64 * 128;             // V item block: [64 keys x 64 d] = 8 KB
+constexpr int kVItem = 2 * kVBlk;           // V item: 64 keys x this CTA's 128 d = 16 KB
 constexpr int kPBlk = kBM * 128;            // P block: [128 rows x 64 keys] = 16 KB
 constexpr int kPBytes = 2 * kPBlk;          // 32 KB
 constexpr int kStageRows = 32;              // output rows staged per softmax warp
 constexpr int kOffQ = 0;
 constexpr int kOffRing = kQBytes;
-constexpr int kOffP = kOffRing + kStages * kItemBytes;
-constexpr int kOffCtl = kOffP + kPBytes;
-constexpr int kMaxKeyTiles = (kMaxTokens + kBN - 1) / kBN + 2;
-constexpr int kLists = kThreads / 32;       // one private tile list per warp
+constexpr int kLists = 6;                   // tile lists of warps 0 and 2..5
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: P stays <= 256
 constexpr int kSmemLimit = 232448;          // 227 KB per CTA on sm_100
 
@@ -86,17 +87,37 @@ constexpr uint16_t kTilePartial = 0x8000;
 constexpr uint16_t kTileAnyFast = 0x4000;
 constexpr uint16_t kTileIndex = 0x3FFF;
 
+// Shared-memory layout: a ring of kK K items (32 KB) and a ring of kV V
+// items (16 KB, half a key tile each), and up to kMaxTok tokens of per-token
+// codes.  Each ring has one consumer thread.  Four V slots (two key tiles)
+// fit beside Q and P only for short sequences.
+template <int kK_, int kV_, int kMaxTok_>
+struct Layout {
+  static constexpr int kK = kK_;
+  static constexpr int kV = kV_;
+  static constexpr int kMaxTok = kMaxTok_;
+  static constexpr int kMaxKeyTiles = (kMaxTok + kBN - 1) / kBN + 2;
+  static constexpr int kOffV = kOffRing + kK * kKItem;
+  static constexpr int kOffP = kOffV + kV * kVItem;
+  static constexpr int kOffCtl = kOffP + kPBytes;
+};
+
+template <class L>
 struct __align__(8) Smem {
+  static constexpr int kMaxKeyTiles = L::kMaxKeyTiles;
   uint64_t q_full;               // even CTA: both Q halves landed (one phase per unit)
   uint64_t q_empty;              // each CTA: the unit's last QK has read Q
-  uint64_t kv_full[kStages];     // even CTA: both halves of a K or V item landed
-  uint64_t kv_empty[kStages];    // each CTA: its ring stage may be refilled
+  uint64_t k_full[L::kK];        // even CTA: both CTAs' K items landed
+  uint64_t k_empty[L::kK];       // each CTA: its K slot may be refilled
+  uint64_t v_full[L::kV];        // even CTA: both CTAs' V items landed
+  uint64_t v_empty[L::kV];       // each CTA: its V slot may be refilled
   uint64_t s_full[2];            // each CTA: S tile in its TMEM
   uint64_t s_free[2];            // even CTA: the pair's 8 softmax warps have read S
   uint64_t p_full;               // even CTA: P written by the pair's 8 softmax warps
   uint64_t o_done;               // each CTA: PV finished
   uint64_t o_free;               // even CTA: the pair's softmax warps have read O
-  uint64_t drain;
+  uint64_t drain_qk;             // even CTA: every QK issued has completed
+  uint64_t drain_pv;             // even CTA: every PV issued has completed
   uint32_t tmem_base;
   int abort;
   int scan[kThreads / 32];
@@ -106,15 +127,23 @@ struct __align__(8) Smem {
   uint8_t tile_fast[kMaxKeyTiles];
 };
 
-constexpr int kOffCodes = kOffCtl + ((int)sizeof(Smem) + 127) / 128 * 128;
+template <class L>
+__host__ __device__ constexpr int off_codes() {
+  return L::kOffCtl + ((int)sizeof(Smem<L>) + 127) / 128 * 128;
+}
 
 __host__ __device__ constexpr int pad_tokens(int n) { return (n + 127) / 128 * 128; }
 
-// Bytes the kernel's layout needs past a 1024-byte aligned base.
+// Bytes a layout needs past a 1024-byte aligned base.
+template <class L>
 __host__ __device__ constexpr int layout_bytes(int n_code_tokens) {
-  return kOffCodes + pad_tokens(n_code_tokens) * 2;
+  return off_codes<L>() + pad_tokens(n_code_tokens) * 2;
 }
-static_assert(layout_bytes(kMaxTokens) <= kSmemLimit, "shared-memory layout too large");
+
+using LayoutLong = Layout<2, 2, kMaxTokens>;   // any length
+using LayoutShort = Layout<2, 4, 768>;         // short sequences (<= 768 tokens)
+static_assert(layout_bytes<LayoutLong>(kMaxTokens) <= kSmemLimit, "layout too large");
+static_assert(layout_bytes<LayoutShort>(768) + 1024 <= kSmemLimit, "short layout too large");
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -122,15 +151,15 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Smem& sm,
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* abort,
                                               const DevCtl& ctl) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (*(volatile int*)&sm.abort) return false;
+    if (*(volatile int*)abort) return false;
     if ((unsigned long long)(clock64() - t0) > ctl.wait_limit) {
       record_status(ctl, kStatusTimeout);
-      *(volatile int*)&sm.abort = 1;
+      *(volatile int*)abort = 1;
       return false;
     }
   }
@@ -138,9 +167,10 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Sm
 }
 
 // Warp-uniform bounded wait: every lane polls, all lanes get the same answer.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Smem& sm,
+template <class SmemT>
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, SmemT& sm,
                                           const DevCtl& ctl) {
-  return __all_sync(0xffffffffu, wait_or_abort(bar, parity, sm, ctl));
+  return __all_sync(0xffffffffu, wait_or_abort(bar, parity, &sm.abort, ctl));
 }
 
 struct KvTile {
@@ -170,7 +200,8 @@ struct Unit {
 //   full    every query sees every key (no per-element predicate)
 //   partial per-row visible prefix, FAST hole for expert rows
 // Returns the number of entries (the same in every lane).
-__device__ int build_tile_list(const Smem& sm, const uint16_t* codes, int tq0, int tq1,
+template <class SmemT>
+__device__ int build_tile_list(const SmemT& sm, const uint16_t* codes, int tq0, int tq1,
                                int n_key_tok, uint16_t* list, int lane) {
   const int n_ktiles = (n_key_tok + kBN - 1) / kBN;
   int any_e = 0, all_e = 1;
@@ -197,7 +228,7 @@ __device__ int build_tile_list(const Smem& sm, const uint16_t* codes, int tq0, i
       else c = 2;
     }
     const unsigned m = __ballot_sync(0xffffffffu, c != 0);
-    if (c != 0) {
+    if (c != 0 && list != nullptr) {
       const int pos = base + __popc(m & ((1u << lane) - 1));
       list[pos] = (uint16_t)(t | (c == 2 ? kTilePartial : 0) | (any_f ? kTileAnyFast : 0));
     }
@@ -208,9 +239,9 @@ __device__ int build_tile_list(const Smem& sm, const uint16_t* codes, int tq0, i
 }
 
 // Warp-collective: the unit with index u and this warp's tile list for it.
-template <bool kSuffix>
+template <bool kSuffix, class SmemT>
 __device__ __forceinline__ Unit make_unit(int u, const TcParams& p, int n_pairs, int n_cache,
-                                          const Smem& sm, const uint16_t* codes, uint16_t* list,
+                                          const SmemT& sm, const uint16_t* codes, uint16_t* list,
                                           int lane) {
   Unit x;
   x.split = u % p.n_splits;
@@ -228,22 +259,25 @@ __device__ __forceinline__ Unit make_unit(int u, const TcParams& p, int n_pairs,
   return x;
 }
 
-template <bool kSuffix>
+template <bool kSuffix, class L>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_pair_kernel(const __grid_constant__ TcParams p, const DevCtl ctl, int smem_bytes) {
+  using SmemT = Smem<L>;
+  constexpr int kK = L::kK, kV = L::kV;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   // Both CTAs see the same base offset, so both leave here or neither does.
-  if ((int)(smem - smem_raw) + layout_bytes(p.Sq) > smem_bytes) {
+  if ((int)(smem - smem_raw) + layout_bytes<L>(p.Sq) > smem_bytes || p.Sq > L::kMaxTok) {
     if (threadIdx.x == 0) record_status(ctl, kStatusUnsupported);
     return;
   }
-  Smem& sm = *reinterpret_cast<Smem*>(smem + kOffCtl);
-  uint16_t* codes = reinterpret_cast<uint16_t*>(smem + kOffCodes);
+  SmemT& sm = *reinterpret_cast<SmemT*>(smem + L::kOffCtl);
+  uint16_t* codes = reinterpret_cast<uint16_t*>(smem + off_codes<L>());
   uint8_t* sQ = smem + kOffQ;
-  uint8_t* ring = smem + kOffRing;
-  uint8_t* sP = smem + kOffP;
+  uint8_t* kring = smem + kOffRing;
+  uint8_t* vring = smem + L::kOffV;
+  uint8_t* sP = smem + L::kOffP;
 
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -268,9 +302,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_empty, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
+    for (int s = 0; s < kK; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < kV; ++s) {
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.s_full[s], 1);
@@ -279,7 +317,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(&sm.p_full, 8);
     mbar_init(&sm.o_done, 1);
     mbar_init(&sm.o_free, 8);
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain_qk, 1);
+    mbar_init(&sm.drain_pv, 1);
     sm.abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&p.map_q);
@@ -293,6 +332,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   // Both CTAs' barriers must exist before either side signals the other.
   cluster_sync();
+  // With a single split every unit visits at least one key tile (a query
+  // always sees its own token), so the first unit's Q can load during the
+  // mask scan.
+  const bool early_q = p.n_splits == 1;
+  if (early_q && threadIdx.x == 0) {
+    const int pair0 = cluster % n_pairs, b0 = cluster / n_pairs;
+    if (leader) mbar_arrive_expect_tx(&sm.q_full, 2 * kQBytes);
+    tma_load_4d_pair(sQ, &p.map_q, mapa_shared(smem_u32(&sm.q_full), 0), 0,
+                     pair0 * 2 * kBM + (int)rank * kBM, 0, b0);
+  }
   if (warp == 1) {
     tmem_alloc_pair(&sm.tmem_base, 512);
     tmem_relinquish_pair();
@@ -306,52 +355,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   const uint32_t tO = tmem + kColO;
   const uint32_t tS = tmem + kColS;      // S[b] at +128*b
-  uint16_t* list = sm.list[warp];
+  // Warps 1 and 6 (the MMA issuers) only need the tile count.
+  uint16_t* list = (warp == 0 || (warp >= 2 && warp <= 5)) ? sm.list[warp] : nullptr;
 
   if (warp == 0) {
     // ------------------------------------------------- producer (both CTAs)
+    // Per unit: Q, then K0, K1, and for each tile j: K(j+2), V(j) keys 0-63,
+    // V(j) keys 64-127.  Each ring is filled and consumed in order.
     const uint32_t q_full_l = mapa_shared(smem_u32(&sm.q_full), 0);
-    uint32_t u = 0;                 // ring items issued
+    uint32_t uk = 0, uv = 0;        // K / V items issued
     uint32_t nq = 0;                // Q loads issued
     bool ok = true;
     for (int unit = cluster; unit < n_units && ok; unit += n_clusters) {
       const Unit x = make_unit<kSuffix>(unit, p, n_pairs, n_cache, sm, codes, list, lane);
       if (x.n_it == 0) continue;
       const int row0 = x.pair * 2 * kBM + (int)rank * kBM;
-      if (nq > 0 && !warp_wait(&sm.q_empty, (nq - 1) & 1, sm, ctl)) break;
-      if (lane == 0) {
-        if (leader) mbar_arrive_expect_tx(&sm.q_full, 2 * kQBytes);
-        tma_load_4d_pair(sQ, &p.map_q, q_full_l, 0, row0, 0, x.b);
-      }
-      __syncwarp();
-      ++nq;
-      auto load = [&](int idx, bool is_v) -> bool {
-        const KvTile kt = kv_tile_at<kSuffix>(list, idx, n_cache, p.P);
-        const int s = (int)(u % kStages);
-        const uint32_t rel = u / kStages;
-        if (rel > 0 && !warp_wait(&sm.kv_empty[s], (rel - 1) & 1, sm, ctl)) return false;
+      if (nq > 0 || !early_q) {      // else the first Q was issued before the scan
+        if (nq > 0 && !warp_wait(&sm.q_empty, (nq - 1) & 1, sm, ctl)) break;
         if (lane == 0) {
-          const uint32_t full_l = mapa_shared(smem_u32(&sm.kv_full[s]), 0);
-          if (leader) mbar_arrive_expect_tx(&sm.kv_full[s], 2 * kItemBytes);
-          uint8_t* dst = ring + s * kItemBytes;
-          if (!is_v) {   // this CTA's 64 keys of the tile, all 256 columns
-            const CUtensorMap* map = kt.src ? &p.map_kc : &p.map_k;
-            tma_load_4d_pair(dst, map, full_l, 0, kt.tile * kBN + 64 * (int)rank, 0, x.b);
-          } else {       // all 128 keys of the tile, this CTA's 128 columns
-            const CUtensorMap* map = kt.src ? &p.map_vch : &p.map_vh;
-            tma_load_4d_pair(dst, map, full_l, 0, kt.tile * kBN, 2 * (int)rank, x.b);
-          }
+          if (leader) mbar_arrive_expect_tx(&sm.q_full, 2 * kQBytes);
+          tma_load_4d_pair(sQ, &p.map_q, q_full_l, 0, row0, 0, x.b);
         }
         __syncwarp();
-        ++u;
+      }
+      ++nq;
+      auto load_k = [&](int idx) -> bool {
+        const KvTile kt = kv_tile_at<kSuffix>(list, idx, n_cache, p.P);
+        const int s = (int)(uk % kK);
+        const uint32_t rel = uk / kK;
+        if (rel > 0 && !warp_wait(&sm.k_empty[s], (rel - 1) & 1, sm, ctl)) return false;
+        if (lane == 0) {
+          if (leader) mbar_arrive_expect_tx(&sm.k_full[s], 2 * kKItem);
+          // this CTA's 64 keys of the tile, all 256 columns
+          tma_load_4d_pair(kring + s * kKItem, kt.src ? &p.map_kc : &p.map_k,
+                           mapa_shared(smem_u32(&sm.k_full[s]), 0), 0,
+                           kt.tile * kBN + 64 * (int)rank, 0, x.b);
+        }
+        __syncwarp();
+        ++uk;
         return true;
       };
-      const int it_end = x.it_begin + x.n_it;
-      for (int i = x.it_begin; i < it_end && ok; ++i) {
-        ok = load(i, false);
-        if (ok && i > x.it_begin) ok = load(i - 1, true);
+      auto load_v = [&](int idx, int h) -> bool {
+        const KvTile kt = kv_tile_at<kSuffix>(list, idx, n_cache, p.P);
+        const int s = (int)(uv % kV);
+        const uint32_t rel = uv / kV;
+        if (rel > 0 && !warp_wait(&sm.v_empty[s], (rel - 1) & 1, sm, ctl)) return false;
+        if (lane == 0) {
+          if (leader) mbar_arrive_expect_tx(&sm.v_full[s], 2 * kVItem);
+          // keys [64h, 64h + 64) of the tile, this CTA's 128 columns
+          tma_load_4d_pair(vring + s * kVItem, kt.src ? &p.map_vch : &p.map_vh,
+                           mapa_shared(smem_u32(&sm.v_full[s]), 0), 0, kt.tile * kBN + 64 * h,
+                           2 * (int)rank, x.b);
+        }
+        __syncwarp();
+        ++uv;
+        return true;
+      };
+      const int i0 = x.it_begin, n = x.n_it;
+      ok = load_k(i0);
+      if (ok && n > 1) ok = load_k(i0 + 1);
+      for (int j = 0; j < n && ok; ++j) {
+        if (j + 2 < n) ok = load_k(i0 + j + 2);
+        if (ok) ok = load_v(i0 + j, 0);
+        if (ok) ok = load_v(i0 + j, 1);
       }
-      if (ok) ok = load(it_end - 1, true);
     }
     // Every load completes on the even CTA's barriers: there, wait (bounded)
     // for the last phase of each, so no copy into either CTA is still in
@@ -359,96 +426,121 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // return at once.
     if (leader && lane == 0) {
       if (nq > 0) (void)mbar_wait(&sm.q_full, (nq - 1) & 1, ctl);
-      for (int s = 0; s < kStages; ++s) {
-        const uint32_t n_s = u > (uint32_t)s ? (u - (uint32_t)s + kStages - 1) / kStages : 0;
-        if (n_s > 0) (void)mbar_wait(&sm.kv_full[s], (n_s - 1) & 1, ctl);
+      for (int s = 0; s < kK; ++s) {
+        const uint32_t n_s = uk > (uint32_t)s ? (uk - (uint32_t)s + kK - 1) / kK : 0;
+        if (n_s > 0) (void)mbar_wait(&sm.k_full[s], (n_s - 1) & 1, ctl);
+      }
+      for (int s = 0; s < kV; ++s) {
+        const uint32_t n_s = uv > (uint32_t)s ? (uv - (uint32_t)s + kV - 1) / kV : 0;
+        if (n_s > 0) (void)mbar_wait(&sm.v_full[s], (n_s - 1) & 1, ctl);
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------- MMA issuer (even CTA only)
+  } else if (warp == 1 || warp == 6) {
+    // ------------------------- MMA issuers (even CTA only): QK by warp 1, PV by warp 6
+    // Two issuing threads, so a PV that waits for its P never holds back the
+    // QK of a later tile and vice versa.  Each accumulation chain (S of one
+    // tile, O of one unit) and each ring belongs to one thread: tcgen05
+    // ordering and commit tracking are per thread.
     if (leader) {
-      const uint64_t qdesc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t kdesc0 = sdesc_sw128(smem_u32(ring), 16, 1024);
-      const uint64_t vdesc0 = sdesc_sw128(smem_u32(ring), kVBlk, 1024);
-      const uint64_t pdesc0 = sdesc_sw128(smem_u32(sP), 16, 1024);
       auto commit_both = [&](uint64_t* bar) {
         umma_commit_pair(mapa_shared(smem_u32(bar), 0));
         umma_commit_pair(mapa_shared(smem_u32(bar), 1));
       };
-      uint32_t u = 0;     // ring items consumed
-      uint32_t nq = 0;    // units started (Q loads consumed)
       uint32_t g = 0;     // key tiles processed, across units
+      uint32_t nu = 0;    // units started
       bool ok = true;
-      auto pv = [&](uint32_t x, bool first) -> bool {
-        if (!warp_wait(&sm.p_full, x & 1, sm, ctl)) return false;
-        // The unit's first PV overwrites O: the previous unit's epilogue must
-        // have read it.
-        if (first && nq > 1 && !warp_wait(&sm.o_free, (nq - 2) & 1, sm, ctl)) return false;
-        const int s = (int)(u % kStages);
-        if (!warp_wait(&sm.kv_full[s], (u / kStages) & 1, sm, ctl)) return false;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint64_t vd = vdesc0 + (uint64_t)((s * kItemBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            // A = P[128 rows per CTA x 16 keys], K-major: 8-row groups 1024 B
-            // apart; a K step walks 32 B inside a 64-key block, then the next
-            // block.  B = V[16 keys x (128 columns per CTA)], MN-major: 8-key
-            // groups 1024 B apart, 64-column blocks 16 KB apart; a K step is
-            // 16 rows.
-            const uint32_t poff = (uint32_t)((kk >> 2) * kPBlk + (kk & 3) * 32);
-            umma_pair_ss(tO, pdesc0 + (uint64_t)(poff >> 4), vd + (uint64_t)((kk * 2048) >> 4),
-                         kIdescPV, (!first || kk > 0) ? 1u : 0u);
-          }
-          commit_both(&sm.kv_empty[s]);
-          commit_both(&sm.o_done);
-        }
-        __syncwarp();
-        ++u;
-        return true;
-      };
-      for (int unit = cluster; unit < n_units && ok; unit += n_clusters) {
-        const Unit x = make_unit<kSuffix>(unit, p, n_pairs, n_cache, sm, codes, list, lane);
-        if (x.n_it == 0) continue;
-        if (!warp_wait(&sm.q_full, nq & 1, sm, ctl)) break;
-        ++nq;
-        for (int li = 0; li < x.n_it && ok; ++li) {
-          const uint32_t gi = g + (uint32_t)li;
-          const int s = (int)(u % kStages);
-          if (!warp_wait(&sm.kv_full[s], (u / kStages) & 1, sm, ctl)) { ok = false; break; }
-          // S[gi%2] was last read by the softmax of tile gi-2.
-          if (gi >= 2 && !warp_wait(&sm.s_free[gi & 1], ((gi - 2) >> 1) & 1, sm, ctl)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (lane == 0) {
-            const uint64_t kd = kdesc0 + (uint64_t)((s * kItemBytes) >> 4);
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              // A = Q[128 rows per CTA x 16 d], B = K[64 keys per CTA x 16 d],
-              // both K-major: 8-row groups 1024 B apart; the K step walks 32 B
-              // inside a 64-column block, then the next block.
-              const uint32_t qoff = (uint32_t)((kk >> 2) * kQBlk + (kk & 3) * 32);
-              const uint32_t koff = (uint32_t)((kk >> 2) * kKBlk + (kk & 3) * 32);
-              umma_pair_ss(tS + 128 * (gi & 1), qdesc0 + (uint64_t)(qoff >> 4),
-                           kd + (uint64_t)(koff >> 4), kIdescQK, kk > 0 ? 1u : 0u);
+      if (warp == 1) {
+        const uint64_t qdesc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+        const uint64_t kdesc0 = sdesc_sw128(smem_u32(kring), 16, 1024);
+        uint32_t uk = 0;
+        for (int unit = cluster; unit < n_units && ok; unit += n_clusters) {
+          const Unit x = make_unit<kSuffix>(unit, p, n_pairs, n_cache, sm, codes, list, lane);
+          if (x.n_it == 0) continue;
+          if (!warp_wait(&sm.q_full, nu & 1, sm, ctl)) break;
+          ++nu;
+          for (int j = 0; j < x.n_it; ++j) {
+            const uint32_t gi = g + (uint32_t)j;
+            const int s = (int)(uk % kK);
+            if (!warp_wait(&sm.k_full[s], (uk / kK) & 1, sm, ctl)) { ok = false; break; }
+            // S[gi%2] was last read by the softmax of tile gi-2.
+            if (gi >= 2 && !warp_wait(&sm.s_free[gi & 1], ((gi - 2) >> 1) & 1, sm, ctl)) {
+              ok = false;
+              break;
             }
-            commit_both(&sm.kv_empty[s]);
-            commit_both(&sm.s_full[gi & 1]);
-            if (li == x.n_it - 1) commit_both(&sm.q_empty);
+            tc_fence_after();
+            if (lane == 0) {
+              const uint64_t kd = kdesc0 + (uint64_t)((s * kKItem) >> 4);
+#pragma unroll
+              for (int kk = 0; kk < kD / 16; ++kk) {
+                // A = Q[128 rows per CTA x 16 d], B = K[64 keys per CTA x 16 d],
+                // both K-major: 8-row groups 1024 B apart; the K step walks
+                // 32 B inside a 64-column block, then the next block.
+                const uint32_t qoff = (uint32_t)((kk >> 2) * kQBlk + (kk & 3) * 32);
+                const uint32_t koff = (uint32_t)((kk >> 2) * kKBlk + (kk & 3) * 32);
+                umma_pair_ss(tS + 128 * (gi & 1), qdesc0 + (uint64_t)(qoff >> 4),
+                             kd + (uint64_t)(koff >> 4), kIdescQK, kk > 0 ? 1u : 0u);
+              }
+              commit_both(&sm.k_empty[s]);
+              commit_both(&sm.s_full[gi & 1]);
+              if (j == x.n_it - 1) commit_both(&sm.q_empty);   // the unit's last QK read Q
+            }
+            __syncwarp();
+            ++uk;
           }
-          __syncwarp();
-          ++u;
-          if (li >= 1) ok = pv(gi - 1, li == 1);
+          g += (uint32_t)x.n_it;
         }
-        if (ok) ok = pv(g + (uint32_t)x.n_it - 1, x.n_it == 1);
-        g += (uint32_t)x.n_it;
+        if (lane == 0) umma_commit_pair(smem_u32(&sm.drain_qk));
+        __syncwarp();
+        (void)mbar_wait(&sm.drain_qk, 0, ctl);
+      } else {
+        const uint64_t pdesc0 = sdesc_sw128(smem_u32(sP), 16, 1024);
+        const uint64_t vdesc0 = sdesc_sw128(smem_u32(vring), kVBlk, 1024);
+        uint32_t uv = 0;
+        for (int unit = cluster; unit < n_units && ok; unit += n_clusters) {
+          const Unit x = make_unit<kSuffix>(unit, p, n_pairs, n_cache, sm, codes, list, lane);
+          if (x.n_it == 0) continue;
+          ++nu;
+          for (int j = 0; j < x.n_it && ok; ++j) {
+            const uint32_t gi = g + (uint32_t)j;
+            if (!warp_wait(&sm.p_full, gi & 1, sm, ctl)) { ok = false; break; }
+            // The unit's first PV overwrites O: the previous unit's epilogue
+            // must have read it.
+            if (j == 0 && nu > 1 && !warp_wait(&sm.o_free, (nu - 2) & 1, sm, ctl)) {
+              ok = false;
+              break;
+            }
+            for (int h = 0; h < 2 && ok; ++h) {
+              const int s = (int)(uv % kV);
+              if (!warp_wait(&sm.v_full[s], (uv / kV) & 1, sm, ctl)) { ok = false; break; }
+              tc_fence_after();
+              if (lane == 0) {
+                const uint64_t vd = vdesc0 + (uint64_t)((s * kVItem) >> 4);
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                  // A = P[128 rows per CTA x 16 keys], K-major: 8-row groups
+                  // 1024 B apart; a K step walks 32 B inside a 64-key block.
+                  // B = V[16 keys x (128 columns per CTA)], MN-major: 8-key
+                  // groups 1024 B apart, 64-column blocks 8 KB apart; a K
+                  // step is 16 rows.
+                  const uint32_t poff = (uint32_t)(h * kPBlk + k4 * 32);
+                  umma_pair_ss(tO, pdesc0 + (uint64_t)(poff >> 4),
+                               vd + (uint64_t)((k4 * 2048) >> 4), kIdescPV,
+                               (j > 0 || h > 0 || k4 > 0) ? 1u : 0u);
+                }
+                commit_both(&sm.v_empty[s]);
+                if (h == 1) commit_both(&sm.o_done);
+              }
+              __syncwarp();
+              ++uv;
+            }
+          }
+          g += (uint32_t)x.n_it;
+        }
+        if (lane == 0) umma_commit_pair(smem_u32(&sm.drain_pv));
+        __syncwarp();
+        (void)mbar_wait(&sm.drain_pv, 0, ctl);
       }
-      if (lane == 0) umma_commit_pair(smem_u32(&sm.drain));
-      __syncwarp();
-      (void)mbar_wait(&sm.drain, 0, ctl);
     }
   } else {
     // ------------------------------------ softmax / epilogue (both CTAs)
@@ -773,8 +865,19 @@ __global__ void __launch_bounds__(256)
 // Dynamic shared memory for S code tokens: the layout plus up to 1 KB to
 // align its base, capped at the per-CTA limit (the kernel checks that its
 // aligned layout fits what it was given).
+template <class L>
 int pair_smem_bytes(int n_code_tokens) {
-  return min(layout_bytes(n_code_tokens) + 1024, kSmemLimit);
+  return min(layout_bytes<L>(n_code_tokens) + 1024, kSmemLimit);
+}
+
+template <bool kSuffix, class L>
+cudaError_t launch_pair(const TcParams& p, const DevCtl& ctl, dim3 grid, cudaStream_t st) {
+  static const cudaError_t attr_err = cudaFuncSetAttribute(
+      tc_pair_kernel<kSuffix, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+  if (attr_err != cudaSuccess) return attr_err;
+  const int smem = pair_smem_bytes<L>(p.Sq);
+  tc_pair_kernel<kSuffix, L><<<grid, kThreads, smem, st>>>(p, ctl, smem);
+  return cudaGetLastError();
 }
 
 int sm_count() {
@@ -798,21 +901,11 @@ cudaError_t launch_tc_pair(const TcParams& p, bool suffix_mode, const DevCtl& ct
   // per-batch masks get one cluster per unit (each scans its own row).
   const int n_clusters = p.mask_bs == 0 ? min(n_units, max(sm_count() / 2, 1)) : n_units;
   dim3 grid(2 * n_clusters, 1);
-  const int smem = pair_smem_bytes(p.Sq);
-  static const cudaError_t attr_err = [] {
-    cudaError_t a = cudaFuncSetAttribute(tc_pair_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-    cudaError_t b = cudaFuncSetAttribute(tc_pair_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-    return a != cudaSuccess ? a : b;
-  }();
-  if (attr_err != cudaSuccess) return attr_err;
-  if (suffix_mode) {
-    tc_pair_kernel<true><<<grid, kThreads, smem, st>>>(p, ctl, smem);
-  } else {
-    tc_pair_kernel<false><<<grid, kThreads, smem, st>>>(p, ctl, smem);
-  }
-  cudaError_t e = cudaGetLastError();
+  const bool short_s = p.Sq <= LayoutShort::kMaxTok;
+  cudaError_t e = suffix_mode ? (short_s ? launch_pair<true, LayoutShort>(p, ctl, grid, st)
+                                         : launch_pair<true, LayoutLong>(p, ctl, grid, st))
+                              : (short_s ? launch_pair<false, LayoutShort>(p, ctl, grid, st)
+                                         : launch_pair<false, LayoutLong>(p, ctl, grid, st));
   if (e != cudaSuccess || p.n_splits <= 1) return e;
   const long long n_rows = (long long)p.B * rows;
   combine_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, st>>>(
