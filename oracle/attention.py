@@ -28,6 +28,11 @@ Conventions (readings the pages leave open):
 * ``scale`` multiplies the dot product before the softmax (the pages never state
   it; the workloads fold 1/sqrt(d) into q and k and use scale = 1).
 * ``lse`` is the natural-log log-sum-exp of the scaled, visible scores.
+* Padding (not in the pages' workloads; openpi and Pi0-FAST AND a per-token
+  validity mask into the attention mask): a negative segment id marks a
+  padding token.  A padding key is visible to no query and a padding query
+  sees no key.  A query row with no visible key outputs 0 with lse = -inf.
+  In the suffix pass a per-batch ``cache_valid`` mask hides padded prefix keys.
 """
 
 from __future__ import annotations
@@ -38,6 +43,7 @@ import numpy as np
 OTHER = 0   # prefix (image patches, text, discrete state) or anything else
 FAST = 1    # FAST discrete action tokens
 EXPERT = 2  # the action expert's continuous chunk
+PAD = -1    # any negative id: a padding token
 
 
 def _as_batched(x, B, name):
@@ -82,38 +88,48 @@ def prefill_mask(ar, seg=None, B=None, rows=None):
         seg = _as_batched(seg, B, "seg")
         forbid = (seg[:, qi, None] == EXPERT) & (seg[:, None, :] == FAST)
         M = M & ~forbid
+        valid = seg >= 0                                 # padding: negative ids
+        M = M & valid[:, qi, None] & valid[:, None, :]
     return M
 
 
-def suffix_mask(ar_suf, P, B=None):
+def suffix_mask(ar_suf, P, B=None, seg_suf=None, cache_valid=None):
     """[B, Sq, P + Sq] visibility of the suffix-only pass against a P-token cache.
 
     "VLA 代码精读 - OpenPI & StarVLA", 1.6: every suffix query sees every (valid)
     prefix key -- the prefix mask repeated over the suffix rows -- concatenated
     on the key axis with make_attn_mask over the suffix tokens alone.
+    ``cache_valid`` ([P] or [B, P], nonzero = valid) hides padded prefix keys;
+    ``seg_suf`` tags the suffix tokens as in ``prefill_mask`` (negative =
+    padding).
     """
     ar_suf = np.asarray(ar_suf)
     if B is None:
         B = ar_suf.shape[0] if ar_suf.ndim == 2 else 1
-    Msuf = prefill_mask(ar_suf, None, B=B)               # [B, Sq, Sq]
+    Msuf = prefill_mask(ar_suf, seg_suf, B=B)            # [B, Sq, Sq]
     Sq = Msuf.shape[1]
     pre = np.ones((B, Sq, P), dtype=bool)
+    if cache_valid is not None:
+        cv = _as_batched(np.asarray(cache_valid) != 0, B, "cache_valid")
+        pre = pre & cv[:, None, :]
+    if seg_suf is not None:
+        vq = _as_batched(seg_suf, B, "seg_suf") >= 0
+        pre = pre & vq[:, :, None]
     return np.concatenate([pre, Msuf], axis=2)
 
 
 def softmax_probs(s, M):
     """Row softmax of the scores ``s`` restricted to the visible entries ``M``.
 
-    Masked entries get probability exactly 0.  A row with no visible entry
-    would be 0/0; such rows cannot arise from the cumsum rule (every token sees
-    itself) and raise here.
+    Masked entries get probability exactly 0.  A row with no visible entry (a
+    padding query) has all probabilities 0.
     """
     s = np.where(M, s, -np.inf)
     m = s.max(axis=-1, keepdims=True)
-    if not np.all(np.isfinite(m)):
-        raise ValueError("a query row has no visible key")
-    e = np.exp(s - m)
-    return e / e.sum(axis=-1, keepdims=True)
+    empty = ~np.isfinite(m)
+    e = np.exp(s - np.where(empty, 0.0, m))
+    den = e.sum(axis=-1, keepdims=True)
+    return np.where(empty, 0.0, e / np.where(empty, 1.0, den))
 
 
 def attention(q, k, v, M, scale=1.0, rows=None):
@@ -145,6 +161,9 @@ def attention(q, k, v, M, scale=1.0, rows=None):
             p = softmax_probs(s[None, :], M[b, i][None, :])[0]
             o[h] = p @ v[b, :, kv, :]
             vis = s[M[b, i]]
+            if vis.size == 0:
+                lse[h] = -np.inf
+                continue
             mx = vis.max()
             lse[h] = mx + np.log(np.exp(vis - mx).sum())
         return o, lse
@@ -164,7 +183,11 @@ def attention(q, k, v, M, scale=1.0, rows=None):
             out[b, :, h, :] = p @ v[b, :, kv, :]
             sm = np.where(M[b], s, -np.inf)
             mx = sm.max(axis=-1, keepdims=True)
-            lse[b, :, h] = (mx + np.log(np.exp(sm - mx).sum(axis=-1, keepdims=True)))[:, 0]
+            empty = ~np.isfinite(mx)
+            mxf = np.where(empty, 0.0, mx)
+            with np.errstate(divide="ignore"):
+                lse_b = mxf + np.log(np.exp(sm - mxf).sum(axis=-1, keepdims=True))
+            lse[b, :, h] = np.where(empty, -np.inf, lse_b)[:, 0]
     return out, lse
 
 
@@ -179,16 +202,17 @@ def prefill(q, k, v, ar, seg=None, scale=1.0, rows=None):
     return attention(q, k, v, M, scale, rows)
 
 
-def suffix(q_suf, k_suf, v_suf, k_cache, v_cache, ar_suf, scale=1.0, rows=None):
+def suffix(q_suf, k_suf, v_suf, k_cache, v_cache, ar_suf, scale=1.0, rows=None,
+           seg_suf=None, cache_valid=None):
     """Suffix-only pass: suffix queries against [prefix cache, suffix] keys.
 
     "VLA 代码精读 - OpenPI & StarVLA", 1.6 Pi0.sample_actions: the keys are the
     cached prefix keys followed by this step's suffix keys; the cache is not
-    extended.
+    extended.  ``seg_suf`` / ``cache_valid`` add padding as in ``suffix_mask``.
     """
     B = q_suf.shape[0]
     P = np.asarray(k_cache).shape[1]
-    M = suffix_mask(ar_suf, P, B=B)
+    M = suffix_mask(ar_suf, P, B=B, seg_suf=seg_suf, cache_valid=cache_valid)
     k = np.concatenate([np.asarray(k_cache, np.float64), np.asarray(k_suf, np.float64)], axis=1)
     v = np.concatenate([np.asarray(v_cache, np.float64), np.asarray(v_suf, np.float64)], axis=1)
     return attention(q_suf, k, v, M, scale, rows)

@@ -13,6 +13,7 @@ Sources (page title, section):
   attention with the tokens before them.
 * "π0.5 vs MM-DiT joint attention", permission table: expert queries never read
   FAST keys; every other row follows the block structure.
+* Padding (negative segment id): a padding token is neither read nor reads.
 """
 
 from __future__ import annotations
@@ -28,6 +29,8 @@ def visible(i, j, ar, seg=None):
     boundary (a True ar entry) lies in (i, j]: the key is then in the query's
     own bidirectional block.
     """
+    if seg is not None and (seg[i] < 0 or seg[j] < 0):
+        return False
     if seg is not None and seg[i] == EXPERT and seg[j] == FAST:
         return False
     if j <= i:
@@ -56,6 +59,8 @@ def attention_row(q_row, keys, values, vis, scale=1.0):
     for j, kj in enumerate(keys):
         if vis[j]:
             scores.append((j, scale * sum(a * b for a, b in zip(q_row, kj))))
+    if not scores:                 # a padding query: no visible key
+        return [0.0] * len(q_row)
     mx = max(s for _, s in scores)
     w = [(j, math.exp(s - mx)) for j, s in scores]
     den = sum(x for _, x in w)

@@ -403,3 +403,124 @@ def test_planted_value_mistakes_are_caught():
     # transposed mask
     bad_t, _ = oracle.attention(q, k, v, np.swapaxes(M, 1, 2), 0.5)
     assert np.abs(bad_t - ref).max() > 1e-3
+
+
+# ---------------------------------------------------------------- padding
+# A negative segment id marks a padding token (openpi and Pi0-FAST AND a
+# per-token validity mask into the attention mask; the workloads have none).
+# The pins below tie the padded oracle to what padding must mean: a padding
+# token behaves exactly as if it were absent, and a query row that sees no
+# key outputs 0 with lse = -inf.
+
+def _rand_qkv(rng, B, S, Hq=2, d=8):
+    q = rng.standard_normal((B, S, Hq, d))
+    k = rng.standard_normal((B, S, 1, d))
+    v = rng.standard_normal((B, S, 1, d))
+    return q, k, v
+
+
+def test_padding_brute_force_all_patterns():
+    """Exhaustive: every ar pattern (S <= 7) with random pad / FAST / EXPERT tags."""
+    rng = np.random.default_rng(11)
+    for S in range(1, 8):
+        for bits in itertools.product([0, 1], repeat=S):
+            ar = np.array(bits, dtype=np.uint8)
+            seg = rng.integers(-1, 3, size=S)
+            got = oracle.prefill_mask(ar, seg)[0]
+            want = np.array(brute.mask(ar, seg))
+            assert np.array_equal(got, want), (ar, seg)
+
+
+def test_padding_equals_removing_the_tokens():
+    """Pad tokens with ar = False anywhere in the sequence: every valid row's
+    output equals the oracle on the sequence with the pad tokens deleted, and
+    pad rows are 0 with lse = -inf."""
+    rng = np.random.default_rng(12)
+    for trial in range(20):
+        S = int(rng.integers(2, 40))
+        ar = (rng.random(S) < 0.25).astype(np.uint8)
+        seg = rng.choice([OTHER, FAST, EXPERT], size=S)
+        pad = rng.random(S) < 0.3
+        ar[pad] = 0
+        seg_p = np.where(pad, -1, seg)
+        q, k, v = _rand_qkv(rng, 1, S)
+        out, lse = oracle.prefill(q, k, v, ar, seg_p, scale=0.7)
+        keep = ~pad
+        if keep.any():
+            o2, l2 = oracle.prefill(q[:, keep], k[:, keep], v[:, keep], ar[keep], seg[keep],
+                                    scale=0.7)
+            np.testing.assert_allclose(out[:, keep], o2, atol=1e-12)
+            np.testing.assert_allclose(lse[:, keep], l2, atol=1e-12)
+        assert np.all(out[:, pad] == 0.0)
+        assert np.all(np.isneginf(lse[:, pad]))
+
+
+def test_padding_matches_torch_sdpa_on_valid_rows():
+    rng = np.random.default_rng(13)
+    B, S, Hq, d = 2, 30, 4, 16
+    ar = (rng.random((B, S)) < 0.2).astype(np.uint8)
+    seg = np.where(rng.random((B, S)) < 0.25, -1, 0)
+    q, k, v = _rand_qkv(rng, B, S, Hq, d)
+    out, _ = oracle.prefill(q, k, v, ar, seg)
+    M = oracle.prefill_mask(ar, seg)
+    for b in range(B):
+        rows = np.nonzero(M[b].any(axis=1))[0]
+        qt = torch.from_numpy(q[b].transpose(1, 0, 2)[:, rows])          # [Hq, R, d]
+        kt = torch.from_numpy(np.repeat(k[b].transpose(1, 0, 2), Hq, 0))  # [Hq, S, d]
+        vt = torch.from_numpy(np.repeat(v[b].transpose(1, 0, 2), Hq, 0))
+        mt = torch.from_numpy(M[b][rows])
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mt,
+                                                               scale=1.0)
+        np.testing.assert_allclose(out[b, rows].transpose(1, 0, 2), ref.numpy(), atol=1e-12)
+
+
+def test_suffix_cache_padding_equals_removing_cache_rows():
+    rng = np.random.default_rng(14)
+    B, P, Sq, Hq, d = 3, 37, 9, 2, 8
+    ar = np.zeros(Sq, np.uint8); ar[0] = 1; ar[1] = 1
+    q = rng.standard_normal((B, Sq, Hq, d))
+    ks = rng.standard_normal((B, Sq, 1, d)); vs = rng.standard_normal((B, Sq, 1, d))
+    kc = rng.standard_normal((B, P, 1, d)); vc = rng.standard_normal((B, P, 1, d))
+    valid = rng.random((B, P)) < 0.6
+    valid[2] = False                         # a batch element whose cache is all padding
+    out, lse = oracle.suffix(q, ks, vs, kc, vc, ar, cache_valid=valid)
+    for b in range(B):
+        keep = valid[b]
+        o2, l2 = oracle.suffix(q[b:b + 1], ks[b:b + 1], vs[b:b + 1], kc[b:b + 1, keep],
+                               vc[b:b + 1, keep], ar)
+        np.testing.assert_allclose(out[b:b + 1], o2, atol=1e-12)
+        np.testing.assert_allclose(lse[b:b + 1], l2, atol=1e-12)
+
+
+def test_suffix_token_padding_rows_are_zero():
+    rng = np.random.default_rng(15)
+    B, P, Sq, Hq, d = 1, 12, 6, 2, 8
+    ar = np.array([1, 1, 0, 0, 0, 0], np.uint8)
+    seg = np.array([0, 0, 0, -1, 0, -1])
+    q = rng.standard_normal((B, Sq, Hq, d))
+    ks = rng.standard_normal((B, Sq, 1, d)); vs = rng.standard_normal((B, Sq, 1, d))
+    kc = rng.standard_normal((B, P, 1, d)); vc = rng.standard_normal((B, P, 1, d))
+    out, lse = oracle.suffix(q, ks, vs, kc, vc, ar, seg_suf=seg)
+    assert np.all(out[:, seg < 0] == 0.0) and np.all(np.isneginf(lse[:, seg < 0]))
+    keep = seg >= 0
+    o2, _ = oracle.suffix(q[:, keep], ks[:, keep], vs[:, keep], kc, vc, ar[keep])
+    np.testing.assert_allclose(out[:, keep], o2, atol=1e-12)
+
+
+def test_planted_padding_mistakes_are_caught():
+    """A padding term that forgets the query side, or the key side, fails."""
+    rng = np.random.default_rng(16)
+    S = 12
+    ar = (rng.random(S) < 0.3).astype(np.uint8)
+    seg = np.where(rng.random(S) < 0.3, -1, 0)
+    seg[0] = -1
+    seg[5] = -1
+    good = oracle.prefill_mask(ar, seg)[0]
+    base = oracle.prefill_mask(ar, None)[0]
+    valid = seg >= 0
+    keys_only = base & valid[None, :]
+    rows_only = base & valid[:, None]
+    brute_m = np.array(brute.mask(ar, seg))
+    assert np.array_equal(good, brute_m)
+    assert not np.array_equal(keys_only, brute_m)
+    assert not np.array_equal(rows_only, brute_m)
