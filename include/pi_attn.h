@@ -26,8 +26,9 @@
  * Memory layout (all entry points): every tensor is a dense, contiguous,
  * caller-owned DEVICE buffer in token-major order [B, S, H, d] (d innermost,
  * then heads, then tokens, then batch).  ar_mask is uint8 (0 = False,
- * nonzero = True); segment_ids is int32 (PI_SEG_*; any other value is treated
- * as PI_SEG_OTHER).  Both are [S] rows, one per batch element at a distance of
+ * nonzero = True); segment_ids is int32 (PI_SEG_*; a negative value marks a
+ * padding token, any other unknown value is treated as PI_SEG_OTHER).  Both
+ * are [S] rows, one per batch element at a distance of
  * desc->mask_batch_stride elements (0 = one row shared by the whole batch).
  *
  * Ownership and threading: the library never allocates, frees or retains a
@@ -73,10 +74,21 @@ enum pi_status {
 };
 
 enum pi_segment {
+  PI_SEG_PAD = -1,   /* any negative id: a padding token (see below)     */
   PI_SEG_OTHER = 0,  /* prefix: image patches, text, discrete state      */
   PI_SEG_FAST = 1,   /* FAST discrete action tokens                      */
   PI_SEG_EXPERT = 2  /* the action expert's continuous chunk             */
 };
+
+/*
+ * Padding.  The pages' workloads have none, but openpi ANDs a per-token
+ * validity mask (input_mask) into the attention mask ("VLA 代码精读 - OpenPI &
+ * StarVLA", 1.5 Pi0.compute_loss; also "Pi0-FAST 模型架构", 2.3).  Here a
+ * padding token (negative segment id) is visible to no query and its own
+ * query row sees no key.  A query row with no visible key writes out = 0 and
+ * lse = -inf.  In the suffix pass, pi_attn_suffix_masked additionally takes a
+ * per-batch validity mask for the cached prefix keys.
+ */
 
 typedef struct pi_attn_desc {
   int32_t B;    /* batch size (B == 0 is a no-op)                            */
@@ -108,11 +120,13 @@ typedef struct pi_attn_desc {
  *   q    [B, S, Hq, d]     (S = desc->Sq, desc->P must be 0)
  *   k, v [B, S, Hkv, d]
  *   ar_mask     [B or 1, S] uint8            (required)
- *   segment_ids [B or 1, S] int32 or NULL    (NULL: no expert<-FAST rule)
+ *   segment_ids [B or 1, S] int32 or NULL    (NULL: no expert<-FAST rule, no
+ *                                             padding; negative = padding)
  *   out  [B, S, Hq, d]  same dtype as q      (written)
  *   lse  [B, S, Hq] fp32 or NULL             (natural-log log-sum-exp of the
  *                                             scaled visible scores; written)
- * Every query sees at least itself, so no row is empty.
+ * Every non-padding query sees at least itself; a padding row writes 0 and
+ * lse = -inf.
  */
 int pi_attn_prefill(const pi_attn_desc* desc, const void* q, const void* k, const void* v,
                     const uint8_t* ar_mask, const int32_t* segment_ids, void* out, float* lse,
@@ -144,12 +158,29 @@ int pi_attn_suffix(const pi_attn_desc* desc, const void* q_suf, const void* k_su
 size_t pi_attn_suffix_workspace_bytes(const pi_attn_desc* desc);
 
 /*
+ * pi_attn_suffix_masked -- pi_attn_suffix with padding (see "Padding" above).
+ *   segment_ids_suf [B or 1, Sq] int32 or NULL: tags of the suffix tokens, at
+ *     desc->mask_batch_stride like ar_mask_suf; negative = padding.  The
+ *     expert<-FAST rule applies among suffix tokens as in the prefill.
+ *   cache_valid [B, P] uint8 or NULL: nonzero = the cached prefix key is valid;
+ *     invalid keys are visible to no suffix query.  NULL = every key valid.
+ * Everything else (arguments, layout, workspace, errors) as pi_attn_suffix,
+ * which is this call with both masks NULL.  segment_ids_suf must be 4-byte
+ * aligned (PI_ERR_ALIGN).
+ */
+int pi_attn_suffix_masked(const pi_attn_desc* desc, const void* q_suf, const void* k_suf,
+                          const void* v_suf, const void* k_cache, const void* v_cache,
+                          const uint8_t* ar_mask_suf, const int32_t* segment_ids_suf,
+                          const uint8_t* cache_valid, void* out, void* workspace,
+                          size_t ws_bytes, pi_stream_t stream);
+
+/*
  * pi_attn_debug_mask -- writes the visibility matrix the kernels evaluate, as
  * uint8 0/1, for bit-exact comparison with an explicitly built mask.
  * Uses the same in-kernel predicate (cumsum of ar_mask, the expert<-FAST
  * rule, and the suffix-pass prefix columns) as the attention kernels.
- *   mode 0 (prefill): mask_out [B, Sq, Sq];      seg may be NULL
- *   mode 1 (suffix) : mask_out [B, Sq, P + Sq];  seg must be NULL
+ *   mode 0 (prefill): mask_out [B, Sq, Sq];      seg may be NULL (negative = padding)
+ *   mode 1 (suffix) : mask_out [B, Sq, P + Sq];  seg must be NULL (no cache mask)
  * Only desc->B, Sq, P and mask_batch_stride are read.
  */
 int pi_attn_debug_mask(const pi_attn_desc* desc, int mode, const uint8_t* ar_mask,

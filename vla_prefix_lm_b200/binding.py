@@ -32,6 +32,7 @@ EXPORTED = (
     "pi_attn_status_string",
     "pi_attn_set_wait_limit",
     "pi_attn_selftest_wait",
+    "pi_attn_suffix_masked",
     "pi_attn_suffix_noalloc",
     "pi_attn_suffix_noalloc_capacity",
 )
@@ -86,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.pi_attn_set_wait_limit.restype = ctypes.c_uint64
         L.pi_attn_selftest_wait.argtypes = [vp]
         L.pi_attn_selftest_wait.restype = i32
+        L.pi_attn_suffix_masked.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.pi_attn_suffix_masked.restype = i32
         L.pi_attn_suffix_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.pi_attn_suffix_noalloc.restype = i32
         L.pi_attn_suffix_noalloc_capacity.argtypes = []
@@ -183,11 +186,14 @@ def pi_attn_suffix_workspace_bytes(q_suf, k_suf, k_cache, ar_mask_suf, softmax_s
 
 
 def pi_attn_suffix(q_suf, k_suf, v_suf, k_cache, v_cache, ar_mask_suf, out=None,
-                   workspace=None, softmax_scale=1.0, stream=None):
+                   workspace=None, softmax_scale=1.0, stream=None, segment_ids=None,
+                   cache_valid=None):
     """Suffix-only pass.  q_suf [B,Sq,Hq,d]; k_suf, v_suf [B,Sq,Hkv,d];
     k_cache, v_cache [B,P,Hkv,d]; ar_mask_suf uint8 [Sq] or [B,Sq].
     ``workspace``: a CUDA uint8 tensor of at least pi_attn_suffix_workspace_bytes
-    (allocated here if None and needed)."""
+    (allocated here if None and needed).  ``segment_ids`` (int32, same layout
+    as ar_mask_suf; negative = padding) and ``cache_valid`` (uint8 [B,P],
+    nonzero = valid) select pi_attn_suffix_masked."""
     _need(q_suf, "q_suf", dims=4)
     _need(k_suf, "k_suf", q_suf.dtype, 4)
     _need(v_suf, "v_suf", q_suf.dtype, 4)
@@ -205,11 +211,27 @@ def pi_attn_suffix(q_suf, k_suf, v_suf, k_cache, v_cache, ar_mask_suf, out=None,
         out = torch.empty_like(q_suf)
     _need(out, "out", q_suf.dtype, 4)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = lib().pi_attn_suffix(ctypes.byref(desc), _ptr(q_suf), _ptr(k_suf), _ptr(v_suf),
-                              _ptr(k_cache), _ptr(v_cache), _ptr(ar_mask_suf), _ptr(out),
-                              _ptr(workspace), ws_bytes, ctypes.c_void_p(_stream(stream)))
+    if segment_ids is None and cache_valid is None:
+        rc = lib().pi_attn_suffix(ctypes.byref(desc), _ptr(q_suf), _ptr(k_suf), _ptr(v_suf),
+                                  _ptr(k_cache), _ptr(v_cache), _ptr(ar_mask_suf), _ptr(out),
+                                  _ptr(workspace), ws_bytes, ctypes.c_void_p(_stream(stream)))
+        if rc != PI_OK:
+            raise PiAttnError(rc, "pi_attn_suffix")
+        return out
+    if segment_ids is not None:
+        _need(segment_ids, "segment_ids", torch.int32)
+        if segment_ids.shape != ar_mask_suf.shape:
+            raise ValueError("segment_ids must have the layout of ar_mask_suf")
+    if cache_valid is not None:
+        _need(cache_valid, "cache_valid", torch.uint8)
+        if k_cache is None or tuple(cache_valid.shape) != tuple(k_cache.shape[:2]):
+            raise ValueError("cache_valid must be [B, P]")
+    rc = lib().pi_attn_suffix_masked(ctypes.byref(desc), _ptr(q_suf), _ptr(k_suf), _ptr(v_suf),
+                                     _ptr(k_cache), _ptr(v_cache), _ptr(ar_mask_suf),
+                                     _ptr(segment_ids), _ptr(cache_valid), _ptr(out),
+                                     _ptr(workspace), ws_bytes, ctypes.c_void_p(_stream(stream)))
     if rc != PI_OK:
-        raise PiAttnError(rc, "pi_attn_suffix")
+        raise PiAttnError(rc, "pi_attn_suffix_masked")
     return out
 
 

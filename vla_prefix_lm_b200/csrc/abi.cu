@@ -167,10 +167,11 @@ size_t pi_attn_suffix_workspace_bytes(const pi_attn_desc* d) {
   return tc_suffix_workspace_bytes(d->B, d->Sq, d->P, d->Hq);
 }
 
-int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
-                   const void* v_suf, const void* k_cache, const void* v_cache,
-                   const uint8_t* ar_mask_suf, void* out, void* workspace, size_t ws_bytes,
-                   pi_stream_t stream) {
+int pi_attn_suffix_masked(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
+                          const void* v_suf, const void* k_cache, const void* v_cache,
+                          const uint8_t* ar_mask_suf, const int32_t* segment_ids_suf,
+                          const uint8_t* cache_valid, void* out, void* workspace,
+                          size_t ws_bytes, pi_stream_t stream) {
   int rc = check_desc(d, true);
   if (rc != PI_OK) return rc;
   if (d->B == 0 || d->Sq == 0) return PI_OK;
@@ -179,6 +180,8 @@ int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
   if (!aligned16(q_suf) || !aligned16(k_suf) || !aligned16(v_suf) || !aligned16(out) ||
       (d->P > 0 && (!aligned16(k_cache) || !aligned16(v_cache))))
     return PI_ERR_ALIGN;
+  if (segment_ids_suf && (reinterpret_cast<uintptr_t>(segment_ids_suf) & 3u)) return PI_ERR_ALIGN;
+  if (d->P == 0) cache_valid = nullptr;
   DevCtl ctl;
   if (!make_ctl(&ctl)) return PI_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -190,10 +193,11 @@ int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
     p.kc = static_cast<const float*>(k_cache);
     p.vc = static_cast<const float*>(v_cache);
     p.ar = ar_mask_suf;
-    p.seg = nullptr;
+    p.seg = segment_ids_suf;
     p.mask_bs = d->mask_batch_stride;
     p.out = static_cast<float*>(out);
     p.lse = nullptr;
+    p.cache_valid = cache_valid;
     p.B = d->B; p.Sq = d->Sq; p.P = d->P; p.Hq = d->Hq; p.Hkv = d->Hkv; p.d = d->d;
     p.scale = d->softmax_scale;
     return launched(launch_simt_f32(p, ctl, st));
@@ -221,9 +225,10 @@ int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
     p.map_vch = p.map_vh;
   }
   p.ar = ar_mask_suf;
-  p.seg = nullptr;
+  p.seg = segment_ids_suf;
   p.mask_bs = d->mask_batch_stride;
   p.lse = nullptr;
+  p.cache_valid = cache_valid;
   p.ws = static_cast<float*>(workspace);
   p.out_ptr = out;
   p.B = d->B; p.Sq = d->Sq; p.P = d->P; p.Hq = d->Hq;
@@ -231,6 +236,14 @@ int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
   p.scale = d->softmax_scale;
   p.scale_log2 = d->softmax_scale * 1.4426950408889634f;
   return launched(launch_tc_pair(p, true, ctl, st));
+}
+
+int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
+                   const void* v_suf, const void* k_cache, const void* v_cache,
+                   const uint8_t* ar_mask_suf, void* out, void* workspace, size_t ws_bytes,
+                   pi_stream_t stream) {
+  return pi_attn_suffix_masked(d, q_suf, k_suf, v_suf, k_cache, v_cache, ar_mask_suf, nullptr,
+                               nullptr, out, workspace, ws_bytes, stream);
 }
 
 int pi_attn_debug_mask(const pi_attn_desc* d, int mode, const uint8_t* ar_mask,

@@ -22,6 +22,7 @@ struct SimtParams {
   long long mask_bs;
   float* out;
   float* lse;
+  const uint8_t* cache_valid;  // suffix mode: [B, P] nonzero = valid cached key; may be null
   int B, Sq, P, Hq, Hkv, d;
   float scale;
 };
@@ -48,6 +49,7 @@ struct TcParams {
   const int32_t* seg;
   long long mask_bs;
   float* lse;           // prefill only; may be null
+  const uint8_t* cache_valid;  // suffix mode: [B, P] nonzero = valid cached key; may be null
   float* ws;            // split-K partials (suffix mode); may be null
   void* out_ptr;        // bf16 output rows (written by the combine kernel under split-K)
   int B, Sq, P, Hq;

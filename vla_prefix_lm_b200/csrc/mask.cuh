@@ -10,11 +10,17 @@
 // keys are visible to every suffix query; suffix keys follow the rule over the
 // suffix tokens alone.
 //
+// Padding (not in the pages' workloads; openpi and Pi0-FAST AND a per-token
+// validity mask into the attention mask): a negative segment id marks a
+// padding token, which no query reads and which reads no key.
+//
 // Encoding.  Each token carries one packed code:
-//     code = (cs << 2) | (is_expert << 1) | is_fast
-// so that   visible(cq, ck) = (ck >> 2) <= (cq >> 2) && !((cq & 2) && (ck & 1)).
-// Cached prefix keys get code 0, which every query code admits.  cs <= S, so
-// S <= 16383 keeps a code within 16 bits.
+//     code = (cs << 2) | (is_expert << 1) | is_fast,   padding: both flag bits
+// so that   visible(cq, ck) = neither is padding
+//                             && (ck >> 2) <= (cq >> 2) && !((cq & 2) && (ck & 1)).
+// (Padding keys also carry the FAST bit, so the expert rule alone already
+// hides them from expert queries.)  Cached prefix keys get code 0, which every
+// non-padding query admits.  cs <= S, so S <= 16383 keeps a code in 16 bits.
 #pragma once
 #include <cstdint>
 
@@ -25,11 +31,14 @@ constexpr int kSegExpert = 2;
 constexpr int kMaxTokens = 16383;
 
 __host__ __device__ __forceinline__ uint32_t make_code(uint32_t cs, int seg) {
+  if (seg < 0) return (cs << 2) | 3u;
   return (cs << 2) | (seg == kSegExpert ? 2u : 0u) | (seg == kSegFast ? 1u : 0u);
 }
 
+__host__ __device__ __forceinline__ bool is_pad(uint32_t code) { return (code & 3u) == 3u; }
+
 __host__ __device__ __forceinline__ bool visible(uint32_t cq, uint32_t ck) {
-  return (ck >> 2) <= (cq >> 2) && !((cq & 2u) && (ck & 1u));
+  return !is_pad(cq) && !is_pad(ck) && (ck >> 2) <= (cq >> 2) && !((cq & 2u) && (ck & 1u));
 }
 
 // Block-wide inclusive scan of (ar != 0) over one batch row of S tokens,
@@ -88,6 +97,7 @@ __device__ __forceinline__ uint32_t nonzero_byte_bits(uint32_t w) {
 
 // The ar_mask bits and segment flags of 32 consecutive tokens starting at t0
 // (16-byte vector loads when aligned).  Tokens at or past S read as False / 0.
+// A padding token sets both its fast and its expert bit.
 struct Flags32 {
   uint32_t bits, fast, expert;
 };
@@ -116,16 +126,16 @@ __device__ __forceinline__ Flags32 load_flags32(const uint8_t* __restrict__ ar,
         const int sv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-          f.fast |= (sv[h] == kSegFast ? 1u : 0u) << (4 * g + h);
-          f.expert |= (sv[h] == kSegExpert ? 1u : 0u) << (4 * g + h);
+          f.fast |= (sv[h] == kSegFast || sv[h] < 0 ? 1u : 0u) << (4 * g + h);
+          f.expert |= (sv[h] == kSegExpert || sv[h] < 0 ? 1u : 0u) << (4 * g + h);
         }
       }
     } else {
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const int sv = t0 + i < S ? seg[t0 + i] : 0;
-        f.fast |= (sv == kSegFast ? 1u : 0u) << i;
-        f.expert |= (sv == kSegExpert ? 1u : 0u) << i;
+        f.fast |= (sv == kSegFast || sv < 0 ? 1u : 0u) << i;
+        f.expert |= (sv == kSegExpert || sv < 0 ? 1u : 0u) << i;
       }
     }
   }
@@ -141,11 +151,12 @@ __device__ __forceinline__ Flags32 load_flags32(const uint8_t* __restrict__ ar,
 // ints.  Every thread of the block must call it; it ends with a block barrier.
 // Per-128-token summaries the tile classifier needs: the block index (cs) of
 // the tile's first token, the largest cs in it, and whether it holds any /
-// only FAST tokens.
+// only FAST tokens (padding counts as FAST there), and whether it holds any /
+// only padding tokens.
 struct TileSums {
   uint16_t* cs_first;
   uint16_t* cs_last;
-  uint8_t* fast;   // bit 0: any FAST token, bit 1: all tokens FAST
+  uint8_t* fast;   // bit 0: any FAST, bit 1: all FAST, bit 2: any padding, bit 3: all padding
 };
 
 template <int kThreads>
@@ -200,20 +211,25 @@ __device__ void build_codes_x32(const uint8_t* __restrict__ ar, const int32_t* _
       // Four consecutive lanes own one 128-token tile: combine their parts.
       const int nv = min(max(S - t0, 0), 32);                 // valid tokens here
       const uint32_t vmask = nv >= 32 ? 0xFFFFFFFFu : ((1u << nv) - 1u);
+      const uint32_t pad = f.fast & f.expert;
       uint32_t any_f = (f.fast & vmask) != 0u ? 1u : 0u;
       uint32_t all_f = (f.fast & vmask) == vmask ? 1u : 0u;   // vacuous when nv == 0
+      uint32_t any_p = (pad & vmask) != 0u ? 1u : 0u;
+      uint32_t all_p = (pad & vmask) == vmask ? 1u : 0u;
       uint32_t cs_hi = nv > 0 ? (uint32_t)excl + (uint32_t)__popc(f.bits & vmask) : 0u;
 #pragma unroll
       for (int off = 1; off < 4; off <<= 1) {
         any_f |= __shfl_xor_sync(0xffffffffu, any_f, off);
         all_f &= __shfl_xor_sync(0xffffffffu, all_f, off);
+        any_p |= __shfl_xor_sync(0xffffffffu, any_p, off);
+        all_p &= __shfl_xor_sync(0xffffffffu, all_p, off);
         cs_hi = max(cs_hi, __shfl_xor_sync(0xffffffffu, cs_hi, off));
       }
       if ((lane & 3) == 0 && t0 < S) {
         const int tile = t0 >> 7;
         sums.cs_first[tile] = (uint16_t)((uint32_t)excl + (f.bits & 1u));
         sums.cs_last[tile] = (uint16_t)cs_hi;
-        sums.fast[tile] = (uint8_t)(any_f | (all_f << 1));
+        sums.fast[tile] = (uint8_t)(any_f | (all_f << 1) | (any_p << 2) | (all_p << 3));
       }
     }
     carry += total;

@@ -49,7 +49,8 @@ __global__ void __launch_bounds__(kSimtThreads)
     for (int j = 0; j < Sk; ++j) {
       const float* krow;
       const float* vrow;
-      if (j < p.P) {  // cached prefix key: visible to every suffix query
+      if (j < p.P) {  // cached prefix key: visible to every valid suffix query
+        if (is_pad(cq) || (p.cache_valid && p.cache_valid[(long long)b * p.P + j] == 0)) continue;
         krow = p.kc + (((long long)b * p.P + j) * p.Hkv + g) * D;
         vrow = p.vc + (((long long)b * p.P + j) * p.Hkv + g) * D;
       } else {
@@ -71,11 +72,12 @@ __global__ void __launch_bounds__(kSimtThreads)
       for (int c = 0; c < C; ++c) acc[c] = fmaf(acc[c], corr, e * vrow[lane + 32 * c]);
       m = m_new;
     }
-    const float inv = 1.f / l;
+    const float inv = l > 0.f ? 1.f / l : 0.f;   // no visible key (padding): 0
     float* orow = p.out + (((long long)b * p.Sq + i) * p.Hq + h) * D;
 #pragma unroll
     for (int c = 0; c < C; ++c) orow[lane + 32 * c] = acc[c] * inv;
-    if (p.lse && lane == 0) p.lse[((long long)b * p.Sq + i) * p.Hq + h] = m + logf(l);
+    if (p.lse && lane == 0)
+      p.lse[((long long)b * p.Sq + i) * p.Hq + h] = l > 0.f ? m + logf(l) : -INFINITY;
   }
 }
 

@@ -85,7 +85,8 @@ constexpr uint32_t kColO = 0, kColS = 256;
 
 constexpr uint16_t kTilePartial = 0x8000;
 constexpr uint16_t kTileAnyFast = 0x4000;
-constexpr uint16_t kTileIndex = 0x3FFF;
+constexpr uint16_t kTileAnyPad = 0x2000;
+constexpr uint16_t kTileIndex = 0x1FFF;
 
 // Shared-memory layout: a ring of kK K items (32 KB) and a ring of kV V
 // items (16 KB, half a key tile each), and up to kMaxTok tokens of per-token
@@ -178,13 +179,18 @@ struct KvTile {
   int tile;
   bool partial;
   bool any_fast;
+  bool any_pad;
 };
 
+// Cached tiles are partial when ragged or when the cache has a validity mask.
 template <bool kSuffix>
-__device__ __forceinline__ KvTile kv_tile_at(const uint16_t* list, int idx, int n_cache, int P) {
-  if (kSuffix && idx < n_cache) return KvTile{1, idx, (idx + 1) * kBN > P, false};
+__device__ __forceinline__ KvTile kv_tile_at(const uint16_t* list, int idx, int n_cache, int P,
+                                             bool cache_masked) {
+  if (kSuffix && idx < n_cache)
+    return KvTile{1, idx, cache_masked || (idx + 1) * kBN > P, false, false};
   const uint16_t e = list[kSuffix ? idx - n_cache : idx];
-  return KvTile{0, (int)(e & kTileIndex), (e & kTilePartial) != 0, (e & kTileAnyFast) != 0};
+  return KvTile{0, (int)(e & kTileIndex), (e & kTilePartial) != 0, (e & kTileAnyFast) != 0,
+                (e & kTileAnyPad) != 0};
 }
 
 // One work unit: a (batch, pair tile, key split) triple, plus its key range.
@@ -218,19 +224,24 @@ __device__ int build_tile_list(const SmemT& sm, const uint16_t* codes, int tq0, 
     const int t = t0 + lane;
     int c = 0;
     bool any_f = false;
+    bool any_p = false;
     if (t < n_ktiles) {
       const uint32_t csk0 = sm.tile_cs_first[t], csk1 = sm.tile_cs_last[t];
-      any_f = (sm.tile_fast[t] & 1) != 0;
-      const bool all_f = (sm.tile_fast[t] & 2) != 0;
+      const uint32_t fl = sm.tile_fast[t];
+      any_f = (fl & 1) != 0;
+      const bool all_f = (fl & 2) != 0;
+      any_p = (fl & 4) != 0;
+      const bool all_p = (fl & 8) != 0;
       const bool complete = (t + 1) * kBN <= n_key_tok;
-      if (csk0 > csq1 || (all_e && all_f)) c = 0;
-      else if (csk1 <= csq0 && !(any_e && any_f) && complete) c = 1;
+      if (csk0 > csq1 || (all_e && all_f) || all_p) c = 0;
+      else if (csk1 <= csq0 && !(any_e && any_f) && !any_p && complete) c = 1;
       else c = 2;
     }
     const unsigned m = __ballot_sync(0xffffffffu, c != 0);
     if (c != 0 && list != nullptr) {
       const int pos = base + __popc(m & ((1u << lane) - 1));
-      list[pos] = (uint16_t)(t | (c == 2 ? kTilePartial : 0) | (any_f ? kTileAnyFast : 0));
+      list[pos] = (uint16_t)(t | (c == 2 ? kTilePartial : 0) | (any_f ? kTileAnyFast : 0) |
+                             (any_p ? kTileAnyPad : 0));
     }
     base += __popc(m);
   }
@@ -251,7 +262,15 @@ __device__ __forceinline__ Unit make_unit(int u, const TcParams& p, int n_pairs,
   const int tok_per_pair = 2 * kBM / p.Hq;
   x.tq0 = x.pair * tok_per_pair;
   x.tq1 = min(x.tq0 + tok_per_pair, p.Sq) - 1;
-  const int n_list = build_tile_list(sm, codes, x.tq0, x.tq1, p.Sq, list, lane);
+  int n_list = build_tile_list(sm, codes, x.tq0, x.tq1, p.Sq, list, lane);
+  if (p.n_splits == 1 && n_cache + n_list == 0) {
+    // Only padding can leave a unit without a key tile (a valid query sees
+    // its own token).  Keep one fully masked tile so that every unit of a
+    // one-split launch visits a tile and writes its (zero) rows.
+    if (list != nullptr && lane == 0) list[0] = (uint16_t)(kTilePartial | kTileAnyPad);
+    __syncwarp();
+    n_list = 1;
+  }
   const int n_total = n_cache + n_list;
   const int per = (n_total + p.n_splits - 1) / p.n_splits;
   x.it_begin = min(x.split * per, n_total);
@@ -288,6 +307,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
   const int n_key_tok = p.Sq;
   const int n_cache = kSuffix ? (p.P + kBN - 1) / kBN : 0;
+  const bool cache_masked = kSuffix && p.cache_valid != nullptr;
 
   // The mask bytes are the first global reads: issue them before anything
   // else so their latency hides behind the barrier and TMEM set-up.  With a
@@ -295,7 +315,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // this cluster runs exactly one unit and scans that unit's batch row.
   const int b_codes = (cluster / p.n_splits) / n_pairs;
   const uint8_t* ar_b = p.ar + (long long)b_codes * p.mask_bs;
-  const int32_t* seg_b = (!kSuffix && p.seg) ? p.seg + (long long)b_codes * p.mask_bs : nullptr;
+  const int32_t* seg_b = p.seg ? p.seg + (long long)b_codes * p.mask_bs : nullptr;
   const Flags32 flags0 = load_flags32(ar_b, seg_b, n_key_tok, (int)threadIdx.x * 32);
 
   // ---------------------------------------------------------------- set-up
@@ -332,9 +352,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   // Both CTAs' barriers must exist before either side signals the other.
   cluster_sync();
-  // With a single split every unit visits at least one key tile (a query
-  // always sees its own token), so the first unit's Q can load during the
-  // mask scan.
+  // With a single split every unit visits at least one key tile (a valid
+  // query sees its own token; a unit of padding rows gets one masked tile),
+  // so the first unit's Q can load during the mask scan.
   const bool early_q = p.n_splits == 1;
   if (early_q && threadIdx.x == 0) {
     const int pair0 = cluster % n_pairs, b0 = cluster / n_pairs;
@@ -380,7 +400,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       ++nq;
       auto load_k = [&](int idx) -> bool {
-        const KvTile kt = kv_tile_at<kSuffix>(list, idx, n_cache, p.P);
+        const KvTile kt = kv_tile_at<kSuffix>(list, idx, n_cache, p.P, cache_masked);
         const int s = (int)(uk % kK);
         const uint32_t rel = uk / kK;
         if (rel > 0 && !warp_wait(&sm.k_empty[s], (rel - 1) & 1, sm, ctl)) return false;
@@ -396,7 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         return true;
       };
       auto load_v = [&](int idx, int h) -> bool {
-        const KvTile kt = kv_tile_at<kSuffix>(list, idx, n_cache, p.P);
+        const KvTile kt = kv_tile_at<kSuffix>(list, idx, n_cache, p.P, cache_masked);
         const int s = (int)(uv % kV);
         const uint32_t rel = uv / kV;
         if (rel > 0 && !warp_wait(&sm.v_empty[s], (rel - 1) & 1, sm, ctl)) return false;
@@ -503,6 +523,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ++nu;
           for (int j = 0; j < x.n_it && ok; ++j) {
             const uint32_t gi = g + (uint32_t)j;
+            // V arrives long before P: wait for it first, off the critical path.
+            if (!warp_wait(&sm.v_full[uv % kV], (uv / kV) & 1, sm, ctl)) { ok = false; break; }
             if (!warp_wait(&sm.p_full, gi & 1, sm, ctl)) { ok = false; break; }
             // The unit's first PV overwrites O: the previous unit's epilogue
             // must have read it.
@@ -512,7 +534,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             for (int h = 0; h < 2 && ok; ++h) {
               const int s = (int)(uv % kV);
-              if (!warp_wait(&sm.v_full[s], (uv / kV) & 1, sm, ctl)) { ok = false; break; }
+              if (h == 1 && !warp_wait(&sm.v_full[s], (uv / kV) & 1, sm, ctl)) {
+                ok = false;
+                break;
+              }
               tc_fence_after();
               if (lane == 0) {
                 const uint64_t vd = vdesc0 + (uint64_t)((s * kVItem) >> 4);
@@ -576,15 +601,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t cq = codes[tok];
       const uint32_t csq = cq >> 2;
       const bool row_expert = (cq & 2u) != 0;
+      const bool row_pad = is_pad(cq);               // a padding query sees nothing
       float m_run = -INFINITY;
       float l_run = 0.f;
 
       for (int li = 0; li < x.n_it; ++li) {
         const uint32_t gi = g + (uint32_t)li;
         const int bs = (int)(gi & 1);
+        const KvTile kt = kv_tile_at<kSuffix>(list, x.it_begin + li, n_cache, p.P, cache_masked);
+        // Validity bytes of a cached tile, loaded before the wait for S: byte
+        // lane + 32w of the tile in v[w].
+        uint32_t vraw[4] = {0u, 0u, 0u, 0u};
+        if (kSuffix && kt.src == 1 && cache_masked) {
+          const uint8_t* cv = p.cache_valid + (long long)x.b * p.P + kt.tile * kBN;
+          const int n_here = min(kBN, p.P - kt.tile * kBN);
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            vraw[w] = (lane + 32 * w < n_here) ? (uint32_t)cv[lane + 32 * w] : 0u;
+        }
         if (!warp_wait(&sm.s_full[bs], (gi >> 1) & 1, sm, ctl)) { ok = false; break; }
         tc_fence_after();
-        const KvTile kt = kv_tile_at<kSuffix>(list, x.it_begin + li, n_cache, p.P);
         float xs[kBN];
         {
           // all four 32-column loads in flight, one wait
@@ -616,6 +652,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           bool hole = false;
           if (kSuffix && kt.src == 1) {
             e = min(kBN, p.P - k0);
+            if (cache_masked) {
+              // Padded prefix keys: bit j of vb[j / 32] set iff key j is valid.
+              uint32_t vb[4];
+#pragma unroll
+              for (int w = 0; w < 4; ++w) vb[w] = __ballot_sync(0xffffffffu, vraw[w] != 0u);
+#pragma unroll
+              for (int j = 0; j < kBN; ++j)
+                xs[j] = (j < e && ((vb[j >> 5] >> (j & 31)) & 1u)) ? xs[j] : -INFINITY;
+              e = kBN;                              // applied above
+            }
           } else {
             e = 0;
 #pragma unroll
@@ -624,9 +670,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               if (probe <= kBN && (uint32_t)(codes[k0 + probe - 1] >> 2) <= csq) e = probe;
             }
             e = min(e, n_key_tok - k0);
-            hole = row_expert && kt.any_fast;
+            hole = (row_expert && kt.any_fast) || kt.any_pad;
           }
           if (hole) {
+            // Per key: FAST keys are hidden from expert rows, padding keys
+            // from every row (padding also carries the FAST bit).
             const uint4* kc = reinterpret_cast<const uint4*>(codes + k0);
 #pragma unroll
             for (int q8 = 0; q8 < kBN / 8; ++q8) {
@@ -635,14 +683,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int h = 0; h < 8; ++h) {
                 const int j = 8 * q8 + h;
-                const bool fast = ((wv[h >> 1] >> (16 * (h & 1))) & 1u) != 0;
-                xs[j] = (j < e && !fast) ? xs[j] : -INFINITY;
+                const uint32_t ck = (wv[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+                const bool hide = (row_expert && (ck & 1u)) || is_pad(ck);
+                xs[j] = (j < e && !hide) ? xs[j] : -INFINITY;
               }
             }
           } else {
 #pragma unroll
             for (int j = 0; j < kBN; ++j) xs[j] = j < e ? xs[j] : -INFINITY;
           }
+        }
+        if (row_pad) {
+#pragma unroll
+          for (int j = 0; j < kBN; ++j) xs[j] = -INFINITY;
         }
         // Row maximum: eight independent chains of three-input max.
         float m8[8];
@@ -729,7 +782,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const long long grow = (long long)x.b * rows_per_b + row0 + r;
       if (p.n_splits == 1) {
-        const float inv = 1.f / l_run;
+        // A row that saw no key (a padding query) writes 0, lse = -inf.
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
         // The P buffer is free once the last PV has finished: each warp stages
         // its own 32 rows there, 64 columns per 4 KB swizzled box, in two
         // rounds of two boxes.
@@ -781,7 +835,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         store_pending = true;
         if (!kSuffix && p.lse && row_valid)
-          p.lse[grow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+          p.lse[grow] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
       } else {
         // Split-K partial: unnormalised O and (m, l) for the combine kernel.
         // tcgen05.ld is warp-collective (.sync.aligned): every lane loads,
@@ -853,7 +907,7 @@ __global__ void __launch_bounds__(256)
     acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
     acc[4] += w * c.x; acc[5] += w * c.y; acc[6] += w * c.z; acc[7] += w * c.w;
   }
-  const float inv = 1.f / L;
+  const float inv = L > 0.f ? 1.f / L : 0.f;   // every split empty: a padding row
   uint4 pk;
   pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
