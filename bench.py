@@ -47,7 +47,7 @@ L2_BYTES = 126 * 2**20
 # DRAM traffic of the prefill kernel per launch on the pi0 workload, from one
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the
 # kernel sources whose digest is recorded beside it.
-TRAFFIC = {"bytes": 25173888, "src_sha": "7f2601ec518fb63d"}
+TRAFFIC = {"bytes": 25184896, "src_sha": "f6025ed41baa6bac"}
 KERNEL_SOURCES = ("vla_prefix_lm_b200/csrc/tc_pair.cu", "vla_prefix_lm_b200/csrc/common.cuh",
                   "vla_prefix_lm_b200/csrc/mask.cuh")
 
@@ -278,6 +278,7 @@ def run_ours(args, rank, ws, local):
 
     # suffix pass: 10 Euler steps against the prefix cache (warm L2, back to back)
     suffix = suffix_control(args, dev, stream, rank)
+    decode = decode_steps(args, dev, stream, rank)
 
     traffic = TRAFFIC["bytes"] if TRAFFIC["src_sha"] == kernel_digest() else None
     line = {
@@ -326,10 +327,65 @@ def run_ours(args, rank, ws, local):
         "gpu_launches": args.steps,
         "clocks": clocks,
         "suffix_ctrl": suffix,
+        "decode": decode,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, seconds=args.cpu_seconds)
     return line
+
+
+def decode_steps(args, dev, stream, rank):
+    """FAST-style single-token decode: B=32 queries of one token (8 heads)
+    against a cache of 880 tokens (816 prefix + 64 generated), cold L2.  Each
+    step reads the whole cache once: HBM-bound."""
+    import torch
+
+    from vla_prefix_lm_b200 import binding, dist
+    from vla_prefix_lm_b200 import workloads as W
+
+    B, P, Hq, d = 32, 880, 8, 256
+    P_ = peaks()
+    kc, _ = W.draw((B, P, 1, d), 9001 + rank, d, "bf16")
+    vc, _ = W.draw((B, P, 1, d), 9002 + rank, d, "bf16")
+    q, _ = W.draw((B, 1, Hq, d), 9003 + rank, d, "bf16")
+    k, _ = W.draw((B, 1, 1, d), 9004 + rank, d, "bf16")
+    v, _ = W.draw((B, 1, 1, d), 9005 + rank, d, "bf16")
+    kc, vc, q, k, v = (t.to(dev) for t in (kc, vc, q, k, v))
+    ar = torch.ones(1, dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    need = binding.pi_attn_suffix_workspace_bytes(q, k, kc, ar)
+    wsb = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            binding.pi_attn_suffix(q, k, v, kc, vc, ar, out=out, workspace=wsb, stream=stream)
+    torch.cuda.synchronize()
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1, stream=stream):
+        binding.pi_attn_suffix(q, k, v, kc, vc, ar, out=out, workspace=wsb, stream=stream)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cold = []
+    dist.barrier()
+    for _ in range(20):
+        with torch.cuda.stream(stream):
+            flush.fill_(1.0)
+            e0.record(stream)
+            g1.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        cold.append(e0.elapsed_time(e1) * 1e3)
+    us = dist.max_over_ranks(float(np.median(cold)))
+    del flush
+    assert binding.pi_attn_read_status(stream) == binding.PI_OK
+    bytes_step = 2 * B * P * d * 2 + 2 * B * Hq * d * 2 + 2 * B * d * 2
+    return {
+        "workload": "single-token decode: B=32, Hq=8, d=256, cache 880 (pi_attn_suffix, Sq=1)",
+        "us_per_step_cold_l2": us,
+        "gb_per_s_algorithmic": bytes_step / (us / 1e6) / 1e9,
+        "hbm_frac": bytes_step / (us / 1e6) / 1e9 / P_["hbm_gbs"],
+        "algorithmic_bytes_per_step": bytes_step,
+        "splits": binding.pi_attn_suffix_workspace_bytes(q, k, kc, ar) > 0,
+    }
 
 
 def suffix_control(args, dev, stream, rank):

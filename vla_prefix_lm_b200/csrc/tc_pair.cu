@@ -278,7 +278,7 @@ __device__ __forceinline__ Unit make_unit(int u, const TcParams& p, int n_pairs,
   return x;
 }
 
-template <bool kSuffix, class L>
+template <bool kSuffix, bool kCacheMask, class L>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_pair_kernel(const __grid_constant__ TcParams p, const DevCtl ctl, int smem_bytes) {
   using SmemT = Smem<L>;
@@ -307,7 +307,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
   const int n_key_tok = p.Sq;
   const int n_cache = kSuffix ? (p.P + kBN - 1) / kBN : 0;
-  const bool cache_masked = kSuffix && p.cache_valid != nullptr;
+  // A separate instantiation carries the cached-key validity mask, so the
+  // unmasked suffix pass pays nothing for it.
+  constexpr bool cache_masked = kSuffix && kCacheMask;
 
   // The mask bytes are the first global reads: issue them before anything
   // else so their latency hides behind the barrier and TMEM set-up.  With a
@@ -924,14 +926,23 @@ int pair_smem_bytes(int n_code_tokens) {
   return min(layout_bytes<L>(n_code_tokens) + 1024, kSmemLimit);
 }
 
-template <bool kSuffix, class L>
+template <bool kSuffix, bool kCacheMask, class L>
 cudaError_t launch_pair(const TcParams& p, const DevCtl& ctl, dim3 grid, cudaStream_t st) {
   static const cudaError_t attr_err = cudaFuncSetAttribute(
-      tc_pair_kernel<kSuffix, L>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+      tc_pair_kernel<kSuffix, kCacheMask, L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      kSmemLimit);
   if (attr_err != cudaSuccess) return attr_err;
   const int smem = pair_smem_bytes<L>(p.Sq);
-  tc_pair_kernel<kSuffix, L><<<grid, kThreads, smem, st>>>(p, ctl, smem);
+  tc_pair_kernel<kSuffix, kCacheMask, L><<<grid, kThreads, smem, st>>>(p, ctl, smem);
   return cudaGetLastError();
+}
+
+template <class L>
+cudaError_t launch_mode(const TcParams& p, bool suffix_mode, const DevCtl& ctl, dim3 grid,
+                        cudaStream_t st) {
+  if (!suffix_mode) return launch_pair<false, false, L>(p, ctl, grid, st);
+  return p.cache_valid ? launch_pair<true, true, L>(p, ctl, grid, st)
+                       : launch_pair<true, false, L>(p, ctl, grid, st);
 }
 
 int sm_count() {
@@ -956,10 +967,8 @@ cudaError_t launch_tc_pair(const TcParams& p, bool suffix_mode, const DevCtl& ct
   const int n_clusters = p.mask_bs == 0 ? min(n_units, max(sm_count() / 2, 1)) : n_units;
   dim3 grid(2 * n_clusters, 1);
   const bool short_s = p.Sq <= LayoutShort::kMaxTok;
-  cudaError_t e = suffix_mode ? (short_s ? launch_pair<true, LayoutShort>(p, ctl, grid, st)
-                                         : launch_pair<true, LayoutLong>(p, ctl, grid, st))
-                              : (short_s ? launch_pair<false, LayoutShort>(p, ctl, grid, st)
-                                         : launch_pair<false, LayoutLong>(p, ctl, grid, st));
+  cudaError_t e = short_s ? launch_mode<LayoutShort>(p, suffix_mode, ctl, grid, st)
+                          : launch_mode<LayoutLong>(p, suffix_mode, ctl, grid, st);
   if (e != cudaSuccess || p.n_splits <= 1) return e;
   const long long n_rows = (long long)p.B * rows;
   combine_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, st>>>(
