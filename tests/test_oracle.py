@@ -524,3 +524,56 @@ def test_planted_padding_mistakes_are_caught():
     assert np.array_equal(good, brute_m)
     assert not np.array_equal(keys_only, brute_m)
     assert not np.array_equal(rows_only, brute_m)
+
+
+# ---------------------------------------------------- pre/post steps (f3)
+from oracle import prepost  # noqa: E402
+
+
+def test_positions_follow_the_pages():
+    """Prefix positions are cumsum(mask) - 1; suffix positions continue after
+    the valid prefix tokens ('VLA 代码精读 - OpenPI & StarVLA', 1.6)."""
+    pm = np.array([[1, 1, 1, 0, 0], [1, 0, 1, 1, 1]])
+    assert prepost.positions(pm).tolist() == [[0, 1, 2, 2, 2], [0, 0, 1, 2, 3]]
+    sm = np.ones((2, 3), np.uint8)
+    assert prepost.positions(sm, pm).tolist() == [[3, 4, 5], [4, 5, 6]]
+
+
+def test_rope_closed_forms():
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((2, 5, 3, 16))
+    # position 0 is the identity
+    assert np.allclose(prepost.rope(x, np.zeros((2, 5))), x, atol=0)
+    # each (i, i + d/2) pair is rotated: the pair's norm is kept
+    y = prepost.rope(x, rng.integers(0, 1000, (2, 5)))
+    n_x = x[..., :8] ** 2 + x[..., 8:] ** 2
+    n_y = y[..., :8] ** 2 + y[..., 8:] ** 2
+    np.testing.assert_allclose(n_y, n_x, rtol=1e-12)
+    # pair 0 turns by exactly pos radians (frequency base^0 = 1), counter-clockwise
+    e = np.zeros((1, 1, 1, 16)); e[..., 0] = 1.0
+    z = prepost.rope(e, np.array([[np.pi / 2]]))
+    np.testing.assert_allclose(z[0, 0, 0, [0, 8]], [0.0, 1.0], atol=1e-15)
+
+
+def test_rope_scores_depend_only_on_relative_position():
+    """<rope(q, m), rope(k, n)> is a function of m - n (the property RoPE is
+    built for); a wrong sign or pairing breaks it."""
+    rng = np.random.default_rng(22)
+    q = rng.standard_normal((1, 1, 1, 32))
+    k = rng.standard_normal((1, 1, 1, 32))
+    def score(m, n):
+        return float(np.sum(prepost.rope(q, np.array([[m]])) * prepost.rope(k, np.array([[n]]))))
+    for m, n in [(5, 2), (105, 102), (7, 7), (1000, 997)]:
+        np.testing.assert_allclose(score(m, n), score(m - n, 0), atol=1e-9)
+    assert abs(score(5, 2) - score(2, 5)) > 1e-3   # but not symmetric
+
+
+def test_euler_step_reaches_the_ode_solution():
+    """dx/dt = v constant: ten steps of dt = -1/10 from t = 1 land on x - v."""
+    rng = np.random.default_rng(23)
+    x = rng.standard_normal((4, 50, 32))
+    v = rng.standard_normal((4, 50, 32))
+    y = x.copy()
+    for _ in range(10):
+        y = prepost.euler_step(y, v, -0.1)
+    np.testing.assert_allclose(y, x - v, atol=1e-12)
