@@ -241,6 +241,46 @@ int pi_attn_suffix_noalloc(const pi_attn_desc* desc, const void* q_suf, const vo
 /* Size in bytes of the fixed buffer pi_attn_suffix_noalloc uses. */
 size_t pi_attn_suffix_noalloc_capacity(void);
 
+/*
+ * Steps on either side of the attention (the Euler sampling loop of
+ * "VLA 代码精读 - OpenPI & StarVLA", 1.6 Pi0.sample_actions).
+ *
+ * pi_rope_inplace -- rotary position embedding of q (and k) in place.
+ * Positions are cumsum(token_mask) - 1 over the call's S tokens (1.5: the
+ * joint forward), and with a prefix mask they continue after its valid
+ * tokens: sum(prefix_mask) + cumsum(token_mask) - 1 (1.6: the suffix pass).
+ * The pages name the LLM's built-in RoPE without a formula; this is the
+ * standard rotation of each head vector's (i, i + d/2) pairs by the angle
+ * pos * base^(-2i/d):  [x1 cos - x2 sin, x2 cos + x1 sin].
+ *   q [B, S, Hq, d], k [B, S, Hkv, d] or NULL  (bf16 or fp32, rotated in place)
+ *   token_mask [B or 1, S] uint8 (nonzero = valid token), at mask_batch_stride
+ *   prefix_mask [B or 1, P] uint8 at prefix_batch_stride; required iff P > 0
+ *   positions_out [B, S] int32 or NULL (written: the positions used)
+ * d must be a multiple of 16 and at most 256; base > 1 (10000 for Gemma).
+ * Errors as the attention calls (host-side checks, PI_ERR_ALIGN for pointers
+ * not 16-byte aligned).
+ */
+typedef struct pi_rope_desc {
+  int32_t B, S, P;         /* batch, tokens to rotate, prefix tokens (0 = none) */
+  int32_t Hq, Hkv, d;      /* heads of q and k, head dimension                   */
+  int32_t dtype;           /* PI_BF16 or PI_F32 (q and k alike)                  */
+  float base;              /* rotary base, > 1                                   */
+  int64_t mask_batch_stride;    /* token_mask: 0 = shared by the batch, else >= S */
+  int64_t prefix_batch_stride;  /* prefix_mask: 0 = shared, else >= P             */
+} pi_rope_desc;
+
+int pi_rope_inplace(const pi_rope_desc* desc, void* q, void* k, const uint8_t* token_mask,
+                    const uint8_t* prefix_mask, int32_t* positions_out, pi_stream_t stream);
+
+/*
+ * pi_euler_update -- one Euler step of the flow-matching sampler in place,
+ * x <- x + dt * v (1.6: dt = -1 / num_steps, from t = 1 to t = 0).
+ *   x [n] fp32 (the action chunk, read and written), v [n] bf16 or fp32
+ *   (v_dtype PI_BF16 / PI_F32).  Both 16-byte aligned.
+ */
+int pi_euler_update(float* x, const void* v, int32_t v_dtype, float dt, int64_t n,
+                    pi_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

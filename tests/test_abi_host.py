@@ -22,7 +22,7 @@ def _lib():
 
 def _declared():
     src = open(os.path.join(ROOT, "include", "pi_attn.h")).read()
-    return sorted(set(re.findall(r"\b(pi_attn_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(pi_(?:attn|rope|euler)\w*)\s*\(", src)))
 
 
 def test_header_declares_the_two_calls():
@@ -137,3 +137,29 @@ def test_product_path_has_no_oracle_import():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
+
+
+def _rope_desc(binding, **kw):
+    d = dict(B=2, S=16, P=0, Hq=8, Hkv=1, d=256, dtype=binding.PI_BF16, base=10000.0,
+             mask_batch_stride=0, prefix_batch_stride=0)
+    d.update(kw)
+    return binding.PiRopeDesc(**d)
+
+
+def test_rope_and_euler_argument_errors():
+    b, L = _lib()
+    rope = lambda desc, q=FAKE, k=FAKE, tm=FAKE, pm=None: L.pi_rope_inplace(
+        ctypes.byref(desc) if desc is not None else None, q, k, tm, pm, None, None)
+    assert rope(None) == b.PI_ERR_ARG
+    assert rope(_rope_desc(b, d=250)) == b.PI_ERR_UNSUPPORTED
+    assert rope(_rope_desc(b, d=512)) == b.PI_ERR_UNSUPPORTED
+    assert rope(_rope_desc(b, base=1.0)) == b.PI_ERR_ARG
+    assert rope(_rope_desc(b, P=4)) == b.PI_ERR_ARG            # a prefix needs its mask
+    assert rope(_rope_desc(b), q=FAKE_MIS) == b.PI_ERR_ALIGN
+    assert rope(_rope_desc(b), tm=None) == b.PI_ERR_ARG
+    assert rope(_rope_desc(b, B=0), q=None, tm=None) == b.PI_OK
+    eu = L.pi_euler_update
+    assert eu(FAKE, FAKE, 7, ctypes.c_float(0.1), 16, None) == b.PI_ERR_UNSUPPORTED
+    assert eu(FAKE, FAKE, b.PI_F32, ctypes.c_float(float("nan")), 16, None) == b.PI_ERR_ARG
+    assert eu(FAKE_MIS, FAKE, b.PI_F32, ctypes.c_float(0.1), 16, None) == b.PI_ERR_ALIGN
+    assert eu(None, None, b.PI_F32, ctypes.c_float(0.1), 0, None) == b.PI_OK

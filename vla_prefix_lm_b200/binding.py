@@ -34,6 +34,8 @@ EXPORTED = (
     "pi_attn_selftest_wait",
     "pi_attn_suffix_masked",
     "pi_attn_suffix_noalloc",
+    "pi_rope_inplace",
+    "pi_euler_update",
     "pi_attn_suffix_noalloc_capacity",
 )
 
@@ -42,6 +44,21 @@ class PiAttnError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
         super().__init__(f"{what}: {status_string(code)} ({code})")
+
+
+class PiRopeDesc(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32),
+        ("S", ctypes.c_int32),
+        ("P", ctypes.c_int32),
+        ("Hq", ctypes.c_int32),
+        ("Hkv", ctypes.c_int32),
+        ("d", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+        ("base", ctypes.c_float),
+        ("mask_batch_stride", ctypes.c_int64),
+        ("prefix_batch_stride", ctypes.c_int64),
+    ]
 
 
 class PiAttnDesc(ctypes.Structure):
@@ -89,6 +106,10 @@ def lib() -> ctypes.CDLL:
         L.pi_attn_selftest_wait.restype = i32
         L.pi_attn_suffix_masked.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.pi_attn_suffix_masked.restype = i32
+        L.pi_rope_inplace.argtypes = [ctypes.POINTER(PiRopeDesc), vp, vp, vp, vp, vp, vp]
+        L.pi_rope_inplace.restype = i32
+        L.pi_euler_update.argtypes = [vp, vp, i32, ctypes.c_float, ctypes.c_int64, vp]
+        L.pi_euler_update.restype = i32
         L.pi_attn_suffix_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.pi_attn_suffix_noalloc.restype = i32
         L.pi_attn_suffix_noalloc_capacity.argtypes = []
@@ -261,6 +282,46 @@ def pi_attn_suffix_noalloc(q_suf, k_suf, v_suf, k_cache, v_cache, ar_mask_suf, o
                  if rc == PI_ERR_UNSUPPORTED and need > cap else "")
         raise PiAttnError(rc, "pi_attn_suffix_noalloc" + extra)
     return out
+
+
+def pi_rope_inplace(q, k, token_mask, prefix_mask=None, base=10000.0, positions=False,
+                    stream=None):
+    """Rotary embedding of q [B,S,Hq,d] (and k [B,S,Hkv,d] or None) in place at
+    positions cumsum(token_mask) - 1 (+ the valid prefix count when
+    ``prefix_mask`` [B,P] is given).  Returns the int32 [B,S] positions when
+    ``positions`` is true."""
+    _need(q, "q", dims=4)
+    if k is not None:
+        _need(k, "k", q.dtype, 4)
+    _need(token_mask, "token_mask", torch.uint8)
+    B, S, Hq, d = q.shape
+    tbs = _mask_stride(token_mask, B, S)
+    P, pbs = 0, 0
+    if prefix_mask is not None:
+        _need(prefix_mask, "prefix_mask", torch.uint8)
+        P = prefix_mask.shape[-1]
+        pbs = _mask_stride(prefix_mask, B, P)
+    pos = torch.empty((B, S), dtype=torch.int32, device=q.device) if positions else None
+    desc = PiRopeDesc(B, S, P, Hq, 1 if k is None else k.shape[2], d, _dtype_code(q),
+                      float(base), tbs, pbs)
+    rc = lib().pi_rope_inplace(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(token_mask),
+                               _ptr(prefix_mask), _ptr(pos), ctypes.c_void_p(_stream(stream)))
+    if rc != PI_OK:
+        raise PiAttnError(rc, "pi_rope_inplace")
+    return pos
+
+
+def pi_euler_update(x, v, dt, stream=None):
+    """x (fp32) += dt * v (bf16 or fp32, same number of elements), in place."""
+    _need(x, "x", torch.float32)
+    _need(v, "v")
+    if v.numel() != x.numel():
+        raise ValueError("x and v must have the same number of elements")
+    rc = lib().pi_euler_update(_ptr(x), _ptr(v), _dtype_code(v), float(dt), x.numel(),
+                               ctypes.c_void_p(_stream(stream)))
+    if rc != PI_OK:
+        raise PiAttnError(rc, "pi_euler_update")
+    return x
 
 
 def pi_attn_debug_mask(ar_mask, segment_ids=None, B=None, P=0, mode=0, stream=None):

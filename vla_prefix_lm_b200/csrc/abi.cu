@@ -246,6 +246,48 @@ int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
                                nullptr, out, workspace, ws_bytes, stream);
 }
 
+int pi_rope_inplace(const pi_rope_desc* d, void* q, void* k, const uint8_t* token_mask,
+                    const uint8_t* prefix_mask, int32_t* positions_out, pi_stream_t stream) {
+  if (!d) return PI_ERR_ARG;
+  if (d->B < 0 || d->S < 0 || d->P < 0 || d->Hq <= 0 || d->Hkv <= 0 || d->d <= 0)
+    return PI_ERR_ARG;
+  if (!(d->base > 1.f) || !std::isfinite(d->base)) return PI_ERR_ARG;
+  if (d->dtype != PI_BF16 && d->dtype != PI_F32) return PI_ERR_UNSUPPORTED;
+  if (d->d > 256 || d->d % 16 != 0) return PI_ERR_UNSUPPORTED;
+  if (d->mask_batch_stride < 0 || (d->mask_batch_stride != 0 && d->mask_batch_stride < d->S))
+    return PI_ERR_ARG;
+  if (d->prefix_batch_stride < 0 ||
+      (d->prefix_batch_stride != 0 && d->prefix_batch_stride < d->P))
+    return PI_ERR_ARG;
+  if (d->B == 0 || d->S == 0) return PI_OK;
+  if (!q || !token_mask) return PI_ERR_ARG;
+  if (d->P > 0 && !prefix_mask) return PI_ERR_ARG;
+  if (!aligned16(q) || (k && !aligned16(k))) return PI_ERR_ALIGN;
+  if (positions_out && (reinterpret_cast<uintptr_t>(positions_out) & 3u)) return PI_ERR_ALIGN;
+  RopeParams p;
+  p.q = q;
+  p.k = k;
+  p.tmask = token_mask;
+  p.tmask_bs = d->mask_batch_stride;
+  p.pmask = d->P > 0 ? prefix_mask : nullptr;
+  p.pmask_bs = d->prefix_batch_stride;
+  p.pos_out = positions_out;
+  p.B = d->B; p.S = d->S; p.P = d->P; p.Hq = d->Hq; p.Hkv = d->Hkv; p.d = d->d;
+  p.base = d->base;
+  p.f32 = d->dtype == PI_F32;
+  return launched(launch_rope(p, static_cast<cudaStream_t>(stream)));
+}
+
+int pi_euler_update(float* x, const void* v, int32_t v_dtype, float dt, int64_t n,
+                    pi_stream_t stream) {
+  if (n < 0 || !std::isfinite(dt)) return PI_ERR_ARG;
+  if (v_dtype != PI_BF16 && v_dtype != PI_F32) return PI_ERR_UNSUPPORTED;
+  if (n == 0) return PI_OK;
+  if (!x || !v) return PI_ERR_ARG;
+  if (!aligned16(x) || !aligned16(v)) return PI_ERR_ALIGN;
+  return launched(launch_euler(x, v, v_dtype == PI_F32, dt, n, static_cast<cudaStream_t>(stream)));
+}
+
 int pi_attn_debug_mask(const pi_attn_desc* d, int mode, const uint8_t* ar_mask,
                        const int32_t* segment_ids, uint8_t* mask_out, pi_stream_t stream) {
   if (!d || !ar_mask || !mask_out) return PI_ERR_ARG;

@@ -35,6 +35,27 @@ cudaError_t launch_debug_mask(int mode, int B, int Sq, int P, const uint8_t* ar,
 
 cudaError_t launch_selftest_wait(const DevCtl& ctl, cudaStream_t st);
 
+// Rotary embedding of q (and k) in place at positions cumsum(tmask) - 1
+// (+ the valid prefix count when pmask is given).
+struct RopeParams {
+  void* q;
+  void* k;                 // may be null
+  const uint8_t* tmask;
+  long long tmask_bs;
+  const uint8_t* pmask;    // may be null
+  long long pmask_bs;
+  int32_t* pos_out;        // may be null
+  int B, S, P, Hq, Hkv, d;
+  float base;
+  bool f32;
+};
+
+cudaError_t launch_rope(const RopeParams& p, cudaStream_t st);
+
+// x (fp32) += dt * v (bf16 or fp32), n elements.
+cudaError_t launch_euler(float* x, const void* v, bool v_f32, float dt, long long n,
+                         cudaStream_t st);
+
 // bf16 tcgen05 path.  All tensors are [B, tokens, heads, 256] bf16; maps are
 // encoded by the ABI layer.
 struct TcParams {
