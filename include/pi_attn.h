@@ -256,7 +256,8 @@ size_t pi_attn_suffix_noalloc_capacity(void);
  *   token_mask [B or 1, S] uint8 (nonzero = valid token), at mask_batch_stride
  *   prefix_mask [B or 1, P] uint8 at prefix_batch_stride; required iff P > 0
  *   positions_out [B, S] int32 or NULL (written: the positions used)
- * d must be a multiple of 16 and at most 256; base > 1 (10000 for Gemma).
+ * d must be a multiple of 16 and at most 256, B at most 65535 (else
+ * PI_ERR_UNSUPPORTED); base > 1 (10000 for Gemma).
  * Errors as the attention calls (host-side checks, PI_ERR_ALIGN for pointers
  * not 16-byte aligned).
  */

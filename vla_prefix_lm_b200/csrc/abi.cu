@@ -253,7 +253,7 @@ int pi_rope_inplace(const pi_rope_desc* d, void* q, void* k, const uint8_t* toke
     return PI_ERR_ARG;
   if (!(d->base > 1.f) || !std::isfinite(d->base)) return PI_ERR_ARG;
   if (d->dtype != PI_BF16 && d->dtype != PI_F32) return PI_ERR_UNSUPPORTED;
-  if (d->d > 256 || d->d % 16 != 0) return PI_ERR_UNSUPPORTED;
+  if (d->d > 256 || d->d % 16 != 0 || d->B > 65535) return PI_ERR_UNSUPPORTED;
   if (d->mask_batch_stride < 0 || (d->mask_batch_stride != 0 && d->mask_batch_stride < d->S))
     return PI_ERR_ARG;
   if (d->prefix_batch_stride < 0 ||
