@@ -279,6 +279,7 @@ def run_ours(args, rank, ws, local):
     # suffix pass: 10 Euler steps against the prefix cache (warm L2, back to back)
     suffix = suffix_control(args, dev, stream, rank)
     decode = decode_steps(args, dev, stream, rank)
+    prepost = prepost_steps(args, dev, stream, rank)
 
     traffic = TRAFFIC["bytes"] if TRAFFIC["src_sha"] == kernel_digest() else None
     line = {
@@ -328,10 +329,123 @@ def run_ours(args, rank, ws, local):
         "clocks": clocks,
         "suffix_ctrl": suffix,
         "decode": decode,
+        "prepost": prepost,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, seconds=args.cpu_seconds)
     return line
+
+
+def _cold_graph_us(fn, stream, reps=20):
+    """Median device time of one graph replay of ``fn`` with L2 flushed before each."""
+    import torch
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=stream.device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t = []
+    for _ in range(reps):
+        with torch.cuda.stream(stream):
+            flush.fill_(1.0)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        t.append(e0.elapsed_time(e1) * 1e3)
+    del g, flush
+    return float(np.median(t))
+
+
+def prepost_steps(args, dev, stream, rank):
+    """RoPE and the Euler update around the attention, each timed alone (cold
+    L2), and the whole pi0 sampling loop -- per step RoPE of the suffix q/k at
+    the continued positions, the suffix pass, the Euler update -- as one graph."""
+    import torch
+
+    from vla_prefix_lm_b200 import binding, dist
+    from vla_prefix_lm_b200 import workloads as W
+
+    P_ = peaks()
+    hbm = P_["hbm_gbs"]
+    res = {}
+    # prefill: q [8, 611, 8, 256], k [8, 611, 1, 256] bf16, all tokens valid
+    B, S, Hq, d = 8, 611, 8, 256
+    q, _ = W.draw((B, S, Hq, d), 9101 + rank, d, "bf16")
+    k, _ = W.draw((B, S, 1, d), 9102 + rank, d, "bf16")
+    q, k = q.to(dev), k.to(dev)
+    tm = torch.ones((B, S), dtype=torch.uint8, device=dev)
+    us = dist.max_over_ranks(_cold_graph_us(
+        lambda: binding.pi_rope_inplace(q, k, tm, stream=stream), stream))
+    nb = 2 * (q.numel() + k.numel()) * 2 + tm.numel()
+    res["rope_prefill"] = {"shape": "q [8,611,8,256], k [8,611,1,256] bf16", "us_cold_l2": us,
+                           "algorithmic_bytes": nb, "gb_per_s": nb / us / 1e3,
+                           "hbm_frac": nb / us / 1e3 / hbm}
+    del q, k, tm
+
+    # suffix loop of the pi0 workload: B=32, 51 suffix tokens, cache 816, 10 steps
+    w = W.workload(3)
+    c = W.cache_inputs(w, W.seed_for(3, 999) + rank * 7, B=w.B)
+    kc, vc = c.k.to(dev), c.v.to(dev)
+    steps = [W.suffix_inputs(w, W.seed_for(3, s) + rank * 7, B=w.B) for s in range(w.calls)]
+    ins = [(x.q.to(dev), x.k.to(dev), x.v.to(dev), x.ar.to(dev)) for x in steps]
+    outs = [torch.empty_like(x[0]) for x in ins]
+    pm = torch.ones((w.B, w.P), dtype=torch.uint8, device=dev)
+    sm_ = torch.ones((w.B, w.Sq), dtype=torch.uint8, device=dev)
+    A, D = w.Sq - 1, 32
+    x = torch.zeros((w.B, A, D), dtype=torch.float32, device=dev)
+    vel = [torch.randn((w.B, A, D), dtype=torch.float32, device=dev) for _ in range(w.calls)]
+    need = binding.pi_attn_suffix_workspace_bytes(ins[0][0], ins[0][1], kc, ins[0][3])
+    wsb = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+
+    q0, k0 = ins[0][0], ins[0][1]
+    us = dist.max_over_ranks(_cold_graph_us(
+        lambda: binding.pi_rope_inplace(q0, k0, sm_, prefix_mask=pm, stream=stream), stream))
+    nb = 2 * (q0.numel() + k0.numel()) * 2 + sm_.numel() + pm.numel()
+    res["rope_suffix"] = {"shape": "q [32,51,8,256], k [32,51,1,256] bf16, prefix mask [32,816]",
+                          "us_cold_l2": us, "algorithmic_bytes": nb, "gb_per_s": nb / us / 1e3,
+                          "hbm_frac": nb / us / 1e3 / hbm}
+    us = dist.max_over_ranks(_cold_graph_us(
+        lambda: binding.pi_euler_update(x, vel[0], -0.1, stream=stream), stream))
+    nb = 3 * x.numel() * 4
+    res["euler"] = {"shape": "x, v [32,50,32] fp32", "us_cold_l2": us, "algorithmic_bytes": nb,
+                    "gb_per_s": nb / us / 1e3}
+
+    def ctrl():
+        for s, (q, k, v, ar) in enumerate(ins):
+            binding.pi_rope_inplace(q, k, sm_, prefix_mask=pm, stream=stream)
+            binding.pi_attn_suffix(q, k, v, kc, vc, ar, out=outs[s], workspace=wsb, stream=stream)
+            binding.pi_euler_update(x, vel[s], -1.0 / w.calls, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            ctrl()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        ctrl()
+    reps = max(5, min(200, args.steps // 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us_ctrl = dist.max_over_ranks(e0.elapsed_time(e1) * 1e3 / reps)
+    del g
+    assert binding.pi_attn_read_status(stream) == binding.PI_OK
+    res["sampling_loop"] = {
+        "workload": "pi0 10-step loop: RoPE(suffix q/k) + suffix pass + Euler per step, B=32",
+        "us_per_ctrl": us_ctrl, "gpu_launches_per_ctrl": 3 * w.calls,
+        "timing": f"one graph of 30 launches replayed {reps}x (warm L2)"}
+    return res
 
 
 def decode_steps(args, dev, stream, rank):
