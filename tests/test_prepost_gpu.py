@@ -28,13 +28,16 @@ def _err(t, ref):
     return float(np.abs(t.float().cpu().numpy().astype(np.float64) - ref).max())
 
 
-@pytest.mark.parametrize("dtype,S,tol", [("bf16", 611, 2e-2), ("f32", 4250, 1e-4)])
-def test_rope_prefill_positions(dtype, S, tol):
+@pytest.mark.parametrize("dtype,S,Hq,Hkv,d,tol", [("bf16", 611, 8, 1, 256, 2e-2),
+                                                   ("f32", 4250, 8, 1, 256, 1e-4),
+                                                   ("bf16", 97, 4, 2, 64, 2e-2),
+                                                   ("f32", 131, 11, 1, 48, 1e-4)])
+def test_rope_prefill_positions(dtype, S, Hq, Hkv, d, tol):
     rng = np.random.default_rng(31)
-    B, Hq, d = 2, 8, 256
+    B = 2
     mask = (rng.random((B, S)) < 0.9).astype(np.uint8)        # some padded tokens
     q, q64 = W.draw((B, S, Hq, d), 601, d, dtype)
-    k, k64 = W.draw((B, S, 1, d), 602, d, dtype)
+    k, k64 = W.draw((B, S, Hkv, d), 602, d, dtype)
     qd, kd = q.cuda(), k.cuda()
     pos = _b().pi_rope_inplace(qd, kd, torch.from_numpy(mask).cuda(), positions=True)
     want_pos = prepost.positions(mask)

@@ -9,12 +9,15 @@
 // without a formula: here the standard rotation of (i, i + d/2) pairs by
 // pos * base^(-2i/d).
 //
-// Both kernels are HBM-bound elementwise passes.  RoPE: one CTA per (batch,
-// 32-token chunk); the chunk's positions come from a block count of the mask
-// bytes before it plus a warp scan inside it, the angles are formed and
-// reduced modulo 2*pi in fp64 (so large positions keep fp32-level accuracy),
-// their sine and cosine are tabulated in shared memory once per (token, pair)
-// and applied to every head with 16-byte vector loads and stores.
+// Both kernels are HBM-bound elementwise passes.  RoPE: a thread owns one
+// (token, N-column slice of the first half) and the matching slice of the
+// second half; it forms that slice's angles once (pos * base^(-2i/d), the
+// inverse frequencies tabulated in fp64 per CTA and the product reduced modulo
+// 2*pi in fp64, so that large positions keep fp32-level accuracy) and applies
+// them to every head of q and k with 16-byte vector loads and stores.  The
+// head loads are issued before the position prologue (a block count of the
+// mask bytes before the CTA's tokens), so the prologue hides under their
+// latency; tokens per CTA are chosen so that a CTA has 128 busy threads.
 #include <cstdint>
 
 #include "launch.h"
@@ -23,8 +26,9 @@ namespace piattn {
 
 namespace {
 
-constexpr int kRopeTokens = 32;
-constexpr int kRopeThreads = 256;
+constexpr int kRopeThreads = 128;
+constexpr int kRopeMaxTok = 32;
+constexpr int kRopeHeadBatch = 8;              // head vectors in flight per thread
 
 template <typename T> struct Vec;
 template <> struct Vec<__nv_bfloat16> { static constexpr int N = 8; };   // 16 B
@@ -51,53 +55,46 @@ __device__ __forceinline__ uint4 pack(const float (&f)[4], float*) {
                     __float_as_uint(f[3]));
 }
 
-// Rotates the heads of one tensor [B, S, H, d] for the chunk's tokens.
+// Row of head h (q heads first, then k heads) of token t.
 template <typename T>
-__device__ void rope_rows(T* x, int H, int d, int S, int b, int t0, int nt, const float* cs,
-                          const float* sn) {
-  constexpr int N = Vec<T>::N;
-  const int half = d / 2;
-  const int vpr = half / N;                     // vectors per half row
-  const int total = nt * H * vpr;
-  for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
-    const int vi = idx % vpr;
-    const int h = (idx / vpr) % H;
-    const int tl = idx / (vpr * H);
-    T* row = x + (((long long)b * S + t0 + tl) * H + h) * d;
-    uint4* p1 = reinterpret_cast<uint4*>(row + vi * N);
-    uint4* p2 = reinterpret_cast<uint4*>(row + half + vi * N);
-    float a[N], c[N];
-    unpack(*p1, a, (T*)nullptr);
-    unpack(*p2, c, (T*)nullptr);
-    const float* ct = cs + tl * half + vi * N;
-    const float* st = sn + tl * half + vi * N;
-    float o1[N], o2[N];
-#pragma unroll
-    for (int e = 0; e < N; ++e) {
-      o1[e] = a[e] * ct[e] - c[e] * st[e];
-      o2[e] = c[e] * ct[e] + a[e] * st[e];
-    }
-    *p1 = pack(o1, (T*)nullptr);
-    *p2 = pack(o2, (T*)nullptr);
-  }
+__device__ __forceinline__ T* head_row(T* q, T* k, int Hq, int Hkv, int d, long long bt, int h) {
+  return h < Hq ? q + (bt * Hq + h) * d : k + (bt * Hkv + (h - Hq)) * d;
 }
 
 template <typename T>
 __global__ void __launch_bounds__(kRopeThreads)
     rope_kernel(T* q, T* k, const uint8_t* tmask, long long tmask_bs, const uint8_t* pmask,
-                long long pmask_bs, int S, int P, int Hq, int Hkv, int d, double log2_base,
-                int32_t* pos_out) {
-  extern __shared__ float tab[];                // cos [32][d/2] | sin [32][d/2]
+                long long pmask_bs, int S, int P, int Hq, int Hkv, int d, int tok_per_cta,
+                double log2_base, int32_t* pos_out) {
+  constexpr int N = Vec<T>::N;
+  __shared__ double s_inv[128];                 // base^(-2i/d), i < d/2 <= 128
   __shared__ int s_count[kRopeThreads / 32];
-  __shared__ int s_pos[kRopeTokens];
   const int b = blockIdx.y;
-  const int t0 = blockIdx.x * kRopeTokens;
-  const int nt = min(kRopeTokens, S - t0);
+  const int t0 = blockIdx.x * tok_per_cta;
+  const int nt = min(tok_per_cta, S - t0);
   const int half = d / 2;
+  const int vpr = half / N;                     // vectors per half row
+  const int tl = threadIdx.x / vpr, vi = threadIdx.x % vpr;
+  const bool active = tl < nt;
+  const int Ht = Hq + (k ? Hkv : 0);
+  const long long bt = (long long)b * S + t0 + tl;
   const uint8_t* tm = tmask + (long long)b * tmask_bs;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-  // Valid tokens before the chunk (and valid prefix tokens): block count.
+  uint4 ra[kRopeHeadBatch], rc[kRopeHeadBatch];
+  auto load_batch = [&](int h0) {
+#pragma unroll
+    for (int j = 0; j < kRopeHeadBatch; ++j) {
+      if (active && h0 + j < Ht) {
+        const T* row = head_row(q, k, Hq, Hkv, d, bt, h0 + j);
+        ra[j] = *reinterpret_cast<const uint4*>(row + vi * N);
+        rc[j] = *reinterpret_cast<const uint4*>(row + half + vi * N);
+      }
+    }
+  };
+  load_batch(0);
+
+  // Valid tokens before the CTA's first token (and valid prefix tokens).
   int cnt = 0;
   for (int t = threadIdx.x; t < t0; t += blockDim.x) cnt += tm[t] != 0;
   if (pmask) {
@@ -107,43 +104,47 @@ __global__ void __launch_bounds__(kRopeThreads)
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
   if (lane == 0) s_count[warp] = cnt;
+  for (int i = threadIdx.x; i < half; i += blockDim.x)
+    s_inv[i] = exp2(-2.0 * (double)i / (double)d * log2_base);
   __syncthreads();
-  if (warp == 0) {
-    int base = 0;
+  if (!active) return;
+  int pos = -1;
 #pragma unroll
-    for (int w = 0; w < kRopeThreads / 32; ++w) base += s_count[w];
-    // inclusive scan of the chunk's own mask bits
-    int v = (lane < nt && tm[t0 + lane] != 0) ? 1 : 0;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, v, off);
-      if (lane >= off) v += y;
-    }
-    if (lane < nt) {
-      const int pos = base + v - 1;
-      s_pos[lane] = pos;
-      if (pos_out) pos_out[(long long)b * S + t0 + lane] = pos;
-    }
-  }
-  __syncthreads();
+  for (int w = 0; w < kRopeThreads / 32; ++w) pos += s_count[w];
+  for (int u = 0; u <= tl; ++u) pos += tm[t0 + u] != 0;
+  if (pos_out && vi == 0) pos_out[bt] = pos;
 
-  // cos / sin table for the chunk: angle = pos * base^(-2i/d), reduced in fp64.
-  float* cs = tab;
-  float* sn = tab + kRopeTokens * half;
   const double two_pi = 6.283185307179586476925286766559;
-  for (int idx = threadIdx.x; idx < nt * half; idx += blockDim.x) {
-    const int tl = idx / half, i = idx % half;
-    const double inv = exp2(-2.0 * (double)i / (double)d * log2_base);
-    double ang = (double)s_pos[tl] * inv;
-    ang -= two_pi * rint(ang / two_pi);
-    float sv, cv;
-    sincosf((float)ang, &sv, &cv);
-    cs[idx] = cv;
-    sn[idx] = sv;
+  const double inv_two_pi = 0.15915494309189533576888376337251;
+  float cs[N], sn[N];
+#pragma unroll
+  for (int e = 0; e < N; ++e) {
+    double ang = (double)pos * s_inv[vi * N + e];
+    ang -= two_pi * rint(ang * inv_two_pi);
+    sincosf((float)ang, &sn[e], &cs[e]);
   }
-  __syncthreads();
-  rope_rows(q, Hq, d, S, b, t0, nt, cs, sn);
-  if (k) rope_rows(k, Hkv, d, S, b, t0, nt, cs, sn);
+
+  for (int h0 = 0;;) {
+#pragma unroll
+    for (int j = 0; j < kRopeHeadBatch; ++j) {
+      if (h0 + j < Ht) {
+        float a[N], c[N], o1[N], o2[N];
+        unpack(ra[j], a, (T*)nullptr);
+        unpack(rc[j], c, (T*)nullptr);
+#pragma unroll
+        for (int e = 0; e < N; ++e) {
+          o1[e] = a[e] * cs[e] - c[e] * sn[e];
+          o2[e] = c[e] * cs[e] + a[e] * sn[e];
+        }
+        T* row = head_row(q, k, Hq, Hkv, d, bt, h0 + j);
+        *reinterpret_cast<uint4*>(row + vi * N) = pack(o1, (T*)nullptr);
+        *reinterpret_cast<uint4*>(row + half + vi * N) = pack(o2, (T*)nullptr);
+      }
+    }
+    h0 += kRopeHeadBatch;
+    if (h0 >= Ht) break;
+    load_batch(h0);
+  }
 }
 
 template <typename T>
@@ -182,17 +183,18 @@ __global__ void __launch_bounds__(256)
 }  // namespace
 
 cudaError_t launch_rope(const RopeParams& p, cudaStream_t st) {
-  dim3 grid((p.S + kRopeTokens - 1) / kRopeTokens, p.B);
-  const size_t smem = (size_t)2 * kRopeTokens * (p.d / 2) * sizeof(float);
+  const int vpr = p.d / 2 / (p.f32 ? Vec<float>::N : Vec<__nv_bfloat16>::N);
+  const int tok = std::max(1, std::min(kRopeMaxTok, kRopeThreads / vpr));
+  dim3 grid((p.S + tok - 1) / tok, p.B);
   const double log2_base = log2((double)p.base);
   if (p.f32) {
-    rope_kernel<float><<<grid, kRopeThreads, smem, st>>>(
+    rope_kernel<float><<<grid, kRopeThreads, 0, st>>>(
         static_cast<float*>(p.q), static_cast<float*>(p.k), p.tmask, p.tmask_bs, p.pmask,
-        p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, log2_base, p.pos_out);
+        p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, tok, log2_base, p.pos_out);
   } else {
-    rope_kernel<__nv_bfloat16><<<grid, kRopeThreads, smem, st>>>(
+    rope_kernel<__nv_bfloat16><<<grid, kRopeThreads, 0, st>>>(
         static_cast<__nv_bfloat16*>(p.q), static_cast<__nv_bfloat16*>(p.k), p.tmask, p.tmask_bs,
-        p.pmask, p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, log2_base, p.pos_out);
+        p.pmask, p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, tok, log2_base, p.pos_out);
   }
   return cudaGetLastError();
 }
