@@ -254,6 +254,9 @@ int pi_rope_inplace(const pi_rope_desc* d, void* q, void* k, const uint8_t* toke
   if (!(d->base > 1.f) || !std::isfinite(d->base)) return PI_ERR_ARG;
   if (d->dtype != PI_BF16 && d->dtype != PI_F32) return PI_ERR_UNSUPPORTED;
   if (d->d > 256 || d->d % 16 != 0 || d->B > 65535) return PI_ERR_UNSUPPORTED;
+  if (((size_t)d->Hq + (k ? (size_t)d->Hkv : 0)) * d->d * (d->dtype == PI_F32 ? 4 : 2) >
+      rope_max_smem())
+    return PI_ERR_UNSUPPORTED;
   if (d->mask_batch_stride < 0 || (d->mask_batch_stride != 0 && d->mask_batch_stride < d->S))
     return PI_ERR_ARG;
   if (d->prefix_batch_stride < 0 ||
@@ -275,7 +278,9 @@ int pi_rope_inplace(const pi_rope_desc* d, void* q, void* k, const uint8_t* toke
   p.B = d->B; p.S = d->S; p.P = d->P; p.Hq = d->Hq; p.Hkv = d->Hkv; p.d = d->d;
   p.base = d->base;
   p.f32 = d->dtype == PI_F32;
-  return launched(launch_rope(p, static_cast<cudaStream_t>(stream)));
+  DevCtl ctl;
+  if (!make_ctl(&ctl)) return PI_ERR_CUDA;
+  return launched(launch_rope(p, ctl, static_cast<cudaStream_t>(stream)));
 }
 
 int pi_euler_update(float* x, const void* v, int32_t v_dtype, float dt, int64_t n,

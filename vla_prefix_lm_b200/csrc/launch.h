@@ -50,7 +50,9 @@ struct RopeParams {
   bool f32;
 };
 
-cudaError_t launch_rope(const RopeParams& p, cudaStream_t st);
+cudaError_t launch_rope(const RopeParams& p, const DevCtl& ctl, cudaStream_t st);
+// Shared memory one RoPE CTA may use: (Hq + Hkv) * d * element size must fit.
+size_t rope_max_smem();
 
 // x (fp32) += dt * v (bf16 or fp32), n elements.
 cudaError_t launch_euler(float* x, const void* v, bool v_f32, float dt, long long n,
