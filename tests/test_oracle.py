@@ -553,6 +553,13 @@ def test_rope_closed_forms():
     e = np.zeros((1, 1, 1, 16)); e[..., 0] = 1.0
     z = prepost.rope(e, np.array([[np.pi / 2]]))
     np.testing.assert_allclose(z[0, 0, 0, [0, 8]], [0.0, 1.0], atol=1e-15)
+    # pair 4 of d = 16 has frequency 10000^(-8/16) = 1/100: position 50*pi
+    # turns it by a quarter turn, while pair 0 turns by 50*pi (25 whole turns:
+    # unchanged).  A wrong exponent (-i/d, or base^(+2i/d)) fails here.
+    e4 = np.zeros((1, 1, 1, 16)); e4[..., 4] = 1.0; e4[..., 0] = 1.0
+    z4 = prepost.rope(e4, np.array([[50 * np.pi]]))
+    np.testing.assert_allclose(z4[0, 0, 0, [4, 12]], [0.0, 1.0], atol=1e-12)
+    np.testing.assert_allclose(z4[0, 0, 0, [0, 8]], [1.0, 0.0], atol=1e-12)
 
 
 def test_rope_scores_depend_only_on_relative_position():
