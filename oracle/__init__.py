@@ -24,6 +24,15 @@ Parity status per function (what pins it; tests live in tests/test_oracle.py):
   invariances (duplicated heads, key permutation inside a bidirectional
   block), equality with torch's scaled_dot_product_attention in float64, the
   log-sum-exp against scipy, and suffix-pass == prefill suffix rows.
+* ``backward.prefill_backward`` -- pinned: central finite differences of
+  ``prefill`` on tiny inputs (every element of dq, dk, dv), torch autograd
+  through float64 scaled_dot_product_attention with the oracle's mask, and the
+  closed forms sum_j dK_j = 0 (softmax is shift-invariant in the keys) and
+  sum_j dV_j = sum of dO over the rows that see a key.
+* ``prepost.positions`` / ``rope`` / ``euler_step`` -- pinned: a worked
+  positions example with padding and a padded prefix, RoPE's closed forms
+  (identity at 0, pair norms kept, a stated turn of pairs 0 and 4), the
+  relative-position property, and the Euler loop against the exact solution.
 * ``counts.control_step_pairs`` -- parity unpinned: the pages quote about
   1.2e6 pairs per pi0.5 control step without a derivation; the count is only
   checked to be of that order.
@@ -41,4 +50,4 @@ from .attention import (  # noqa: F401
     suffix,
     suffix_mask,
 )
-from . import brute, counts  # noqa: F401
+from . import backward, brute, counts, prepost  # noqa: F401

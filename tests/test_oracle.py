@@ -584,3 +584,108 @@ def test_euler_step_reaches_the_ode_solution():
     for _ in range(10):
         y = prepost.euler_step(y, v, -0.1)
     np.testing.assert_allclose(y, x - v, atol=1e-12)
+
+
+# --------------------------------------------------------------- backward (f2)
+
+from oracle import backward  # noqa: E402
+
+
+def _fd_grads(q, k, v, ar, seg, dout, scale, eps=1e-6):
+    """Central differences of L = sum(dout * prefill(q, k, v)) -- uses only the
+    forward, so it is independent of the backward's formulas."""
+    def loss(q_, k_, v_):
+        out, _ = oracle.prefill(q_, k_, v_, ar, seg, scale=scale)
+        return float(np.sum(dout * out))
+    grads = []
+    for which in range(3):
+        xs = [q.copy(), k.copy(), v.copy()]
+        g = np.zeros_like(xs[which])
+        it = np.nditer(xs[which], flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            x0 = xs[which][idx]
+            xs[which][idx] = x0 + eps
+            lp = loss(*xs)
+            xs[which][idx] = x0 - eps
+            lm = loss(*xs)
+            xs[which][idx] = x0
+            g[idx] = (lp - lm) / (2 * eps)
+        grads.append(g)
+    return grads
+
+
+def _tiny_case(seed=40):
+    rng = np.random.default_rng(seed)
+    B, S, Hq, Hkv, d = 2, 7, 4, 2, 3
+    ar = [0, 0, 1, 1, 0, 1, 0]
+    seg = [OTHER, OTHER, FAST, FAST, EXPERT, EXPERT, -1]        # a padded token at the end
+    q = _rand((B, S, Hq, d), rng)
+    k = _rand((B, S, Hkv, d), rng)
+    v = _rand((B, S, Hkv, d), rng)
+    dout = _rand((B, S, Hq, d), rng)
+    return q, k, v, ar, seg, dout
+
+
+def test_backward_equals_finite_differences():
+    """Every element of dq, dk, dv against central differences of the forward,
+    on a layout with a bidirectional prefix, a causal block, the expert <- FAST
+    hole and a padded token."""
+    q, k, v, ar, seg, dout = _tiny_case()
+    dq, dk, dv = backward.prefill_backward(q, k, v, ar, dout, seg=seg, scale=0.7)
+    fq, fk, fv = _fd_grads(q, k, v, ar, seg, dout, 0.7)
+    np.testing.assert_allclose(dq, fq, atol=1e-8)
+    np.testing.assert_allclose(dk, fk, atol=1e-8)
+    np.testing.assert_allclose(dv, fv, atol=1e-8)
+    # the padded token neither receives nor passes gradient
+    assert np.all(dq[:, -1] == 0) and np.all(dk[:, -1] == 0) and np.all(dv[:, -1] == 0)
+
+
+def test_backward_planted_transposed_mask_fails_finite_differences(monkeypatch):
+    q, k, v, ar, seg, dout = _tiny_case()
+    fq, fk, fv = _fd_grads(q, k, v, ar, seg, dout, 0.7)
+    good = backward.prefill_mask
+    monkeypatch.setattr(backward, "prefill_mask",
+                        lambda *a, **kw: np.swapaxes(good(*a, **kw), 1, 2))
+    dq, dk, dv = backward.prefill_backward(q, k, v, ar, dout, seg=seg, scale=0.7)
+    assert np.abs(dq - fq).max() > 1e-3 or np.abs(dk - fk).max() > 1e-3
+
+
+@pytest.mark.parametrize("Hq,Hkv,scale", [(8, 1, 1.0), (4, 2, 0.37)])
+def test_backward_equals_torch_autograd_float64(Hq, Hkv, scale):
+    """Library special case: autograd through float64 torch SDPA with the
+    explicit mask, on a pi0-like layout (bidirectional prefix, state, actions)."""
+    rng = np.random.default_rng(41)
+    B, S, d = 2, 40, 16
+    ar = [0] * 30 + [1] + [1] + [0] * 8
+    q = _rand((B, S, Hq, d), rng)
+    k = _rand((B, S, Hkv, d), rng)
+    v = _rand((B, S, Hkv, d), rng)
+    dout = _rand((B, S, Hq, d), rng)
+    dq, dk, dv = backward.prefill_backward(q, k, v, ar, dout, scale=scale)
+    M = torch.from_numpy(np.array(brute.mask(ar)))
+    tq, tk, tv = (torch.from_numpy(x).permute(0, 2, 1, 3).clone().requires_grad_(True)
+                  for x in (q, k, v))
+    out = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk, tv, attn_mask=M, scale=scale, enable_gqa=True)
+    out.backward(torch.from_numpy(dout).permute(0, 2, 1, 3))
+    for mine, t in ((dq, tq), (dk, tk), (dv, tv)):
+        np.testing.assert_allclose(mine, t.grad.permute(0, 2, 1, 3).numpy(), atol=1e-11)
+
+
+def test_backward_closed_forms():
+    """Softmax is invariant to adding one vector to every key a row sees, so
+    the key gradients of each (batch, kv head) sum to zero; the value
+    gradients sum to the sum of dO over the rows that see any key."""
+    rng = np.random.default_rng(42)
+    B, S, Hq, Hkv, d = 2, 23, 4, 1, 8
+    ar = [0] * 10 + [1] * 5 + [1] + [0] * 7
+    seg = [OTHER] * 10 + [FAST] * 5 + [EXPERT] * 7 + [-1]
+    q = _rand((B, S, Hq, d), rng)
+    k = _rand((B, S, Hkv, d), rng)
+    v = _rand((B, S, Hkv, d), rng)
+    dout = _rand((B, S, Hq, d), rng)
+    dq, dk, dv = backward.prefill_backward(q, k, v, ar, dout, seg=seg, scale=0.5)
+    np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-12)
+    live = np.array([s >= 0 for s in seg])
+    np.testing.assert_allclose(dv.sum(axis=1)[:, 0], dout[:, live].sum(axis=(1, 2)), atol=1e-12)
