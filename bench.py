@@ -280,6 +280,7 @@ def run_ours(args, rank, ws, local):
     suffix = suffix_control(args, dev, stream, rank)
     decode = decode_steps(args, dev, stream, rank)
     prepost = prepost_steps(args, dev, stream, rank)
+    bwd = backward_steps(args, dev, stream, rank)
 
     traffic = TRAFFIC["bytes"] if TRAFFIC["src_sha"] == kernel_digest() else None
     line = {
@@ -330,6 +331,7 @@ def run_ours(args, rank, ws, local):
         "suffix_ctrl": suffix,
         "decode": decode,
         "prepost": prepost,
+        "backward": bwd,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, seconds=args.cpu_seconds)
@@ -446,6 +448,68 @@ def prepost_steps(args, dev, stream, rank):
         "us_per_ctrl": us_ctrl, "gpu_launches_per_ctrl": 3 * w.calls,
         "timing": f"one graph of 30 launches replayed {reps}x (warm L2)"}
     return res
+
+
+def backward_steps(args, dev, stream, rank):
+    """Gradient of the pi0 joint prefill (B=8, S=611): dq, dk, dv from the
+    forward's out and lse, fp32 SIMT.  Visible-pair work: five dot products or
+    updates of length d per (query head, visible key) -- the scores, dP, dV,
+    dQ and dK -- 10 * d FLOP per pair."""
+    import torch
+
+    from vla_prefix_lm_b200 import binding, dist
+    from vla_prefix_lm_b200 import workloads as W
+
+    w = W.workload(2)
+    x = W.prefill_inputs(w, W.seed_for(2, 555) + rank * 7, B=w.B)
+    q, k, v, ar = x.q.to(dev), x.k.to(dev), x.v.to(dev), x.ar.to(dev)
+    dout, _ = W.draw(tuple(x.q.shape), 9201 + rank, w.d, w.dtype, 0.5)
+    dout = dout.to(dev)
+    lse = torch.empty((w.B, w.Sq, w.Hq), dtype=torch.float32, device=dev)
+    out = binding.pi_attn_prefill(q, k, v, ar, lse=lse, stream=stream)
+    wsb = torch.empty(binding.pi_attn_prefill_backward_workspace_bytes(q, k, ar),
+                      dtype=torch.uint8, device=dev)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=dev)
+
+    def step():
+        binding.pi_attn_prefill_backward(q, k, v, ar, out, lse, dout, dq=dq, dk=dk, dv=dv,
+                                         workspace=wsb, stream=stream)
+
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    reps = 3
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us = dist.max_over_ranks(e0.elapsed_time(e1) * 1e3 / reps)
+    assert binding.pi_attn_read_status(stream) == binding.PI_OK
+    pairs = visible_pairs_per_bh(w.ar) * w.B * w.Hq
+    flops = 10 * w.d * pairs
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            sm_mhz = float(json.load(f).get("sm_max_mhz", 1965.0))
+    except (OSError, ValueError):
+        sm_mhz = 1965.0
+    fp32_peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12       # FFMA lanes x 2 FLOP x clock
+    return {
+        "workload": "pi0 joint prefill backward: B=8, S=611, Hq=8, d=256, bf16 in, fp32 grads",
+        "us_per_call": us,
+        "tflops": flops / (us / 1e6) / 1e12,
+        "bound": "alu",
+        "fp32_fma_peak_tflops": fp32_peak,
+        "frac_of_fp32_peak": flops / (us / 1e6) / 1e12 / fp32_peak,
+        "algorithmic_flop_per_call": flops,
+        "gpu_launches_per_call": 3,
+        "timing": f"{reps} calls back to back after one warm-up (warm L2)",
+    }
 
 
 def decode_steps(args, dev, stream, rank):

@@ -133,6 +133,39 @@ int pi_attn_prefill(const pi_attn_desc* desc, const void* q, const void* k, cons
                     pi_stream_t stream);
 
 /*
+ * pi_attn_prefill_backward -- gradient of pi_attn_prefill with respect to q,
+ * k and v, for training.
+ * Source: "VLA 代码精读 - OpenPI & StarVLA", 1.5 Pi0.compute_loss runs the
+ * joint forward under gradient; the pages print no backward, so this is the
+ * plain derivative of the forward: with P the softmax over the visible keys,
+ * dS = P * (dO v^T - rowsum(dO * out)), dq = scale dS k, dk = scale dS^T q,
+ * dv = P^T dO, the key/value gradients summed over the query heads of each
+ * key/value head.
+ *
+ *   desc        as pi_attn_prefill (P = 0); dtype bf16 or fp32, any Hq that
+ *               Hkv divides, d a multiple of 32 up to 256, S <= 16383
+ *   q, k, v, ar_mask, segment_ids   the forward's inputs, same layouts
+ *   out  [B, S, Hq, d], lse [B, S, Hq] fp32   the forward's outputs (required)
+ *   dout [B, S, Hq, d]  same dtype as q       (gradient of the loss w.r.t. out)
+ *   dq   [B, S, Hq, d]  fp32                  (written)
+ *   dk, dv [B, S, Hkv, d] fp32                (written; not accumulated into)
+ *   workspace   device scratch of pi_attn_prefill_backward_workspace_bytes(desc)
+ *               bytes, 16-byte aligned, caller-owned, contents ignored
+ * Padding tokens (negative segment id) get zero gradients.  The result does not
+ * depend on launch timing (no atomics).  Errors: PI_ERR_ARG (bad descriptor,
+ * NULL pointer, workspace too small), PI_ERR_ALIGN (a tensor or the workspace
+ * not 16-byte aligned, lse / segment_ids not 4-byte aligned),
+ * PI_ERR_UNSUPPORTED (geometry above), PI_ERR_CUDA (launch failure); all
+ * before anything is enqueued except the last.
+ */
+size_t pi_attn_prefill_backward_workspace_bytes(const pi_attn_desc* desc);
+int pi_attn_prefill_backward(const pi_attn_desc* desc, const void* q, const void* k,
+                             const void* v, const uint8_t* ar_mask, const int32_t* segment_ids,
+                             const void* out, const float* lse, const void* dout, float* dq,
+                             float* dk, float* dv, void* workspace, size_t ws_bytes,
+                             pi_stream_t stream);
+
+/*
  * pi_attn_suffix -- suffix-only pass against a prefix KV cache (mode 2), the
  * call each Euler flow-matching step makes.
  * Source: "VLA 代码精读 - OpenPI & StarVLA", 1.6 Pi0.sample_actions: the key

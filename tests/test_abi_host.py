@@ -163,3 +163,45 @@ def test_rope_and_euler_argument_errors():
     assert eu(FAKE, FAKE, b.PI_F32, ctypes.c_float(float("nan")), 16, None) == b.PI_ERR_ARG
     assert eu(FAKE_MIS, FAKE, b.PI_F32, ctypes.c_float(0.1), 16, None) == b.PI_ERR_ALIGN
     assert eu(None, None, b.PI_F32, ctypes.c_float(0.1), 0, None) == b.PI_OK
+
+
+def test_rope_rejects_heads_beyond_shared_memory():
+    b, L = _lib()
+    desc = _rope_desc(b, Hq=200, d=256, dtype=b.PI_F32)   # 201 KB per token
+    assert L.pi_rope_inplace(ctypes.byref(desc), FAKE, FAKE, FAKE, None, None, None) == \
+        b.PI_ERR_UNSUPPORTED
+
+
+def test_backward_argument_errors():
+    """Every host-side check of pi_attn_prefill_backward, before any launch."""
+    b, L = _lib()
+    ws = L.pi_attn_prefill_backward_workspace_bytes
+    need = ws(ctypes.byref(_desc(b)))
+    assert need == 256 + 2 * 16 * 8 * 4            # codes (rounded to 256) + D
+
+    def bwd(desc, ws_bytes=need, ptrs=None, seg=None, lse=FAKE):
+        p = dict(q=FAKE, k=FAKE, v=FAKE, ar=FAKE, out=FAKE, dout=FAKE, dq=FAKE, dk=FAKE,
+                 dv=FAKE, w=FAKE)
+        p.update(ptrs or {})
+        return L.pi_attn_prefill_backward(
+            ctypes.byref(desc) if desc is not None else None, p["q"], p["k"], p["v"], p["ar"],
+            seg, p["out"], lse, p["dout"], p["dq"], p["dk"], p["dv"], p["w"], ws_bytes, None)
+
+    assert bwd(None) == b.PI_ERR_ARG
+    assert bwd(_desc(b, P=3)) == b.PI_ERR_ARG
+    assert bwd(_desc(b, Hq=6, Hkv=4)) == b.PI_ERR_ARG
+    assert bwd(_desc(b, softmax_scale=0.0)) == b.PI_ERR_ARG
+    assert bwd(_desc(b, mask_batch_stride=3)) == b.PI_ERR_ARG
+    assert bwd(_desc(b, d=48)) == b.PI_ERR_UNSUPPORTED
+    assert bwd(_desc(b, d=512)) == b.PI_ERR_UNSUPPORTED
+    assert bwd(_desc(b, dtype=7)) == b.PI_ERR_UNSUPPORTED
+    assert bwd(_desc(b, Sq=16384)) == b.PI_ERR_UNSUPPORTED
+    assert bwd(_desc(b), lse=None) == b.PI_ERR_ARG
+    assert bwd(_desc(b), ws_bytes=need - 1) == b.PI_ERR_ARG
+    for name in ("q", "dout", "dq", "dk", "dv", "w"):
+        assert bwd(_desc(b), ptrs={name: FAKE_MIS}) == b.PI_ERR_ALIGN, name
+        assert bwd(_desc(b), ptrs={name: None}) == b.PI_ERR_ARG, name
+    assert bwd(_desc(b), seg=ctypes.c_void_p(0x10002)) == b.PI_ERR_ALIGN
+    assert bwd(_desc(b, B=0), ptrs={"q": None}) == b.PI_OK
+    # fp32 and grouped heads are in range of the backward (unlike the bf16 forward)
+    assert ws(ctypes.byref(_desc(b, dtype=b.PI_F32, Hq=4, Hkv=2, d=64))) > 0

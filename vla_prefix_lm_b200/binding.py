@@ -36,6 +36,8 @@ EXPORTED = (
     "pi_attn_suffix_noalloc",
     "pi_rope_inplace",
     "pi_euler_update",
+    "pi_attn_prefill_backward",
+    "pi_attn_prefill_backward_workspace_bytes",
     "pi_attn_suffix_noalloc_capacity",
 )
 
@@ -112,6 +114,10 @@ def lib() -> ctypes.CDLL:
         L.pi_euler_update.restype = i32
         L.pi_attn_suffix_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.pi_attn_suffix_noalloc.restype = i32
+        L.pi_attn_prefill_backward_workspace_bytes.argtypes = [dp]
+        L.pi_attn_prefill_backward_workspace_bytes.restype = sz
+        L.pi_attn_prefill_backward.argtypes = [dp] + [vp] * 12 + [sz, vp]
+        L.pi_attn_prefill_backward.restype = i32
         L.pi_attn_suffix_noalloc_capacity.argtypes = []
         L.pi_attn_suffix_noalloc_capacity.restype = sz
         _lib = L
@@ -191,6 +197,59 @@ def pi_attn_prefill(q, k, v, ar_mask, segment_ids=None, out=None, lse=None,
     if rc != PI_OK:
         raise PiAttnError(rc, "pi_attn_prefill")
     return out
+
+
+def pi_attn_prefill_backward_workspace_bytes(q, k, ar_mask, softmax_scale=1.0):
+    B, S, Hq, d = q.shape
+    desc = PiAttnDesc(B, S, 0, Hq, k.shape[2], d, _dtype_code(q), float(softmax_scale),
+                      _mask_stride(ar_mask, B, S))
+    return int(lib().pi_attn_prefill_backward_workspace_bytes(ctypes.byref(desc)))
+
+
+def pi_attn_prefill_backward(q, k, v, ar_mask, out, lse, dout, segment_ids=None, dq=None,
+                             dk=None, dv=None, workspace=None, softmax_scale=1.0, stream=None):
+    """Gradient of pi_attn_prefill: (dq, dk, dv) in fp32, allocated if None.
+    ``out`` and ``lse`` are the forward's outputs for the same inputs; ``dout``
+    has q's dtype and shape.  ``workspace``: a CUDA uint8 tensor of at least
+    pi_attn_prefill_backward_workspace_bytes (allocated here if None)."""
+    _need(q, "q", dims=4)
+    _need(k, "k", q.dtype, 4)
+    _need(v, "v", q.dtype, 4)
+    _need(out, "out", q.dtype, 4)
+    _need(dout, "dout", q.dtype, 4)
+    _need(lse, "lse", torch.float32)
+    _need(ar_mask, "ar_mask", torch.uint8)
+    B, S, Hq, d = q.shape
+    if k.shape != v.shape or k.shape[0] != B or k.shape[1] != S or k.shape[3] != d:
+        raise ValueError("k/v shape mismatch")
+    if out.shape != q.shape or dout.shape != q.shape or tuple(lse.shape) != (B, S, Hq):
+        raise ValueError("out/dout must have q's shape and lse must be [B, S, Hq]")
+    mbs = _mask_stride(ar_mask, B, S)
+    if segment_ids is not None:
+        _need(segment_ids, "segment_ids", torch.int32)
+        if segment_ids.shape != ar_mask.shape:
+            raise ValueError("segment_ids must have ar_mask's shape")
+    desc = PiAttnDesc(B, S, 0, Hq, k.shape[2], d, _dtype_code(q), float(softmax_scale), mbs)
+    need = int(lib().pi_attn_prefill_backward_workspace_bytes(ctypes.byref(desc)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    f32 = torch.float32
+    dq = torch.empty(q.shape, dtype=f32, device=q.device) if dq is None else dq
+    dk = torch.empty(k.shape, dtype=f32, device=q.device) if dk is None else dk
+    dv = torch.empty(v.shape, dtype=f32, device=q.device) if dv is None else dv
+    _need(dq, "dq", f32, 4)
+    _need(dk, "dk", f32, 4)
+    _need(dv, "dv", f32, 4)
+    if dq.shape != q.shape or dk.shape != k.shape or dv.shape != v.shape:
+        raise ValueError("dq/dk/dv must have the shapes of q/k/v")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().pi_attn_prefill_backward(
+        ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(ar_mask), _ptr(segment_ids),
+        _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+        ws_bytes, ctypes.c_void_p(_stream(stream)))
+    if rc != PI_OK:
+        raise PiAttnError(rc, "pi_attn_prefill_backward")
+    return dq, dk, dv
 
 
 def _suffix_desc(q_suf, k_suf, k_cache, ar_mask_suf, softmax_scale):

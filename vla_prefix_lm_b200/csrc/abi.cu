@@ -107,6 +107,20 @@ int check_desc(const pi_attn_desc* d, bool suffix) {
 
 int launched(cudaError_t e) { return e == cudaSuccess ? PI_OK : PI_ERR_CUDA; }
 
+int check_backward_desc(const pi_attn_desc* d) {
+  if (!d) return PI_ERR_ARG;
+  if (d->B < 0 || d->Sq < 0 || d->P != 0 || d->Hq <= 0 || d->Hkv <= 0 || d->d <= 0)
+    return PI_ERR_ARG;
+  if (d->Hq % d->Hkv != 0) return PI_ERR_ARG;
+  if (!std::isfinite(d->softmax_scale) || !(d->softmax_scale > 0.f)) return PI_ERR_ARG;
+  if (d->mask_batch_stride < 0 || (d->mask_batch_stride != 0 && d->mask_batch_stride < d->Sq))
+    return PI_ERR_ARG;
+  if (d->dtype != PI_BF16 && d->dtype != PI_F32) return PI_ERR_UNSUPPORTED;
+  if (d->Sq > kMaxTokens || d->d % 32 != 0 || d->d > 256) return PI_ERR_UNSUPPORTED;
+  if ((long long)d->B * d->Sq * d->Hq / 8 >= (1ll << 31)) return PI_ERR_UNSUPPORTED;
+  return PI_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -291,6 +305,41 @@ int pi_euler_update(float* x, const void* v, int32_t v_dtype, float dt, int64_t 
   if (!x || !v) return PI_ERR_ARG;
   if (!aligned16(x) || !aligned16(v)) return PI_ERR_ALIGN;
   return launched(launch_euler(x, v, v_dtype == PI_F32, dt, n, static_cast<cudaStream_t>(stream)));
+}
+
+size_t pi_attn_prefill_backward_workspace_bytes(const pi_attn_desc* d) {
+  if (check_backward_desc(d) != PI_OK || d->B == 0 || d->Sq == 0) return 0;
+  return bwd_workspace_bytes(d->B, d->Sq, d->Hq);
+}
+
+int pi_attn_prefill_backward(const pi_attn_desc* d, const void* q, const void* k, const void* v,
+                             const uint8_t* ar_mask, const int32_t* segment_ids, const void* out,
+                             const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                             void* workspace, size_t ws_bytes, pi_stream_t stream) {
+  const int rc = check_backward_desc(d);
+  if (rc != PI_OK) return rc;
+  if (d->B == 0 || d->Sq == 0) return PI_OK;
+  if (!q || !k || !v || !ar_mask || !out || !lse || !dout || !dq || !dk || !dv || !workspace)
+    return PI_ERR_ARG;
+  const size_t need = bwd_workspace_bytes(d->B, d->Sq, d->Hq);
+  if (ws_bytes < need) return PI_ERR_ARG;
+  for (const void* ptr : {q, k, v, out, dout, (const void*)dq, (const void*)dk, (const void*)dv,
+                          (const void*)workspace})
+    if (!aligned16(ptr)) return PI_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (segment_ids && (reinterpret_cast<uintptr_t>(segment_ids) & 3u)))
+    return PI_ERR_ALIGN;
+  BwdParams p;
+  p.q = q; p.k = k; p.v = v; p.out = out; p.dout = dout; p.lse = lse;
+  p.ar = ar_mask; p.seg = segment_ids; p.mask_bs = d->mask_batch_stride;
+  p.dq = dq; p.dk = dk; p.dv = dv;
+  p.codes = static_cast<uint32_t*>(workspace);
+  const size_t codes_bytes = ((size_t)d->B * d->Sq * sizeof(uint32_t) + 255) & ~(size_t)255;
+  p.D = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + codes_bytes);
+  p.B = d->B; p.S = d->Sq; p.Hq = d->Hq; p.Hkv = d->Hkv; p.d = d->d;
+  p.scale = d->softmax_scale;
+  p.f32 = d->dtype == PI_F32;
+  return launched(launch_backward(p, static_cast<cudaStream_t>(stream)));
 }
 
 int pi_attn_debug_mask(const pi_attn_desc* d, int mode, const uint8_t* ar_mask,

@@ -50,6 +50,21 @@ struct RopeParams {
   bool f32;
 };
 
+// Gradient of the prefill attention (backward.cu).
+struct BwdParams {
+  const void* q; const void* k; const void* v; const void* out; const void* dout;
+  const float* lse;
+  const uint8_t* ar; const int32_t* seg; long long mask_bs;
+  float* dq; float* dk; float* dv;
+  uint32_t* codes;                 // workspace: [B, S] packed mask codes
+  float* D;                        // workspace: [B, S, Hq] rowsum(dO * O)
+  int B, S, Hq, Hkv, d;
+  float scale;
+  bool f32;
+};
+size_t bwd_workspace_bytes(int B, int S, int Hq);
+cudaError_t launch_backward(const BwdParams& p, cudaStream_t st);
+
 cudaError_t launch_rope(const RopeParams& p, const DevCtl& ctl, cudaStream_t st);
 // Shared memory one RoPE CTA may use: (Hq + Hkv) * d * element size must fit.
 size_t rope_max_smem();
