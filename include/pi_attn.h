@@ -68,7 +68,7 @@ enum pi_status {
   PI_OK = 0,
   PI_ERR_ARG = 1,         /* NULL pointer, bad shape, stride or size      */
   PI_ERR_ALIGN = 2,       /* a pointer is not 16-byte aligned             */
-  PI_ERR_UNSUPPORTED = 3, /* dtype / head geometry this build lacks       */
+  PI_ERR_UNSUPPORTED = 3, /* dtype / head geometry the library lacks     */
   PI_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed         */
   PI_ERR_TIMEOUT = 5      /* a device-side bounded wait ran out           */
 };
@@ -104,7 +104,7 @@ typedef struct pi_attn_desc {
 } pi_attn_desc;
 
 /*
- * Supported geometry in this build:
+ * Supported geometry:
  *   PI_BF16: Hkv == 1, d == 256, Hq in {1, 2, 4, 8, 16}; tokens Sq <= 16383
  *            (the in-kernel block index is 14 bits), P < 2^31 / Hq.
  *   PI_F32 : Hq % Hkv == 0, d in {32, 64, 128, 256}, Sq <= 16383.

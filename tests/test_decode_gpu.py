@@ -1,4 +1,4 @@
-"""Single-token decode against a growing cache (SURVEY NEXT row f4).
+"""Single-token decode against a growing cache.
 
 "Pi0-FAST 模型架构", 4.1 KV 缓存推理: after the prefix, FAST action tokens are
 decoded one at a time, each attending to the whole cache plus itself, and the
