@@ -646,6 +646,116 @@ def suffix_control(args, dev, stream, rank):
     }
 
 
+# ------------------------------------------------------- per-config table
+
+
+def oracle_seconds_per_call(w, x, max_rows, seconds=5.0):
+    """The oracle's wall time for one whole call of workload ``w``, estimated
+    from a bounded sample: ``max_rows`` query rows of batch element 0 (all
+    heads), timed for about ``seconds``, scaled by B * S / rows."""
+    import oracle
+
+    ar = np.array(w.ar)
+    seg = None if w.seg is None else np.array(w.seg)
+    S = w.Sq
+    n_rows = min(S, max_rows)
+    rows = [(0, int(i)) for i in np.linspace(0, S - 1, n_rows).round().astype(int)]
+    t0 = time.perf_counter()
+    n = 0
+    while n < 1 or time.perf_counter() - t0 < seconds:
+        oracle.prefill(x.q64[:1], x.k64[:1], x.v64[:1], ar, seg, scale=w.scale, rows=rows)
+        n += 1
+    dt = (time.perf_counter() - t0) / n
+    return dt * w.B * S / n_rows, (f"{n_rows} of {S} query rows (all heads) of 1 of {w.B} "
+                                   f"batch elements, {n} repeats, scaled to the whole call")
+
+
+def prefill_config_line(cfg, dev, stream, sets, reps, oracle_rows):
+    """Device time per call of one prefill workload, rotating over ``sets``
+    device-resident input sets, plus the oracle's estimated time per call."""
+    import torch
+
+    from vla_prefix_lm_b200 import binding
+    from vla_prefix_lm_b200 import workloads as W
+
+    w = W.workload(cfg)
+    P_ = peaks()
+    host = [W.prefill_inputs(w, W.seed_for(cfg, c), B=w.B) for c in range(sets)]
+    ins = []
+    for x in host:
+        seg = None if x.seg is None else x.seg.to(dev)
+        ins.append((x.q.to(dev), x.k.to(dev), x.v.to(dev), x.ar.to(dev), seg))
+    outs = [torch.empty_like(t[0]) for t in ins]
+
+    def call(i):
+        q, k, v, ar, seg = ins[i % sets]
+        binding.pi_attn_prefill(q, k, v, ar, segment_ids=seg, out=outs[i % sets],
+                                softmax_scale=w.scale, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(3, sets)):
+            call(i)
+    torch.cuda.synchronize()
+    n = sets * max(1, 8 // sets)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            call(i)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g.replay()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * n)
+    del g
+    assert binding.pi_attn_read_status(stream) == binding.PI_OK
+    elt = 2 if w.dtype == "bf16" else 4
+    pairs = visible_pairs_per_bh(w.ar, w.seg) * w.B * w.Hq
+    flops = 4 * w.d * pairs
+    nbytes = (2 * w.B * w.Sq * w.Hq * w.d + 2 * w.B * w.Sq * w.Hkv * w.d) * elt
+    o_s, sample = oracle_seconds_per_call(w, host[0], oracle_rows)
+    line = {
+        "config": cfg, "workload": f"{w.name}: {w.note}",
+        "shape": {"B": w.B, "S": w.Sq, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "dtype": w.dtype},
+        "us_per_call": us, "pairs_per_call": pairs, "pairs_per_s": pairs / (us / 1e6),
+        "tflops": flops / (us / 1e6) / 1e12, "gb_per_s_algorithmic": nbytes / (us / 1e6) / 1e9,
+        "timing": f"CUDA graph of {n} calls over {sets} input sets, replayed {reps}x",
+        "oracle_s_per_call": o_s, "oracle_sample": sample,
+        "oracle_cores": len(os.sched_getaffinity(0)),
+    }
+    if w.dtype == "bf16":
+        line["frac_of_bf16_peak"] = line["tflops"] / P_["bf16_tflops"]
+        line["frac_of_bf16_sustained"] = line["tflops"] / P_["bf16_tflops_sustained"]
+    if w.calls > 1:
+        line["us_per_workload"] = us * w.calls
+        line["calls"] = w.calls
+    return line
+
+
+def run_configs(args):
+    """One JSON line per workload config: device time, rates, roofline
+    fractions and the oracle's estimated time per call (one GPU, no ranks)."""
+    import torch
+
+    from vla_prefix_lm_b200 import binding
+
+    binding.lib()
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream()
+    plan = {1: (1, 200, 49), 2: (6, 50, 611), 4: (2, 20, 256), 5: (2, 5, 64)}
+    for cfg in (1, 2, 4, 5):
+        sets, reps, rows = plan[cfg]
+        print(json.dumps({"impl": "ours", "mode": "configs",
+                          **prefill_config_line(cfg, dev, stream, sets, reps, rows)}),
+              flush=True)
+    suffix = suffix_control(args, dev, stream, 0)
+    print(json.dumps({"impl": "ours", "mode": "configs", "config": 3, **suffix}), flush=True)
+
+
 # ------------------------------------------------------------ CPU baselines
 
 
@@ -720,12 +830,21 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--configs", action="store_true",
+                    help="instead of the bench line: one line per workload config (1 GPU)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
 
     from vla_prefix_lm_b200 import dist
     rank, ws, local = dist.world()
+    if args.configs:
+        dist.init()
+        try:
+            run_configs(args)
+        finally:
+            dist.shutdown()
+        return
     if args.impl == "reference":
         line = run_reference(args, rank, ws)
         if line is not None:

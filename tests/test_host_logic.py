@@ -127,3 +127,18 @@ def test_reference_arm_nonzero_rank_exits_quietly():
                         "--steps", "1", "--warmup", "0"], capture_output=True, text=True,
                        timeout=120, env=dict(os.environ, RANK="1", WORLD_SIZE="2"))
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_config_table_oracle_estimate_on_cpu():
+    """bench.py --configs: the oracle's per-call estimate runs on a bounded
+    row sample, and the pair count it reports equals the explicit oracle
+    mask's count."""
+    import bench
+    from vla_prefix_lm_b200 import workloads as W
+    w = W.workload(1)
+    x = W.prefill_inputs(w, W.seed_for(1, 0), B=w.B)
+    s, sample = bench.oracle_seconds_per_call(w, x, max_rows=16, seconds=0.05)
+    assert s > 0 and "16 of 49 query rows" in sample
+    w4 = W.workload(4)
+    M = oracle.prefill_mask(np.array(w4.ar), seg=np.array(w4.seg), B=1)
+    assert bench.visible_pairs_per_bh(w4.ar, w4.seg) == int(M.sum())
