@@ -23,6 +23,11 @@
  *   out[b,i,h,:] = sum_j softmax_j( scale * <q[b,i,h,:], k[b,j,g(h),:]> | visible(i,j) ) v[b,j,g(h),:]
  *   g(h) = h / (Hq / Hkv)
  *
+ * Around it (same page, 1.5 and 1.6): pi_rope_inplace rotates q and k at the
+ * positions cumsum(mask) - 1 (continued after the prefix in a suffix pass) and
+ * pi_euler_update takes the sampler's step x += dt * v.  For training (1.5),
+ * pi_attn_prefill_backward returns the gradient of the prefill.
+ *
  * Memory layout (all entry points): every tensor is a dense, contiguous,
  * caller-owned DEVICE buffer in token-major order [B, S, H, d] (d innermost,
  * then heads, then tokens, then batch).  ar_mask is uint8 (0 = False,
@@ -34,8 +39,9 @@
  * Ownership and threading: the library never allocates, frees or retains a
  * caller buffer; all work is enqueued on the caller's stream and the calls
  * return before it runs.  Buffers must stay valid until the stream reaches the
- * work.  Calls on different streams may run concurrently; the only global
- * state is the device status word read by pi_attn_read_status.
+ * work.  Calls on different streams may run concurrently; the global state is
+ * the device status word read by pi_attn_read_status, the wait bound set by
+ * pi_attn_set_wait_limit, and the fixed scratch of pi_attn_suffix_noalloc.
  *
  * Errors: every entry point returns PI_OK or a PI_ERR_* code.  Argument
  * errors are detected on the host before anything is enqueued (nothing is
