@@ -28,13 +28,13 @@ def _err(t, ref):
     return float(np.abs(t.float().cpu().numpy().astype(np.float64) - ref).max())
 
 
-@pytest.mark.parametrize("dtype,S,Hq,Hkv,d,tol", [("bf16", 611, 8, 1, 256, 2e-2),
-                                                   ("f32", 4250, 8, 1, 256, 1e-4),
-                                                   ("bf16", 97, 4, 2, 64, 2e-2),
-                                                   ("f32", 131, 11, 1, 48, 1e-4)])
-def test_rope_prefill_positions(dtype, S, Hq, Hkv, d, tol):
+@pytest.mark.parametrize("dtype,B,S,Hq,Hkv,d,tol", [("bf16", 8, 611, 8, 1, 256, 2e-2),
+                                                     ("f32", 2, 4250, 8, 1, 256, 1e-4),
+                                                     ("bf16", 2, 97, 4, 2, 64, 2e-2),
+                                                     ("f32", 2, 131, 11, 1, 48, 1e-4)])
+def test_rope_prefill_positions(dtype, B, S, Hq, Hkv, d, tol):
+    """The first case is the pi0 prefill at full size (the bench's RoPE leg)."""
     rng = np.random.default_rng(31)
-    B = 2
     mask = (rng.random((B, S)) < 0.9).astype(np.uint8)        # some padded tokens
     q, q64 = W.draw((B, S, Hq, d), 601, d, dtype)
     k, k64 = W.draw((B, S, Hkv, d), 602, d, dtype)
@@ -47,8 +47,9 @@ def test_rope_prefill_positions(dtype, S, Hq, Hkv, d, tol):
 
 
 def test_rope_suffix_positions_continue_after_prefix():
+    """One pi0 Euler step's suffix q/k at full size (B=32, 816 prefix tokens)."""
     rng = np.random.default_rng(32)
-    B, P, Sq, Hq, d = 4, 816, 51, 8, 256
+    B, P, Sq, Hq, d = 32, 816, 51, 8, 256
     pmask = (rng.random((B, P)) < 0.8).astype(np.uint8)
     smask = np.ones((B, Sq), np.uint8)
     q, q64 = W.draw((B, Sq, Hq, d), 611, d, "bf16")
