@@ -539,40 +539,95 @@ def test_positions_follow_the_pages():
     assert prepost.positions(sm, pm).tolist() == [[3, 4, 5], [4, 5, 6]]
 
 
-def test_rope_closed_forms():
-    rng = np.random.default_rng(21)
-    x = rng.standard_normal((2, 5, 3, 16))
-    # position 0 is the identity
-    assert np.allclose(prepost.rope(x, np.zeros((2, 5))), x, atol=0)
-    # each (i, i + d/2) pair is rotated: the pair's norm is kept
-    y = prepost.rope(x, rng.integers(0, 1000, (2, 5)))
-    n_x = x[..., :8] ** 2 + x[..., 8:] ** 2
-    n_y = y[..., :8] ** 2 + y[..., 8:] ** 2
-    np.testing.assert_allclose(n_y, n_x, rtol=1e-12)
-    # pair 0 turns by exactly pos radians (frequency base^0 = 1), counter-clockwise
-    e = np.zeros((1, 1, 1, 16)); e[..., 0] = 1.0
-    z = prepost.rope(e, np.array([[np.pi / 2]]))
-    np.testing.assert_allclose(z[0, 0, 0, [0, 8]], [0.0, 1.0], atol=1e-15)
-    # pair 4 of d = 16 has frequency 10000^(-8/16) = 1/100: position 50*pi
-    # turns it by a quarter turn, while pair 0 turns by 50*pi (25 whole turns:
-    # unchanged).  A wrong exponent (-i/d, or base^(+2i/d)) fails here.
-    e4 = np.zeros((1, 1, 1, 16)); e4[..., 4] = 1.0; e4[..., 0] = 1.0
-    z4 = prepost.rope(e4, np.array([[50 * np.pi]]))
-    np.testing.assert_allclose(z4[0, 0, 0, [4, 12]], [0.0, 1.0], atol=1e-12)
-    np.testing.assert_allclose(z4[0, 0, 0, [0, 8]], [1.0, 0.0], atol=1e-12)
+def _rope_pins_pass(rope):
+    """The RoPE pins as one predicate of a rope function (x, pos) -> x'."""
+    try:
+        rng = np.random.default_rng(21)
+        x = rng.standard_normal((2, 5, 3, 16))
+        # position 0 is the identity
+        assert np.allclose(rope(x, np.zeros((2, 5))), x, atol=0)
+        # each (i, i + d/2) pair is rotated: the pair's norm is kept
+        y = rope(x, rng.integers(0, 1000, (2, 5)))
+        n_x = x[..., :8] ** 2 + x[..., 8:] ** 2
+        n_y = y[..., :8] ** 2 + y[..., 8:] ** 2
+        np.testing.assert_allclose(n_y, n_x, rtol=1e-12)
+        # pair 0 turns by exactly pos radians (frequency base^0 = 1), counter-clockwise
+        e = np.zeros((1, 1, 1, 16)); e[..., 0] = 1.0
+        z = rope(e, np.array([[np.pi / 2]]))
+        np.testing.assert_allclose(z[0, 0, 0, [0, 8]], [0.0, 1.0], atol=1e-15)
+        # pair 4 of d = 16 has frequency 10000^(-8/16) = 1/100: position 50*pi
+        # turns it by a quarter turn, while pair 0 turns by 50*pi (25 whole
+        # turns: unchanged).
+        e4 = np.zeros((1, 1, 1, 16)); e4[..., 4] = 1.0; e4[..., 0] = 1.0
+        z4 = rope(e4, np.array([[50 * np.pi]]))
+        np.testing.assert_allclose(z4[0, 0, 0, [4, 12]], [0.0, 1.0], atol=1e-12)
+        np.testing.assert_allclose(z4[0, 0, 0, [0, 8]], [1.0, 0.0], atol=1e-12)
+        # <rope(q, m), rope(k, n)> is a function of m - n, and not symmetric
+        q = rng.standard_normal((1, 1, 1, 32))
+        k = rng.standard_normal((1, 1, 1, 32))
+
+        def score(m, n):
+            return float(np.sum(rope(q, np.array([[m]])) * rope(k, np.array([[n]]))))
+        for m, n in [(5, 2), (105, 102), (7, 7), (1000, 997)]:
+            np.testing.assert_allclose(score(m, n), score(m - n, 0), atol=1e-9)
+        assert abs(score(5, 2) - score(2, 5)) > 1e-3
+    except AssertionError:
+        return False
+    return True
 
 
-def test_rope_scores_depend_only_on_relative_position():
-    """<rope(q, m), rope(k, n)> is a function of m - n (the property RoPE is
-    built for); a wrong sign or pairing breaks it."""
-    rng = np.random.default_rng(22)
-    q = rng.standard_normal((1, 1, 1, 32))
-    k = rng.standard_normal((1, 1, 1, 32))
-    def score(m, n):
-        return float(np.sum(prepost.rope(q, np.array([[m]])) * prepost.rope(k, np.array([[n]]))))
-    for m, n in [(5, 2), (105, 102), (7, 7), (1000, 997)]:
-        np.testing.assert_allclose(score(m, n), score(m - n, 0), atol=1e-9)
-    assert abs(score(5, 2) - score(2, 5)) > 1e-3   # but not symmetric
+def test_rope_pins_hold_for_the_oracle():
+    assert _rope_pins_pass(prepost.rope)
+
+
+def _rope_variant(mistake):
+    """prepost.rope with one planted mistake."""
+    def rope(x, pos, base=10000.0):
+        x = np.asarray(x, dtype=np.float64)
+        d = x.shape[-1]
+        half = d // 2
+        i = np.arange(half, dtype=np.float64)
+        inv = base ** ((-1.0 if mistake == "exponent" else -2.0) * i / d)
+        if mistake == "growing":
+            inv = base ** (2.0 * i / d)
+        ang = np.asarray(pos, dtype=np.float64)[:, :, None, None] * inv
+        c, s = np.cos(ang), np.sin(ang)
+        if mistake == "cos_sin":
+            c, s = s, c
+        if mistake == "interleaved":
+            x1, x2 = x[..., 0::2], x[..., 1::2]
+            out = np.empty_like(x)
+            out[..., 0::2], out[..., 1::2] = x1 * c - x2 * s, x2 * c + x1 * s
+            return out
+        x1, x2 = x[..., :half], x[..., half:]
+        if mistake == "direction":
+            return np.concatenate([x1 * c + x2 * s, x2 * c - x1 * s], axis=-1)
+        return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+    return rope
+
+
+@pytest.mark.parametrize("mistake", ["direction", "exponent", "growing", "cos_sin",
+                                     "interleaved"])
+def test_rope_pins_catch_planted_mistakes(mistake):
+    assert _rope_variant("none")(np.ones((1, 1, 1, 8)), np.array([[3]])).shape == (1, 1, 1, 8)
+    assert _rope_pins_pass(_rope_variant("none"))
+    assert not _rope_pins_pass(_rope_variant(mistake))
+
+
+def test_positions_pin_catches_planted_mistakes():
+    """An exclusive cumsum, a missing -1, or a prefix offset that counts the
+    padded prefix tokens each break the worked example."""
+    pm = np.array([[1, 1, 1, 0, 0], [1, 0, 1, 1, 1]])
+    sm = np.ones((2, 3), np.uint8)
+    want_pre = [[0, 1, 2, 2, 2], [0, 0, 1, 2, 3]]
+    want_suf = [[3, 4, 5], [4, 5, 6]]
+    exclusive = np.cumsum(pm, axis=-1) - pm
+    assert exclusive.tolist() != want_pre
+    assert np.cumsum(pm, axis=-1).tolist() != want_pre
+    padded_count = np.cumsum(sm, axis=-1) - 1 + pm.shape[1]
+    assert padded_count.tolist() != want_suf
+    assert prepost.positions(pm).tolist() == want_pre
+    assert prepost.positions(sm, pm).tolist() == want_suf
 
 
 def test_euler_step_reaches_the_ode_solution():
