@@ -744,3 +744,38 @@ def test_backward_closed_forms():
     np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-12)
     live = np.array([s >= 0 for s in seg])
     np.testing.assert_allclose(dv.sum(axis=1)[:, 0], dout[:, live].sum(axis=(1, 2)), atol=1e-12)
+
+
+def _backward_variant(mistake):
+    """oracle.backward.prefill_backward with one planted mistake."""
+    def bwd(q, k, v, ar, dout, seg=None, scale=1.0):
+        B, S, Hq, d = q.shape
+        group = Hq // k.shape[2]
+        M = oracle.prefill_mask(ar, seg=seg, B=B)
+        dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+        for b in range(B):
+            for h in range(Hq):
+                g = h // group
+                s = scale * (q[b, :, h] @ k[b, :, g].T)
+                P = oracle.softmax_probs(s, M[b])
+                dP = dout[b, :, h] @ v[b, :, g].T
+                D = 0.0 if mistake == "no_D" else (P * dP).sum(axis=1, keepdims=True)
+                dS = P * (dP - D)
+                dq[b, :, h] = (1.0 if mistake == "dq_scale" else scale) * (dS @ k[b, :, g])
+                dk[b, :, g] += scale * ((dS if mistake == "dk_untransposed" else dS.T) @ q[b, :, h])
+                dv[b, :, g] += (P if mistake == "dv_untransposed" else P.T) @ dout[b, :, h]
+        return dq, dk, dv
+    return bwd
+
+
+@pytest.mark.parametrize("mistake", ["no_D", "dq_scale", "dk_untransposed", "dv_untransposed"])
+def test_backward_pins_catch_planted_mistakes(mistake):
+    """A dropped rowsum term, a missing scale, or an untransposed dS / P each
+    disagree with the finite differences of the forward."""
+    q, k, v, ar, seg, dout = _tiny_case()
+    fd = _fd_grads(q, k, v, ar, seg, dout, 0.7)
+    good = _backward_variant("none")(q, k, v, ar, dout, seg=seg, scale=0.7)
+    for mine, ref in zip(good, fd):
+        np.testing.assert_allclose(mine, ref, atol=1e-8)
+    bad = _backward_variant(mistake)(q, k, v, ar, dout, seg=seg, scale=0.7)
+    assert max(float(np.abs(m - r).max()) for m, r in zip(bad, fd)) > 1e-3
