@@ -205,3 +205,25 @@ def test_backward_argument_errors():
     assert bwd(_desc(b, B=0), ptrs={"q": None}) == b.PI_OK
     # fp32 and grouped heads are in range of the backward (unlike the bf16 forward)
     assert ws(ctypes.byref(_desc(b, dtype=b.PI_F32, Hq=4, Hkv=2, d=64))) > 0
+
+
+def test_plain_c_client_compiles_links_and_runs():
+    """The header is plain C (C11, -Wall -Wextra -Werror) and the library links
+    without torch or C++: a small C client of the host-side paths runs clean."""
+    import shutil
+    import subprocess
+    _lib()                                              # builds the library
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    out_dir = os.path.join(ROOT, "_build")
+    os.makedirs(out_dir, exist_ok=True)
+    exe = os.path.join(out_dir, "abi_check")
+    libdir = os.path.join(ROOT, "vla_prefix_lm_b200")
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-Werror",
+                    "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi", "abi_check.c"),
+                    "-L", libdir, "-lpiattn", f"-Wl,-rpath,{libdir}", "-o", exe], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert "c abi ok" in r.stdout
