@@ -1,24 +1,27 @@
 """Benchmark of the joint (prefix-LM) attention on B200: one JSON line on stdout.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --case NAME [--launches N]     (a few launches, for ncu)
 
-A step is one joint-prefill call (pi_attn_prefill) over one batch of the pi0
-workload: B=8, Hq=8, Hkv=1, d=256, S=611 (2 x 256 image patches + 48 text
-tokens, ar_mask False; 1 state token True; 50 action tokens, the first True).
-`value` is unmasked attention pairs per second, counted per (batch, query
-head, query token, visible key), for the whole job; FLOPs are 4 * d per pair.
-Inputs rotate over enough distinct sets that each step reads HBM-cold inputs
-(more than twice the 126 MB L2); the timed loop replays CUDA graphs of the
-ABI calls, timed with CUDA events on the launching stream.
+The headline workload is the largest configuration: MM-DiT-shaped full
+bidirectional attention, B=4 per rank, Hq=8, Hkv=1, d=256, S=4096 patches +
+154 text tokens (ar_mask all False), 28 calls with fresh inputs.  One step is
+those 28 calls (pi_attn_prefill), each on its own device-resident input set,
+so every call reads its inputs from HBM.  `value` is unmasked attention pairs
+per second, counted per (batch, query head, query token, visible key), for the
+whole job; FLOPs are 4 * d per pair.  The timed loop replays one CUDA graph of
+the 28 ABI calls per step, timed with CUDA events on the launching stream.
 
-The same line also carries the suffix-pass figure of the pi0 Euler loop
-(B=32, 816-token prefix cache, 10 steps x 51 suffix tokens): microseconds per
-10-step control, and the roofline, e2e (host buffers through the C ABI),
-clocks and CPU-oracle baseline objects.
+The same line carries, as sub-objects, the other configurations (the tiny fp32
+prefill, the pi0 prefill B=8 S=611, the pi0.5 three-segment prefill B=16
+S=938, and the pi0 Euler suffix control B=32 with an 816-token cache), the
+single-token decode, RoPE / Euler, the backward, and the roofline, e2e (host
+buffers through the C ABI), clocks and CPU-oracle baseline objects.
 
-N > 1 (torchrun, one process per GPU): every rank runs its own batch shard of
-the same per-rank size (weak scaling, no data-path collective); the timed
-region is bracketed by barriers and the max over ranks is reported.
+N > 1 (one process per GPU): every rank runs its own batch of the same
+per-rank size (weak scaling, no data-path collective); the timed region is
+bracketed by barriers and the max over ranks is reported.  `--gpus N` started
+without a launcher re-runs this script under torch.distributed.run.
 
 --impl reference times the CPU oracle (numpy float64) on a bounded sample of
 the same workload; under torchrun only rank 0 runs it.
@@ -44,10 +47,10 @@ if ROOT not in sys.path:
 METRIC = "unmasked attn pairs/s + TFLOP/s vs bf16 TC peak; suffix-pass µs per 10-step ctrl"
 L2_BYTES = 126 * 2**20
 
-# DRAM traffic of the prefill kernel per launch on the pi0 workload, from one
-# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the
-# kernel sources whose digest is recorded beside it.
-TRAFFIC = {"bytes": 25184896, "src_sha": "f6025ed41baa6bac"}
+# DRAM traffic of the prefill kernel per launch on the headline workload, from
+# one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only for
+# the kernel sources whose digest is recorded beside it.
+TRAFFIC = {"bytes": None, "src_sha": None, "workload": "mmdit"}
 KERNEL_SOURCES = ("vla_prefix_lm_b200/csrc/tc_pair.cu", "vla_prefix_lm_b200/csrc/common.cuh",
                   "vla_prefix_lm_b200/csrc/mask.cuh")
 
@@ -158,7 +161,54 @@ def gpu_id(dev) -> str:
 # ------------------------------------------------------------------ our arm
 
 
+def _mmdit_sets(w, dev, n, seed0):
+    """``n`` fresh MM-DiT input sets (q, k, v, ar) drawn on the device."""
+    import torch
+
+    from vla_prefix_lm_b200 import workloads as W
+
+    ar = torch.tensor(w.ar, dtype=torch.uint8, device=dev)
+    sets = []
+    for i in range(n):
+        s = seed0 + 4 * i
+        q = W.device_draw((w.B, w.Sq, w.Hq, w.d), s, w.d, w.dtype, dev)
+        k = W.device_draw((w.B, w.Sq, w.Hkv, w.d), s + 1, w.d, w.dtype, dev)
+        v = W.device_draw((w.B, w.Sq, w.Hkv, w.d), s + 2, w.d, w.dtype, dev)
+        sets.append((q, k, v, ar))
+    return sets
+
+
+def timed_steps(step, steps, stream, rank):
+    """Runs ``steps`` calls of ``step()`` between a barrier and a synchronize
+    on both sides; returns (device ms on this rank from CUDA events on
+    ``stream``, max over ranks, wall-clock bounds, clock record)."""
+    import torch
+
+    from vla_prefix_lm_b200 import dist
+
+    sampler = ClockSampler(gpu_id(stream.device)) if rank == 0 else None
+    time.sleep(0.3 if sampler else 0)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    dist.barrier()
+    ms = e0.elapsed_time(e1)
+    clocks = sampler.stop(t0, t1) if sampler else None
+    return ms, dist.max_over_ranks(ms), clocks
+
+
 def run_ours(args, rank, ws, local):
+    """The bench line: the MM-DiT workload (the largest config) as the headline,
+    the other configs, the suffix control, decode, RoPE/Euler and backward as
+    sub-objects."""
     import torch
 
     from vla_prefix_lm_b200 import binding, dist
@@ -170,119 +220,61 @@ def run_ours(args, rank, ws, local):
     stream = torch.cuda.Stream(dev)
     P = peaks()
 
-    w = W.workload(2)
-    B = w.B                                   # per-rank batch (weak scaling)
-    pairs_bh = visible_pairs_per_bh(w.ar)
-    pairs_step = pairs_bh * B * w.Hq
-    flops_step = 4.0 * w.d * pairs_step
-    bytes_step = (B * w.Sq * w.Hq * w.d * 2) * 2 + (B * w.Sq * w.d * 2) * 2 + w.Sq
+    # --- headline: MM-DiT, B=4 per rank, S=4250, all False; one step = the
+    # workload's 28 calls, each on its own fresh input set
+    w = W.workload(5)
+    calls = w.calls
+    pairs_call = visible_pairs_per_bh(w.ar) * w.B * w.Hq
+    flops_call = 4.0 * w.d * pairs_call
+    bytes_call = 2 * (2 * w.B * w.Sq * w.Hq * w.d + 2 * w.B * w.Sq * w.Hkv * w.d) + w.Sq
+    sets = _mmdit_sets(w, dev, calls, 5_000_000 + 1000 * rank)
+    outs = [torch.empty_like(s_[0]) for s_ in sets]
+    set_bytes = sum(t.nbytes for t in sets[0][:3]) + outs[0].nbytes
 
-    # rotating device-resident input sets: > 2 x L2 in total
-    set_bytes = B * w.Sq * (w.Hq + 2) * w.d * 2
-    n_sets = max(3, int(np.ceil(2 * L2_BYTES / set_bytes)))
-    sets = []
-    for i in range(n_sets):
-        x = W.prefill_inputs(w, W.seed_for(2, 100 + rank * 1000 + i), B=B)
-        sets.append((x.q.to(dev), x.k.to(dev), x.v.to(dev), x.ar.to(dev)))
-    outs = [torch.empty_like(s[0]) for s in sets]
-
-    def step(i):
-        q, k, v, ar = sets[i % n_sets]
-        binding.pi_attn_prefill(q, k, v, ar, out=outs[i % n_sets], stream=stream)
+    def workload_calls():
+        for i, (q, k, v, ar) in enumerate(sets):
+            binding.pi_attn_prefill(q, k, v, ar, out=outs[i], stream=stream)
 
     with torch.cuda.stream(stream):
-        for i in range(max(args.warmup, 1)):
-            step(i)
+        for _ in range(max(args.warmup, 1)):
+            workload_calls()
     torch.cuda.synchronize()
     assert binding.pi_attn_read_status(stream) == binding.PI_OK
-
-    # one graph per chunk of steps (a whole number of input rotations)
-    chunk = n_sets * max(1, min(64 // n_sets, args.steps // n_sets or 1))
-    graphs = {}
-
-    def graph_for(n):
-        if n not in graphs:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for i in range(n):
-                    step(i)
-            graphs[n] = g
-        return graphs[n]
-
-    plan = [chunk] * (args.steps // chunk) + ([args.steps % chunk] if args.steps % chunk else [])
-    # CUDAGraph.replay() launches on torch's current stream: make it `stream`,
-    # the stream the timing events are recorded on.
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        workload_calls()
+    # CUDAGraph.replay() launches on torch's current stream: timed_steps makes
+    # it `stream`, the stream the events are recorded on.
     with torch.cuda.stream(stream):
-        for n in set(plan):
-            graph_for(n).replay()
+        g.replay()
     torch.cuda.synchronize()
-
-    sampler = ClockSampler(gpu_id(dev)) if rank == 0 else None
-    time.sleep(0.3 if sampler else 0)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dist.barrier()
-    torch.cuda.synchronize()
-    t_wall0 = time.time()
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for n in plan:
-            graph_for(n).replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    t_wall1 = time.time()
-    dist.barrier()
-    ms = e0.elapsed_time(e1)
-    clocks = sampler.stop(t_wall0, t_wall1) if sampler else None
-    ms_max = dist.max_over_ranks(ms)
+    ms, ms_max, clocks = timed_steps(g.replay, args.steps, stream, rank)
     status = binding.pi_attn_read_status(stream)
     if status != binding.PI_OK:
         raise RuntimeError(f"device status after timing: {binding.status_string(status)}")
-
-    value = ws * pairs_step * args.steps / (ms_max / 1e3)
+    del g
     ms_step = ms_max / args.steps
-    achieved_tflops = flops_step / (ms / args.steps / 1e3) / 1e12
+    value = ws * pairs_call * calls * args.steps / (ms_max / 1e3)
+    us_launch = ms / (args.steps * calls) * 1e3
+    achieved_tflops = flops_call / (us_launch / 1e6) / 1e12
 
-    # e2e: host (pinned) buffers through the public API, copies inside the region
-    n_e2e = max(3, min(args.steps, 200))
-    hq = [s[0].cpu().pin_memory() for s in sets[:2]]
-    hk = [s[1].cpu().pin_memory() for s in sets[:2]]
-    hv = [s[2].cpu().pin_memory() for s in sets[:2]]
-    har = [s[3].cpu().pin_memory() for s in sets[:2]]
-    dq, dk, dv, dar = (torch.empty_like(sets[0][j]) for j in range(4))
-    hout = torch.empty(outs[0].shape, dtype=outs[0].dtype, pin_memory=True)
-    h2d = hq[0].nbytes + hk[0].nbytes + hv[0].nbytes + har[0].nbytes
-    d2h = hout.nbytes
+    e2e = e2e_mmdit(args, w, dev, stream, rank, ws, sets[:2])
+    del sets, outs
+    torch.cuda.empty_cache()
 
-    def e2e_step(i):
-        j = i % 2
-        with torch.cuda.stream(stream):
-            dq.copy_(hq[j], non_blocking=True)
-            dk.copy_(hk[j], non_blocking=True)
-            dv.copy_(hv[j], non_blocking=True)
-            dar.copy_(har[j], non_blocking=True)
-            o = binding.pi_attn_prefill(dq, dk, dv, dar, out=outs[0], stream=stream)
-            hout.copy_(o, non_blocking=True)
-
-    for i in range(3):
-        e2e_step(i)
-    torch.cuda.synchronize()
-    dist.barrier()
-    e0.record(stream)
-    for i in range(n_e2e):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    dist.barrier()
-    e2e_ms = dist.max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = ws * pairs_step * n_e2e / (e2e_ms / 1e3)
-
-    # suffix pass: 10 Euler steps against the prefix cache (warm L2, back to back)
-    suffix = suffix_control(args, dev, stream, rank)
+    configs = {
+        "tiny_f32": prefill_config(1, dev, stream, rank, n_sets=1, reps=200),
+        "pi0_prefill": prefill_config(2, dev, stream, rank, n_sets=6, reps=50),
+        "pi05_prefill": prefill_config(4, dev, stream, rank, n_sets=3, reps=20),
+        "pi0_euler_suffix": suffix_control(args, dev, stream, rank),
+    }
     decode = decode_steps(args, dev, stream, rank)
     prepost = prepost_steps(args, dev, stream, rank)
     bwd = backward_steps(args, dev, stream, rank)
 
-    traffic = TRAFFIC["bytes"] if TRAFFIC["src_sha"] == kernel_digest() else None
+    traffic = None
+    if TRAFFIC.get("src_sha") == kernel_digest() and TRAFFIC.get("workload") == "mmdit":
+        traffic = TRAFFIC["bytes"]
     line = {
         "metric": METRIC,
         "value": value,
@@ -295,21 +287,26 @@ def run_ours(args, rank, ws, local):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1)*d^-0.25 q/k/v rounded to bf16)",
+        "data": "synthetic (seeded N(0,1)*d^-0.25 q/k/v, bf16)",
         "config": {
-            "workload": "pi0_joint_prefill: B=8 per rank, Hq=8, Hkv=1, d=256, S=611 "
-                        "(560 prefix False | state True | 50 actions True,False*49)",
-            "per_rank_batch": B,
-            "global_batch": B * ws,
+            "workload": "mmdit_full_bidirectional: B=4 per rank, Hq=8, Hkv=1, d=256, "
+                        "S=4250 (4096 patches + 154 text, ar_mask all False); one step = "
+                        "the workload's 28 calls, each on a fresh input set",
+            "per_rank_batch": w.B,
+            "global_batch": w.B * ws,
             "seq_len": w.Sq,
+            "calls_per_step": calls,
             "parallelism": f"batch replicas x{ws} (no data-path collective)",
-            "l2": f"inputs rotate over {n_sets} device-resident sets "
-                  f"({n_sets * set_bytes / 2**20:.0f} MiB > 2 x L2)",
-            "timing": "CUDA events on the launching stream around CUDA-graph replays "
-                      f"of {chunk} calls; max over ranks",
+            "l2": f"inputs larger than L2: each step reads {calls} distinct input sets "
+                  f"({calls * set_bytes / 2**30:.1f} GiB with outputs), so every call's "
+                  "inputs come from HBM",
+            "timing": "CUDA events on the launching stream around one CUDA-graph replay "
+                      f"(the {calls} calls) per step; barrier + synchronize on both sides; "
+                      "max over ranks",
         },
-        "tflops": ws * flops_step * args.steps / (ms_max / 1e3) / 1e12,
-        "gb_per_s_algorithmic": bytes_step / (ms_step / 1e3) / 1e9,
+        "us_per_call": ms_step / calls * 1e3,
+        "tflops": ws * flops_call * calls * args.steps / (ms_max / 1e3) / 1e12,
+        "gb_per_s_algorithmic": bytes_call / (us_launch / 1e6) / 1e9,
         "roofline": {
             "bound": "tensor",
             "kernel": "tc_pair_kernel<prefill>",
@@ -321,20 +318,168 @@ def run_ours(args, rank, ws, local):
             "frac_of_sustained": (achieved_tflops / P["bf16_tflops_sustained"]
                                   if P["bf16_tflops_sustained"] else None),
             "traffic": traffic,
-            "algorithmic_flop_per_launch": flops_step,
+            "algorithmic_flop_per_launch": flops_call,
+            "launch_us": us_launch,
         },
-        "e2e": {"value": e2e_value, "unit": "pairs/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": n_e2e,
-                "what": "pinned host q/k/v/ar -> device, pi_attn_prefill, out -> pinned host"},
-        "gpu_launches": args.steps,
+        "e2e": e2e,
+        "gpu_launches": calls * args.steps,
         "clocks": clocks,
-        "suffix_ctrl": suffix,
+        "configs": configs,
         "decode": decode,
         "prepost": prepost,
         "backward": bwd,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, seconds=args.cpu_seconds)
+    return line
+
+
+def e2e_mmdit(args, w, dev, stream, rank, ws, dev_sets):
+    """The headline metric end to end through the public API: every call's
+    q/k/v/ar go from pinned host memory to the device, pi_attn_prefill runs,
+    and out comes back to pinned host memory, all inside the timed region.
+    Three streams (host-to-device, compute, device-to-host) and two buffer
+    slots let the copies of neighbouring calls overlap with each other and
+    with the kernel.  Also reports the copy-only floor: the same transfers with
+    no kernel, both directions overlapped."""
+    import torch
+
+    from vla_prefix_lm_b200 import binding, dist
+
+    calls = w.calls
+    n_steps = max(1, min(args.steps, 2))
+    host = []
+    for q, k, v, ar in dev_sets:
+        host.append(tuple(t.cpu().pin_memory() for t in (q, k, v, ar)))
+    hout = [torch.empty(dev_sets[0][0].shape, dtype=torch.bfloat16, pin_memory=True)
+            for _ in range(2)]
+    din = [tuple(torch.empty_like(t) for t in dev_sets[0]) for _ in range(2)]
+    dout = [torch.empty_like(dev_sets[0][0]) for _ in range(2)]
+    h2d_bytes = sum(t.nbytes for t in host[0])
+    d2h_bytes = hout[0].nbytes
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def run(n_calls, compute=True):
+        for i in range(n_calls):
+            j = i % 2
+            if i >= 2:
+                s_in.wait_event(ev_done[j])            # input slot j free again
+            with torch.cuda.stream(s_in):
+                for dst, src in zip(din[j], host[i % len(host)]):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[j].record(s_in)
+            stream.wait_event(ev_in[j])
+            if i >= 2:
+                stream.wait_event(ev_out[j])           # output slot j copied out
+            if compute:
+                q, k, v, ar = din[j]
+                binding.pi_attn_prefill(q, k, v, ar, out=dout[j], stream=stream)
+            ev_done[j].record(stream)
+            s_out.wait_event(ev_done[j])
+            with torch.cuda.stream(s_out):
+                hout[j].copy_(dout[j], non_blocking=True)
+                ev_out[j].record(s_out)
+        stream.wait_stream(s_out)
+        stream.wait_stream(s_in)
+
+    run(4)
+    torch.cuda.synchronize()
+    res = {}
+    for key, compute in (("value", True), ("copy_only", False)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        s_in.wait_stream(stream)
+        run(n_steps * calls, compute)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        res[key] = dist.max_over_ranks(e0.elapsed_time(e1))
+    assert binding.pi_attn_read_status(stream) == binding.PI_OK
+    pairs = ws * visible_pairs_per_bh(w.ar) * w.B * w.Hq * calls * n_steps
+    return {
+        "value": pairs / (res["value"] / 1e3),
+        "unit": "pairs/s",
+        "h2d_bytes_per_step": h2d_bytes * calls,
+        "d2h_bytes_per_step": d2h_bytes * calls,
+        "steps": n_steps,
+        "ms_per_step": res["value"] / n_steps,
+        "copy_floor_ms_per_step": res["copy_only"] / n_steps,
+        "copy_floor_pairs_per_s": pairs / (res["copy_only"] / 1e3),
+        "what": "per call: pinned host q/k/v/ar -> device, pi_attn_prefill, out -> pinned "
+                "host; copies and kernel overlapped over three streams and two buffer "
+                "slots; copy_floor = the same copies with no kernel",
+    }
+
+
+def prefill_config(cfg, dev, stream, rank, n_sets, reps):
+    """Device time per call of one prefill workload: a CUDA graph of calls over
+    ``n_sets`` device-resident input sets (together larger than L2 where the
+    workload is large enough), replayed ``reps`` times."""
+    import torch
+
+    from vla_prefix_lm_b200 import binding, dist
+    from vla_prefix_lm_b200 import workloads as W
+
+    w = W.workload(cfg)
+    P_ = peaks()
+    ar = torch.tensor(w.ar, dtype=torch.uint8, device=dev)
+    seg = None if w.seg is None else torch.tensor(w.seg, dtype=torch.int32, device=dev)
+    ins = []
+    for i in range(n_sets):
+        s = 6_000_000 + 10_000 * cfg + 1000 * rank + 4 * i
+        ins.append(tuple(W.device_draw((w.B, w.Sq, h, w.d), s + j, w.d, w.dtype, dev)
+                         for j, h in enumerate((w.Hq, w.Hkv, w.Hkv))))
+    outs = [torch.empty_like(t[0]) for t in ins]
+
+    def call(i):
+        q, k, v = ins[i % n_sets]
+        binding.pi_attn_prefill(q, k, v, ar, segment_ids=seg, out=outs[i % n_sets],
+                                softmax_scale=w.scale, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(3, n_sets)):
+            call(i)
+    torch.cuda.synchronize()
+    n = n_sets * max(1, 8 // n_sets)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            call(i)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    with torch.cuda.stream(stream):
+        g.replay()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us = dist.max_over_ranks(e0.elapsed_time(e1) * 1e3 / (reps * n))
+    del g
+    assert binding.pi_attn_read_status(stream) == binding.PI_OK
+    elt = 2 if w.dtype == "bf16" else 4
+    pairs = visible_pairs_per_bh(w.ar, w.seg) * w.B * w.Hq
+    flops = 4 * w.d * pairs
+    nbytes = (2 * w.B * w.Sq * w.Hq * w.d + 2 * w.B * w.Sq * w.Hkv * w.d) * elt
+    set_bytes = (2 * w.B * w.Sq * w.Hq * w.d + 2 * w.B * w.Sq * w.Hkv * w.d) * elt
+    line = {
+        "workload": f"{w.name}: B={w.B}, Hq={w.Hq}, Hkv={w.Hkv}, d={w.d}, {w.dtype}; {w.note}",
+        "us_per_call": us, "pairs_per_call": pairs, "pairs_per_s": pairs / (us / 1e6),
+        "tflops": flops / (us / 1e6) / 1e12, "gb_per_s_algorithmic": nbytes / (us / 1e6) / 1e9,
+        "timing": f"CUDA graph of {n} calls over {n_sets} input sets "
+                  f"({n_sets * set_bytes / 2**20:.0f} MiB with outputs), replayed {reps}x",
+    }
+    if w.dtype == "bf16":
+        line["bound"] = "tensor"
+        line["frac_of_bf16_peak"] = line["tflops"] / P_["bf16_tflops"]
+        line["frac_of_bf16_sustained"] = line["tflops"] / P_["bf16_tflops_sustained"]
+    else:
+        line["bound"] = "launch latency (fp32 SIMT path; parity case, throughput not a target)"
     return line
 
 
@@ -646,158 +791,67 @@ def suffix_control(args, dev, stream, rank):
     }
 
 
-# ------------------------------------------------------- per-config table
-
-
-def oracle_seconds_per_call(w, x, max_rows, seconds=5.0):
-    """The oracle's wall time for one whole call of workload ``w``, estimated
-    from a bounded sample: ``max_rows`` query rows of batch element 0 (all
-    heads), timed for about ``seconds``, scaled by B * S / rows."""
-    import oracle
-
-    ar = np.array(w.ar)
-    seg = None if w.seg is None else np.array(w.seg)
-    S = w.Sq
-    n_rows = min(S, max_rows)
-    rows = [(0, int(i)) for i in np.linspace(0, S - 1, n_rows).round().astype(int)]
-    t0 = time.perf_counter()
-    n = 0
-    while n < 1 or time.perf_counter() - t0 < seconds:
-        oracle.prefill(x.q64[:1], x.k64[:1], x.v64[:1], ar, seg, scale=w.scale, rows=rows)
-        n += 1
-    dt = (time.perf_counter() - t0) / n
-    return dt * w.B * S / n_rows, (f"{n_rows} of {S} query rows (all heads) of 1 of {w.B} "
-                                   f"batch elements, {n} repeats, scaled to the whole call")
-
-
-def prefill_config_line(cfg, dev, stream, sets, reps, oracle_rows):
-    """Device time per call of one prefill workload, rotating over ``sets``
-    device-resident input sets, plus the oracle's estimated time per call."""
-    import torch
-
-    from vla_prefix_lm_b200 import binding
-    from vla_prefix_lm_b200 import workloads as W
-
-    w = W.workload(cfg)
-    P_ = peaks()
-    host = [W.prefill_inputs(w, W.seed_for(cfg, c), B=w.B) for c in range(sets)]
-    ins = []
-    for x in host:
-        seg = None if x.seg is None else x.seg.to(dev)
-        ins.append((x.q.to(dev), x.k.to(dev), x.v.to(dev), x.ar.to(dev), seg))
-    outs = [torch.empty_like(t[0]) for t in ins]
-
-    def call(i):
-        q, k, v, ar, seg = ins[i % sets]
-        binding.pi_attn_prefill(q, k, v, ar, segment_ids=seg, out=outs[i % sets],
-                                softmax_scale=w.scale, stream=stream)
-
-    with torch.cuda.stream(stream):
-        for i in range(max(3, sets)):
-            call(i)
-    torch.cuda.synchronize()
-    n = sets * max(1, 8 // sets)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for i in range(n):
-            call(i)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        g.replay()
-        e0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    us = e0.elapsed_time(e1) * 1e3 / (reps * n)
-    del g
-    assert binding.pi_attn_read_status(stream) == binding.PI_OK
-    elt = 2 if w.dtype == "bf16" else 4
-    pairs = visible_pairs_per_bh(w.ar, w.seg) * w.B * w.Hq
-    flops = 4 * w.d * pairs
-    nbytes = (2 * w.B * w.Sq * w.Hq * w.d + 2 * w.B * w.Sq * w.Hkv * w.d) * elt
-    o_s, sample = oracle_seconds_per_call(w, host[0], oracle_rows)
-    line = {
-        "config": cfg, "workload": f"{w.name}: {w.note}",
-        "shape": {"B": w.B, "S": w.Sq, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "dtype": w.dtype},
-        "us_per_call": us, "pairs_per_call": pairs, "pairs_per_s": pairs / (us / 1e6),
-        "tflops": flops / (us / 1e6) / 1e12, "gb_per_s_algorithmic": nbytes / (us / 1e6) / 1e9,
-        "timing": f"CUDA graph of {n} calls over {sets} input sets, replayed {reps}x",
-        "oracle_s_per_call": o_s, "oracle_sample": sample,
-        "oracle_cores": len(os.sched_getaffinity(0)),
-    }
-    if w.dtype == "bf16":
-        line["frac_of_bf16_peak"] = line["tflops"] / P_["bf16_tflops"]
-        line["frac_of_bf16_sustained"] = line["tflops"] / P_["bf16_tflops_sustained"]
-    if w.calls > 1:
-        line["us_per_workload"] = us * w.calls
-        line["calls"] = w.calls
-    return line
-
-
-def run_configs(args):
-    """One JSON line per workload config: device time, rates, roofline
-    fractions and the oracle's estimated time per call (one GPU, no ranks)."""
-    import torch
-
-    from vla_prefix_lm_b200 import binding
-
-    binding.lib()
-    dev = torch.device("cuda:0")
-    torch.cuda.set_device(dev)
-    stream = torch.cuda.Stream()
-    plan = {1: (1, 200, 49), 2: (6, 50, 611), 4: (2, 20, 256), 5: (2, 5, 64)}
-    for cfg in (1, 2, 4, 5):
-        sets, reps, rows = plan[cfg]
-        print(json.dumps({"impl": "ours", "mode": "configs",
-                          **prefill_config_line(cfg, dev, stream, sets, reps, rows)}),
-              flush=True)
-    suffix = suffix_control(args, dev, stream, 0)
-    print(json.dumps({"impl": "ours", "mode": "configs", "config": 3, **suffix}), flush=True)
-
-
 # ------------------------------------------------------------ CPU baselines
 
 
-def cpu_baseline(w, seconds=10.0):
-    """The oracle (numpy float64, as it stands) on a bounded sample of the workload."""
+def _oracle_rows_sample(w, n_tok, i0):
+    """The oracle on ``n_tok`` query tokens (all heads) of batch element 0 of
+    the MM-DiT workload, starting at token ``i0``: its own mask builder and
+    attention, as they stand.  Returns the visible pairs it computed."""
     import oracle
     from vla_prefix_lm_b200 import workloads as W
 
-    x = W.prefill_inputs(w, W.seed_for(2), B=1)
+    x = _ORACLE_INPUTS.get(w.name)
+    if x is None:
+        x = _ORACLE_INPUTS[w.name] = W.prefill_inputs(w, W.seed_for(5, 0), B=1)
     ar = np.array(w.ar)
-    pairs = visible_pairs_per_bh(w.ar) * w.Hq
+    rows = np.arange(i0, min(i0 + n_tok, w.Sq))
+    M = oracle.prefill_mask(ar, rows=rows)
+    oracle.attention(x.q64[:, rows], x.k64, x.v64, M, scale=w.scale)
+    return int(M.sum()) * w.Hq
+
+
+_ORACLE_INPUTS = {}
+
+
+def cpu_baseline(w, seconds=10.0, n_tok=512):
+    """The oracle (numpy float64, as it stands) on a bounded sample of the
+    headline workload: blocks of ``n_tok`` query tokens of one batch element."""
+    _oracle_rows_sample(w, 8, 0)                       # inputs drawn outside the clock
     t0 = time.perf_counter()
-    n = 0
-    while n < 3 or time.perf_counter() - t0 < seconds:
-        oracle.prefill(x.q64, x.k64, x.v64, ar)
+    n, pairs = 0, 0
+    while n < 2 or time.perf_counter() - t0 < seconds:
+        pairs += _oracle_rows_sample(w, n_tok, (n * n_tok) % w.Sq)
         n += 1
     dt = time.perf_counter() - t0
-    return {"value": pairs * n / dt, "unit": "pairs/s", "cores": len(os.sched_getaffinity(0)),
+    return {"value": pairs / dt, "unit": "pairs/s", "cores": len(os.sched_getaffinity(0)),
             "kind": "oracle",
-            "sample": f"{n} oracle.prefill calls on 1 of the 8 batch elements (all 8 heads, "
-                      f"S=611), {dt:.1f} s wall; numpy/BLAS threads = cores"}
+            "sample": f"{n} blocks of {n_tok} query tokens x 8 heads x 4250 keys of batch "
+                      f"element 0 of the MM-DiT workload (oracle.prefill_mask + "
+                      f"oracle.attention), {dt:.1f} s wall; numpy/BLAS threads = cores"}
 
 
 def run_reference(args, rank, ws):
-    import oracle
+    """The oracle arm: each step is a bounded sample of the headline workload
+    (512 query tokens x 8 heads of one batch element against all 4250 keys)."""
     from vla_prefix_lm_b200 import workloads as W
 
     if rank != 0:
         return None
-    w = W.workload(2)
-    x = W.prefill_inputs(w, W.seed_for(2), B=1)
-    ar = np.array(w.ar)
-    pairs = visible_pairs_per_bh(w.ar) * w.Hq
-    for _ in range(args.warmup):
-        oracle.prefill(x.q64, x.k64, x.v64, ar)
+    w = W.workload(5)
+    n_tok = 512
+    _oracle_rows_sample(w, 8, 0)
+    for i in range(args.warmup):
+        _oracle_rows_sample(w, n_tok, (i * n_tok) % w.Sq)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle.prefill(x.q64, x.k64, x.v64, ar)
+    pairs = 0
+    for i in range(args.steps):
+        pairs += _oracle_rows_sample(w, n_tok, (i * n_tok) % w.Sq)
     dt = time.perf_counter() - t0
-    value = pairs * args.steps / dt
+    value = pairs / dt
     cores = len(os.sched_getaffinity(0))
-    sample = "each step: oracle.prefill on 1 of the 8 batch elements of pi0_joint_prefill"
+    sample = (f"each step: oracle.prefill_mask + oracle.attention on {n_tok} query tokens "
+              "(all 8 heads, all 4250 keys) of batch element 0 of the MM-DiT workload")
     return {
         "impl": "reference",
         "metric": METRIC,
@@ -806,14 +860,14 @@ def run_reference(args, rank, ws):
         "n_gpus": ws,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": dt / args.steps * 1e3,
+        "ms_per_step": dt / max(args.steps, 1) * 1e3,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded N(0,1)*d^-0.25 q/k/v rounded to bf16, upcast)",
-        "config": {"workload": "pi0_joint_prefill: Hq=8, Hkv=1, d=256, S=611; "
-                               "sample of 1 batch element per step",
+        "config": {"workload": "mmdit_full_bidirectional: Hq=8, Hkv=1, d=256, S=4250, "
+                               f"ar_mask all False; sample of {n_tok} query tokens per step",
                    "seq_len": w.Sq, "parallelism": "rank 0 only (CPU)"},
         "cpu_baseline": {"value": value, "unit": "pairs/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
@@ -822,37 +876,139 @@ def run_reference(args, rank, ws):
     }
 
 
+# ------------------------------------------------------------- profiling
+
+
+CASES = ("mmdit_prefill", "pi0_prefill", "pi05_prefill", "pi0_suffix_step", "decode_step")
+
+
+def run_case(args):
+    """A few launches of one workload on one input set, for ncu captures:
+    little device memory (one set, no rotation) and no timing."""
+    import torch
+
+    from vla_prefix_lm_b200 import binding
+    from vla_prefix_lm_b200 import workloads as W
+
+    binding.lib()
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)
+    name = args.case
+    if name.endswith("_prefill"):
+        w = W.workload({"mmdit_prefill": 5, "pi0_prefill": 2, "pi05_prefill": 4}[name])
+        q, k, v = (W.device_draw((w.B, w.Sq, h, w.d), 7_000_000 + j, w.d, w.dtype, dev)
+                   for j, h in enumerate((w.Hq, w.Hkv, w.Hkv)))
+        ar = torch.tensor(w.ar, dtype=torch.uint8, device=dev)
+        seg = None if w.seg is None else torch.tensor(w.seg, dtype=torch.int32, device=dev)
+        out = torch.empty_like(q)
+
+        def call():
+            binding.pi_attn_prefill(q, k, v, ar, segment_ids=seg, out=out, stream=stream)
+    else:
+        if name == "pi0_suffix_step":
+            w = W.workload(3)
+            B, P, Sq, ar_np = w.B, w.P, w.Sq, np.array(w.ar, np.uint8)
+        else:
+            B, P, Sq, ar_np = 32, 880, 1, np.ones(1, np.uint8)
+        d = 256
+        kc, vc = (W.device_draw((B, P, 1, d), 7_100_000 + j, d, "bf16", dev) for j in (0, 1))
+        q = W.device_draw((B, Sq, 8, d), 7_100_002, d, "bf16", dev)
+        k, v = (W.device_draw((B, Sq, 1, d), 7_100_003 + j, d, "bf16", dev) for j in (0, 1))
+        ar = torch.from_numpy(ar_np).to(dev)
+        out = torch.empty_like(q)
+        need = binding.pi_attn_suffix_workspace_bytes(q, k, kc, ar)
+        wsb = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+
+        def call():
+            binding.pi_attn_suffix(q, k, v, kc, vc, ar, out=out, workspace=wsb, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.launches):
+            call()
+    torch.cuda.synchronize()
+    st = binding.pi_attn_read_status(stream)
+    print(json.dumps({"case": name, "launches": args.launches,
+                      "status": binding.status_string(st)}), flush=True)
+    if st != binding.PI_OK:
+        raise SystemExit(1)
+
+
+# ------------------------------------------------------------ rank plumbing
+
+
+def run_plumbing_check(args, rank, ws):
+    """The bench's multi-rank plumbing on CPU (gloo): the same barrier / max
+    over ranks / whole-job value arithmetic as the GPU arm, around a fixed
+    host workload; rank 0 prints the line.  Used by the host tests."""
+    from vla_prefix_lm_b200 import dist
+
+    units_per_step = 1000
+    a = np.random.default_rng(rank).standard_normal((256, 256))
+    for _ in range(args.warmup):
+        a = np.tanh(a @ a.T / 256)
+    dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        a = np.tanh(a @ a.T / 256)
+    ms = (time.perf_counter() - t0) * 1e3 + 5.0 * rank   # ranks differ: the max must win
+    dist.barrier()
+    ms_max = dist.max_over_ranks(ms)
+    return {"metric": "plumbing check", "value": ws * units_per_step * args.steps / (ms_max / 1e3),
+            "unit": "units/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_max / args.steps, "rank_ms": ms, "max_rank_ms": ms_max}
+
+
+def relaunch_under_torchrun(n):
+    """``--gpus N`` without a launcher: start N ranks of this script with
+    torch.distributed.run (one process per GPU, rendezvous on 127.0.0.1)."""
+    import socket
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--configs", action="store_true",
-                    help="instead of the bench line: one line per workload config (1 GPU)")
+    ap.add_argument("--case", choices=CASES,
+                    help="run --launches calls of one workload on one input set (for ncu)")
+    ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--plumbing-check", action="store_true",
+                    help="CPU-only multi-rank check of the timing plumbing (gloo)")
     args = ap.parse_args()
-    if args.warmup < 3 and args.impl == "ours":
+    if args.warmup < 3 and args.impl == "ours" and not args.case:
         ap.error("--warmup must be >= 3")
 
     from vla_prefix_lm_b200 import dist
     rank, ws, local = dist.world()
-    if args.configs:
-        dist.init()
-        try:
-            run_configs(args)
-        finally:
-            dist.shutdown()
+    if args.case:
+        run_case(args)
         return
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if ws == 1 and args.gpus > 1 and "LOCAL_RANK" not in os.environ:
+        raise SystemExit(relaunch_under_torchrun(args.gpus))
+    if ws != args.gpus:
+        ap.error(f"--gpus {args.gpus} but the launcher started WORLD_SIZE={ws} ranks")
     if args.impl == "reference":
         line = run_reference(args, rank, ws)
         if line is not None:
             print(json.dumps(line), flush=True)
         return
-    dist.init()
+    dist.init(backend="gloo" if args.plumbing_check else None)
     try:
-        line = run_ours(args, rank, ws, local)
+        line = (run_plumbing_check(args, rank, ws) if args.plumbing_check
+                else run_ours(args, rank, ws, local))
     finally:
         dist.shutdown()
     if rank == 0:

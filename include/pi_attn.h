@@ -42,6 +42,11 @@
  * work.  Calls on different streams may run concurrently; the global state is
  * the device status word read by pi_attn_read_status, the wait bound set by
  * pi_attn_set_wait_limit, and the fixed scratch of pi_attn_suffix_noalloc.
+ * The device addresses of the status word and of that scratch, and each
+ * device's SM count, are looked up on the first call that needs them on that
+ * device and kept for the life of the process: a device reset
+ * (cudaDeviceReset) after the first call invalidates them, so do not reset a
+ * device this library has run on.
  *
  * Errors: every entry point returns PI_OK or a PI_ERR_* code.  Argument
  * errors are detected on the host before anything is enqueued (nothing is

@@ -33,9 +33,9 @@ Parity status per function (what pins it; tests live in tests/test_oracle.py):
   positions example with padding and a padded prefix, RoPE's closed forms
   (identity at 0, pair norms kept, a stated turn of pairs 0 and 4), the
   relative-position property, and the Euler loop against the exact solution.
-* ``counts.control_step_pairs`` -- parity unpinned: the pages quote about
-  1.2e6 pairs per pi0.5 control step without a derivation; the count is only
-  checked to be of that order.
+* ``counts.full_pairs`` / ``visible_pairs`` -- pinned: the pages' worked
+  counts (480^2 = 230,400 fused scores, 32 x 448 cross scores, 28 x 4250^2
+  MM-DiT pairs) and the number of True entries of the explicit masks.
 """
 
 from .attention import (  # noqa: F401

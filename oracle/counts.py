@@ -23,13 +23,3 @@ def full_pairs(Sq, Sk=None):
 def visible_pairs(M):
     return int(np.count_nonzero(np.asarray(M)))
 
-
-def control_step_pairs(prefix_tokens, suffix_queries, steps, suffix_keys=None):
-    """Pairs in one control step: the prefix once, then ``steps`` suffix passes.
-
-    parity unpinned: "π0.5 vs MM-DiT joint attention", 对照与代价, quotes
-    "about 1.2e6" without the derivation; with a full prefix square plus
-    steps x queries x (prefix + suffix keys) the count is about 1.1e6.
-    """
-    sk = suffix_queries if suffix_keys is None else suffix_keys
-    return full_pairs(prefix_tokens) + steps * suffix_queries * (prefix_tokens + sk)

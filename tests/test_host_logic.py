@@ -1,5 +1,5 @@
-"""Host-side logic outside the kernels: the bench's pair counter, batch
-sharding, and the multi-rank timing plumbing (2 gloo ranks on CPU)."""
+"""Host-side logic outside the kernels: the bench's pair counter, the
+multi-rank timing plumbing (2 gloo ranks on CPU), and the launcher checks."""
 
 import os
 import socket
@@ -56,17 +56,6 @@ def test_workload_work_figures():
     assert per_call[5] == 578_000_000
 
 
-def test_batch_shard_covers_batch():
-    for B in (1, 7, 8, 32):
-        for ws in (1, 2, 3, 8):
-            spans = [dist.batch_shard(B, r, ws) for r in range(ws)]
-            assert spans[0][0] == 0 and spans[-1][1] == B
-            for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
-                assert a1 == b0
-            sizes = [b - a for a, b in spans]
-            assert max(sizes) - min(sizes) <= 1
-
-
 _WORKER = r"""
 import os, sys
 sys.path.insert(0, {root!r})
@@ -76,8 +65,7 @@ assert dist.init(backend="gloo", timeout_s=60)
 dist.barrier()
 m = dist.max_over_ranks(10.0 + rank)
 s = dist.sum_over_ranks(1.0)
-lo, hi = dist.batch_shard(16, rank, ws)
-tot = dist.sum_over_ranks(hi - lo)
+tot = dist.sum_over_ranks(8)
 dist.shutdown()
 print("RESULT", rank, m, s, tot, flush=True)
 """
@@ -106,7 +94,7 @@ def test_two_rank_gloo_plumbing():
     for r in res:
         assert float(r[1]) == 11.0      # max over ranks
         assert float(r[2]) == 2.0       # sum over ranks
-        assert float(r[3]) == 16.0      # the shards cover the batch
+        assert float(r[3]) == 16.0      # each rank's 8 batch elements, summed
 
 
 def test_reference_arm_runs_on_cpu():
@@ -124,21 +112,46 @@ def test_reference_arm_runs_on_cpu():
 
 def test_reference_arm_nonzero_rank_exits_quietly():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--steps", "1", "--warmup", "0"], capture_output=True, text=True,
-                       timeout=120, env=dict(os.environ, RANK="1", WORLD_SIZE="2"))
+                        "--gpus", "2", "--steps", "1", "--warmup", "0"], capture_output=True,
+                       text=True, timeout=120,
+                       env=dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1"))
     assert r.returncode == 0 and r.stdout.strip() == ""
 
 
-def test_config_table_oracle_estimate_on_cpu():
-    """bench.py --configs: the oracle's per-call estimate runs on a bounded
-    row sample, and the pair count it reports equals the explicit oracle
-    mask's count."""
-    import bench
-    from vla_prefix_lm_b200 import workloads as W
-    w = W.workload(1)
-    x = W.prefill_inputs(w, W.seed_for(1, 0), B=w.B)
-    s, sample = bench.oracle_seconds_per_call(w, x, max_rows=16, seconds=0.05)
-    assert s > 0 and "16 of 49 query rows" in sample
-    w4 = W.workload(4)
-    M = oracle.prefill_mask(np.array(w4.ar), seg=np.array(w4.seg), B=1)
-    assert bench.visible_pairs_per_bh(w4.ar, w4.seg) == int(M.sum())
+def test_bench_two_rank_plumbing_end_to_end():
+    """bench.py under torch.distributed.run with 2 gloo ranks on CPU: the same
+    barrier / max-over-ranks / whole-job value arithmetic as the GPU arm; rank
+    0 alone prints one line, with n_gpus == 2 and the slower rank's time."""
+    import json
+    port = _free_port()
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                        "--nproc-per-node=2", "--master-addr", "127.0.0.1", "--master-port",
+                        str(port), os.path.join(ROOT, "bench.py"), "--plumbing-check",
+                        "--gpus", "2", "--steps", "4", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300,
+                       env=dict(os.environ, CUDA_VISIBLE_DEVICES=""))
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["steps"] == 4
+    assert line["max_rank_ms"] >= line["rank_ms"]          # rank 1 is slower by design
+    assert abs(line["value"] - 2 * 1000 * 4 / (line["max_rank_ms"] / 1e3)) < 1e-6 * line["value"]
+
+
+def test_bench_gpus_mismatch_is_an_error():
+    """--gpus N with a launcher that started a different number of ranks."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "4",
+                        "--steps", "1", "--warmup", "3"], capture_output=True, text=True,
+                       timeout=120, env=dict(os.environ, RANK="0", WORLD_SIZE="2",
+                                             LOCAL_RANK="0", CUDA_VISIBLE_DEVICES=""))
+    assert r.returncode != 0 and "WORLD_SIZE=2" in r.stderr
+
+
+def test_bench_case_names_cover_profiles():
+    """Every --case a profile summary names exists in bench.py."""
+    import glob
+    import re
+    for f in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        for m in re.findall(r"--case (\w+)", open(f).read()):
+            assert m in bench.CASES, (f, m)

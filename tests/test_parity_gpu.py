@@ -4,8 +4,8 @@ Tolerances: max-abs 2e-2 for bf16 inputs with fp32 accumulation, 1e-4 for the
 fp32 path (the bounds the library's specification states).  Inputs are the
 seeded workload draws; the oracle receives the same rounded values in float64.
 Sizes span several 128-row query tiles and 128-key tiles with ragged tails;
-the full-size workloads are checked in full where the oracle finishes in
-seconds, else on sampled rows.
+the full-size workloads are checked in full (the largest, MM-DiT, on one whole
+call plus one row of every work unit of another).
 """
 
 import numpy as np
@@ -124,19 +124,42 @@ def test_bf16_pi05_workload():
     assert e <= TOL_BF16
 
 
-def test_bf16_mmdit_sampled_rows():
-    """MM-DiT (B=4, S=4250, all False), first and last of the 28 calls, sampled rows."""
+def test_bf16_mmdit_full_call():
+    """MM-DiT (B=4, S=4250, all False), the first of its 28 calls compared in
+    full: every (batch, token, head) row of out and lse against the oracle."""
     w = W.workload(5)
-    rng = np.random.default_rng(5)
-    for call in (0, w.calls - 1):
-        x = W.prefill_inputs(w, W.seed_for(5, call))
-        out = _b().pi_attn_prefill(x.q.cuda(), x.k.cuda(), x.v.cuda(), x.ar.cuda(), None)
-        rows = [(int(b), int(i)) for b, i in zip(rng.integers(0, w.B, 24),
-                                                  rng.integers(0, w.Sq, 24))]
-        rows += [(0, 0), (w.B - 1, w.Sq - 1), (1, 4095), (2, 4096)]
-        ref, _ = oracle.prefill(x.q64, x.k64, x.v64, np.array(w.ar), rows=rows)
-        got = torch.stack([out[b, i] for b, i in rows])
-        assert _err(got, ref) <= TOL_BF16
+    x = W.prefill_inputs(w, W.seed_for(5, 0))
+    tl = torch.empty((w.B, w.Sq, w.Hq), dtype=torch.float32, device="cuda")
+    out = _b().pi_attn_prefill(x.q.cuda(), x.k.cuda(), x.v.cuda(), x.ar.cuda(), None, lse=tl)
+    torch.cuda.synchronize()
+    ref, ref_lse = oracle.prefill(x.q64, x.k64, x.v64, np.array(w.ar))
+    e, el = _err(out, ref), _err(tl, ref_lse)
+    print(f"MM-DiT call 0, all {w.B * w.Sq * w.Hq} rows: max-abs err out {e:.3e}, lse {el:.3e}")
+    assert e <= TOL_BF16
+    assert el <= TOL_BF16
+
+
+def test_bf16_mmdit_every_pair_tile_last_call():
+    """MM-DiT, the last of the 28 calls: one query token (all 8 heads) from
+    every 256-row pair tile (32 tokens) of every batch element, so that every
+    work unit the persistent scheduler walks is compared with the oracle.  The
+    token's offset inside its tile varies, covering both CTAs of the pair."""
+    w = W.workload(5)
+    x = W.prefill_inputs(w, W.seed_for(5, w.calls - 1))
+    out = _b().pi_attn_prefill(x.q.cuda(), x.k.cuda(), x.v.cuda(), x.ar.cuda(), None)
+    torch.cuda.synchronize()
+    tok_per_tile = 256 // w.Hq
+    n_tiles = (w.Sq + tok_per_tile - 1) // tok_per_tile
+    rows = []
+    for b in range(w.B):
+        for t in range(n_tiles):
+            i = min(t * tok_per_tile + (7 * t + 5 * b) % tok_per_tile, w.Sq - 1)
+            rows.append((b, i))
+    ref, _ = oracle.prefill(x.q64, x.k64, x.v64, np.array(w.ar), rows=rows)
+    got = torch.stack([out[b, i] for b, i in rows])
+    e = _err(got, ref)
+    print(f"MM-DiT call {w.calls - 1}, {len(rows)} rows (one per pair tile): max-abs err {e:.3e}")
+    assert e <= TOL_BF16
 
 
 @pytest.mark.parametrize("Hq", [1, 2, 4, 16])

@@ -51,6 +51,7 @@
 // Every wait is bounded (DevCtl).  Counters that index barriers and ring
 // slots run across units; each ring has a single consumer thread, which
 // waits on its slots in fill order.
+#include <atomic>
 #include <cfloat>
 
 #include "launch.h"
@@ -945,14 +946,22 @@ cudaError_t launch_mode(const TcParams& p, bool suffix_mode, const DevCtl& ctl, 
                        : launch_pair<true, false, L>(p, ctl, grid, st);
 }
 
+// SM count of the current device, looked up once per device (a process may
+// drive GPUs with different counts).
 int sm_count() {
-  static const int n = [] {
-    int dev = 0, v = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-      cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    return v > 0 ? v : 148;
-  }();
-  return n;
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> cache[kMaxDev];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < kMaxDev) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int v = 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    v = 148;
+  if (dev < kMaxDev) cache[dev].store(v, std::memory_order_relaxed);
+  return v;
 }
 
 }  // namespace

@@ -66,13 +66,6 @@ def sum_over_ranks(x: float) -> float:
     return float(t.item())
 
 
-def batch_shard(B_total: int, rank: int, world_size: int) -> tuple[int, int]:
-    """[start, stop) of the batch elements rank `rank` owns (contiguous, balanced)."""
-    base, rem = divmod(B_total, world_size)
-    start = rank * base + min(rank, rem)
-    return start, start + base + (1 if rank < rem else 0)
-
-
 def shutdown() -> None:
     if dist.is_initialized():
         dist.destroy_process_group()

@@ -137,6 +137,18 @@ def draw(shape, seed: int, d: int, dtype: str, std_scale: float | None = None):
     return _round(rng.standard_normal(shape) * s, dtype)
 
 
+def device_draw(shape, seed: int, d: int, dtype: str, device, std_scale: float | None = None):
+    """iid N(0,1) * d**-0.25 (or * std_scale) drawn on ``device`` from a seeded
+    torch generator and rounded to ``dtype``.  For timing runs that need many
+    fresh input sets quickly; parity tests use ``draw``, whose float64 values
+    the oracle also receives."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    s = d ** -0.25 if std_scale is None else std_scale
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32) * s
+    return x.to(torch.bfloat16 if dtype == "bf16" else torch.float32)
+
+
 @dataclass
 class PrefillInputs:
     q: torch.Tensor
