@@ -50,7 +50,7 @@ L2_BYTES = 126 * 2**20
 # DRAM traffic of the prefill kernel per launch on the headline workload, from
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only for
 # the kernel sources whose digest is recorded beside it.
-TRAFFIC = {"bytes": None, "src_sha": None, "workload": "mmdit"}
+TRAFFIC = {"bytes": 119506688, "src_sha": "b1592288cba42215", "workload": "mmdit"}
 KERNEL_SOURCES = ("vla_prefix_lm_b200/csrc/tc_pair.cu", "vla_prefix_lm_b200/csrc/common.cuh",
                   "vla_prefix_lm_b200/csrc/mask.cuh")
 
@@ -597,19 +597,21 @@ def prepost_steps(args, dev, stream, rank):
 
 def backward_steps(args, dev, stream, rank):
     """Gradient of the pi0 joint prefill (B=8, S=611): dq, dk, dv from the
-    forward's out and lse, fp32 SIMT.  Visible-pair work: five dot products or
-    updates of length d per (query head, visible key) -- the scores, dP, dV,
-    dQ and dK -- 10 * d FLOP per pair."""
+    forward's out and lse, on tensor cores (a row-dot pass, the score pass,
+    the dK/dV pass and its chunk sum, the dQ pass).  Algorithmic work: the
+    five contractions of length d per (query head, visible key) -- the
+    scores, dP, dV, dK and dQ -- 10 * d FLOP per pair."""
     import torch
 
     from vla_prefix_lm_b200 import binding, dist
     from vla_prefix_lm_b200 import workloads as W
 
     w = W.workload(2)
-    x = W.prefill_inputs(w, W.seed_for(2, 555) + rank * 7, B=w.B)
-    q, k, v, ar = x.q.to(dev), x.k.to(dev), x.v.to(dev), x.ar.to(dev)
-    dout, _ = W.draw(tuple(x.q.shape), 9201 + rank, w.d, w.dtype, 0.5)
-    dout = dout.to(dev)
+    P_ = peaks()
+    q, k, v = (W.device_draw((w.B, w.Sq, h, w.d), 8_000_000 + 10 * rank + j, w.d, w.dtype, dev)
+               for j, h in enumerate((w.Hq, w.Hkv, w.Hkv)))
+    dout = W.device_draw(tuple(q.shape), 8_000_003 + 10 * rank, w.d, w.dtype, dev, 0.5)
+    ar = torch.tensor(w.ar, dtype=torch.uint8, device=dev)
     lse = torch.empty((w.B, w.Sq, w.Hq), dtype=torch.float32, device=dev)
     out = binding.pi_attn_prefill(q, k, v, ar, lse=lse, stream=stream)
     wsb = torch.empty(binding.pi_attn_prefill_backward_workspace_bytes(q, k, ar),
@@ -623,37 +625,38 @@ def backward_steps(args, dev, stream, rank):
                                          workspace=wsb, stream=stream)
 
     with torch.cuda.stream(stream):
-        step()
+        for _ in range(3):
+            step()
     torch.cuda.synchronize()
-    reps = 3
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        step()
+    reps = 20
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
     with torch.cuda.stream(stream):
+        g.replay()
         e0.record(stream)
         for _ in range(reps):
-            step()
+            g.replay()
         e1.record(stream)
     torch.cuda.synchronize()
     us = dist.max_over_ranks(e0.elapsed_time(e1) * 1e3 / reps)
+    del g
     assert binding.pi_attn_read_status(stream) == binding.PI_OK
     pairs = visible_pairs_per_bh(w.ar) * w.B * w.Hq
     flops = 10 * w.d * pairs
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            sm_mhz = float(json.load(f).get("sm_max_mhz", 1965.0))
-    except (OSError, ValueError):
-        sm_mhz = 1965.0
-    fp32_peak = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12       # FFMA lanes x 2 FLOP x clock
+    tf = flops / (us / 1e6) / 1e12
     return {
         "workload": "pi0 joint prefill backward: B=8, S=611, Hq=8, d=256, bf16 in, fp32 grads",
         "us_per_call": us,
-        "tflops": flops / (us / 1e6) / 1e12,
-        "bound": "alu",
-        "fp32_fma_peak_tflops": fp32_peak,
-        "frac_of_fp32_peak": flops / (us / 1e6) / 1e12 / fp32_peak,
+        "tflops": tf,
+        "bound": "tensor",
+        "frac_of_bf16_peak": tf / P_["bf16_tflops"],
+        "peak_source": f"{P_['source']} bf16 dense (burst)",
         "algorithmic_flop_per_call": flops,
-        "gpu_launches_per_call": 3,
-        "timing": f"{reps} calls back to back after one warm-up (warm L2)",
+        "workspace_bytes": int(wsb.numel()),
+        "timing": f"CUDA graph of one call replayed {reps}x (warm L2)",
     }
 
 

@@ -34,7 +34,8 @@ int main(void) {
   d.B = 2;
 
   /* workspace queries are host-only */
-  CHECK(pi_attn_prefill_backward_workspace_bytes(&d) == 256 + 2 * 16 * 8 * 4);
+  /* bf16, one KV head, d = 256: D (fp32 per row) and the bf16 P / dS tiles */
+  CHECK(pi_attn_prefill_backward_workspace_bytes(&d) == 2 * 128 * 4 + 2 * (2 * 128 * 64 * 2));
   d.P = 816; d.Sq = 51; d.B = 1;
   (void)pi_attn_suffix_workspace_bytes(&d);
   CHECK(pi_attn_suffix_noalloc_capacity() > 0);

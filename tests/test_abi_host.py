@@ -177,7 +177,13 @@ def test_backward_argument_errors():
     b, L = _lib()
     ws = L.pi_attn_prefill_backward_workspace_bytes
     need = ws(ctypes.byref(_desc(b)))
-    assert need == 256 + 2 * 16 * 8 * 4            # codes (rounded to 256) + D
+    # bf16 / one KV head / d = 256 runs on tensor cores: D (B x rows fp32) and the
+    # bf16 P and dS tiles (B x rows x S rounded up to 64 keys); one row tile, so the
+    # dK/dV pass needs no partial sums.
+    rows = 16 * 8
+    assert need == 2 * rows * 4 + 2 * (2 * rows * 64 * 2)
+    # the SIMT path (fp32): codes (rounded to 256) + D
+    assert ws(ctypes.byref(_desc(b, dtype=b.PI_F32))) == 256 + 2 * rows * 4
 
     def bwd(desc, ws_bytes=need, ptrs=None, seg=None, lse=FAKE):
         p = dict(q=FAKE, k=FAKE, v=FAKE, ar=FAKE, out=FAKE, dout=FAKE, dq=FAKE, dk=FAKE,

@@ -30,7 +30,10 @@ def _b():
 def _check(got, ref, tol, name):
     got = got.cpu().numpy().astype(np.float64)
     err = float(np.abs(got - ref).max())
-    bound = tol * max(1.0, float(np.abs(ref).max()))
+    scale = max(1.0, float(np.abs(ref).max()))
+    bound = tol * scale
+    print(f"{name}: max-abs err {err:.3e}, max|ref| {float(np.abs(ref).max()):.3e}, "
+          f"scaled err {err / scale:.3e} (bound {tol:.0e})")
     assert err <= bound, f"{name}: max err {err:.3e} > {bound:.3e}"
 
 
@@ -106,6 +109,47 @@ def test_backward_f32_grouped_heads_per_batch_masks_and_padding():
     rq, rk, rv = _oracle(q, k, v, art, segt, dout64, scale=0.6)
     for got, ref, n in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
         _check(got, ref, TOL["f32"], n)
+    pad = torch.from_numpy(seg < 0)
+    assert torch.all(dq.cpu()[pad] == 0) and torch.all(dk.cpu()[pad] == 0)
+    assert torch.all(dv.cpu()[pad] == 0)
+
+
+@pytest.mark.parametrize("Hq", [1, 2, 16])
+def test_backward_bf16_head_counts(Hq):
+    """The tensor-core backward at the other head counts it supports: row
+    tiles of 256 / Hq tokens, a ragged last tile and a causal block."""
+    rng = np.random.default_rng(40 + Hq)
+    S = 150
+    ar = np.concatenate([np.zeros(90, np.uint8), (rng.random(S - 90) < 0.5).astype(np.uint8)])
+    q, _ = W.draw((2, S, Hq, 256), 960 + Hq, 256, "bf16")
+    k, _ = W.draw((2, S, 1, 256), 961 + Hq, 256, "bf16")
+    v, _ = W.draw((2, S, 1, 256), 962 + Hq, 256, "bf16")
+    art = torch.from_numpy(ar)
+    (dq, dk, dv), dout64 = _run(q, k, v, art, None, "bf16", 963 + Hq, scale=0.9)
+    rq, rk, rv = _oracle(q, k, v, art, None, dout64, scale=0.9)
+    for got, ref, n in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+        _check(got, ref, TOL["bf16"], n)
+
+
+def test_backward_bf16_per_batch_masks_segments_and_padding():
+    """bf16 on tensor cores: a per-batch ar_mask, FAST / expert tags (the
+    expert <- FAST hole), padded tokens (exact zero gradients) and a length
+    spanning several 256-key groups."""
+    rng = np.random.default_rng(97)
+    B, S, Hq = 3, 530, 8
+    ar = (rng.random((B, S)) < 0.05).astype(np.uint8)
+    seg = rng.choice([0, 1, 2], size=(B, S), p=[0.6, 0.2, 0.2]).astype(np.int32)
+    seg[0, 100:140] = -1
+    seg[1, -30:] = -1
+    seg[2, :5] = -1
+    q, _ = W.draw((B, S, Hq, 256), 971, 256, "bf16")
+    k, _ = W.draw((B, S, 1, 256), 972, 256, "bf16")
+    v, _ = W.draw((B, S, 1, 256), 973, 256, "bf16")
+    art, segt = torch.from_numpy(ar), torch.from_numpy(seg)
+    (dq, dk, dv), dout64 = _run(q, k, v, art, segt, "bf16", 974, scale=0.75)
+    rq, rk, rv = _oracle(q, k, v, art, segt, dout64, scale=0.75)
+    for got, ref, n in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+        _check(got, ref, TOL["bf16"], n)
     pad = torch.from_numpy(seg < 0)
     assert torch.all(dq.cpu()[pad] == 0) and torch.all(dk.cpu()[pad] == 0)
     assert torch.all(dv.cpu()[pad] == 0)

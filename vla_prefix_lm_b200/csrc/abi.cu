@@ -80,7 +80,31 @@ bool encode_rows(CUtensorMap* map, const void* base, uint64_t rows, uint64_t bat
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A [batch][rows][blocks * 64] bf16 tensor (row pitch `pitch` bytes) viewed as
+// 4-D (64, rows, blocks, batch), box (64, box_rows, box_blocks, 1), 128-byte
+// swizzle: the general form of encode_rows for the backward's workspace.
+bool encode_view(CUtensorMap* map, const void* base, uint64_t rows, uint64_t blocks,
+                 uint64_t batch, uint64_t pitch, uint32_t box_rows, uint32_t box_blocks) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {64, rows, blocks, batch};
+  cuuint64_t strides[3] = {pitch, 64 * 2, pitch * rows};
+  cuuint32_t box[4] = {64, box_rows, box_blocks, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The backward runs on tensor cores for the forward's tensor-core geometry
+// (bf16, one KV head, head_dim 256); every other shape uses the SIMT kernels.
+bool backward_on_tensor_cores(const pi_attn_desc* d) {
+  return d->dtype == PI_BF16 && d->Hkv == 1 && d->d == 256 &&
+         (d->Hq == 1 || d->Hq == 2 || d->Hq == 4 || d->Hq == 8 || d->Hq == 16);
+}
 
 int check_desc(const pi_attn_desc* d, bool suffix) {
   if (!d) return PI_ERR_ARG;
@@ -309,6 +333,7 @@ int pi_euler_update(float* x, const void* v, int32_t v_dtype, float dt, int64_t 
 
 size_t pi_attn_prefill_backward_workspace_bytes(const pi_attn_desc* d) {
   if (check_backward_desc(d) != PI_OK || d->B == 0 || d->Sq == 0) return 0;
+  if (backward_on_tensor_cores(d)) return bwd_tc_plan(d->B, d->Sq, d->Hq, sm_count()).bytes;
   return bwd_workspace_bytes(d->B, d->Sq, d->Hq);
 }
 
@@ -321,7 +346,9 @@ int pi_attn_prefill_backward(const pi_attn_desc* d, const void* q, const void* k
   if (d->B == 0 || d->Sq == 0) return PI_OK;
   if (!q || !k || !v || !ar_mask || !out || !lse || !dout || !dq || !dk || !dv || !workspace)
     return PI_ERR_ARG;
-  const size_t need = bwd_workspace_bytes(d->B, d->Sq, d->Hq);
+  const bool tc = backward_on_tensor_cores(d);
+  const BwdTcPlan plan = tc ? bwd_tc_plan(d->B, d->Sq, d->Hq, sm_count()) : BwdTcPlan{};
+  const size_t need = tc ? plan.bytes : bwd_workspace_bytes(d->B, d->Sq, d->Hq);
   if (ws_bytes < need) return PI_ERR_ARG;
   for (const void* ptr : {q, k, v, out, dout, (const void*)dq, (const void*)dk, (const void*)dv,
                           (const void*)workspace})
@@ -329,6 +356,38 @@ int pi_attn_prefill_backward(const pi_attn_desc* d, const void* q, const void* k
   if ((reinterpret_cast<uintptr_t>(lse) & 3u) ||
       (segment_ids && (reinterpret_cast<uintptr_t>(segment_ids) & 3u)))
     return PI_ERR_ALIGN;
+  if (tc) {
+    DevCtl ctl;
+    if (!make_ctl(&ctl)) return PI_ERR_CUDA;
+    BwdTcParams t;
+    std::memset(&t, 0, sizeof(t));
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    const uint64_t rows = (uint64_t)d->Sq * d->Hq;
+    const uint64_t pitch = (uint64_t)plan.Skp * 2;
+    t.D = reinterpret_cast<float*>(w + plan.off_D);
+    t.P = reinterpret_cast<__nv_bfloat16*>(w + plan.off_P);
+    t.dS = reinterpret_cast<__nv_bfloat16*>(w + plan.off_dS);
+    t.part = plan.n_chunks > 1 ? reinterpret_cast<float*>(w + plan.off_part) : nullptr;
+    if (!encode_rows(&t.map_q, q, rows, d->B, 128) ||
+        !encode_rows(&t.map_do, dout, rows, d->B, 128) ||
+        !encode_rows(&t.map_k32, k, d->Sq, d->B, 32) ||
+        !encode_rows(&t.map_v32, v, d->Sq, d->B, 32) ||
+        !encode_rows(&t.map_kh, k, d->Sq, d->B, 64, 2) ||
+        !encode_rows(&t.map_qh, q, rows, d->B, 64, 2) ||
+        !encode_rows(&t.map_doh, dout, rows, d->B, 64, 2) ||
+        !encode_view(&t.map_pT, t.P, rows, plan.Skp / 64, d->B, pitch, 64, 2) ||
+        !encode_view(&t.map_dsT, t.dS, rows, plan.Skp / 64, d->B, pitch, 64, 2) ||
+        !encode_view(&t.map_ds, t.dS, rows, plan.Skp / 64, d->B, pitch, 128, 1))
+      return PI_ERR_CUDA;
+    t.ar = ar_mask; t.seg = segment_ids; t.mask_bs = d->mask_batch_stride;
+    t.out = out; t.dout = dout; t.lse = lse;
+    t.dq = dq; t.dk = dk; t.dv = dv;
+    t.B = d->B; t.S = d->Sq; t.Hq = d->Hq; t.Skp = plan.Skp;
+    t.n_chunks = plan.n_chunks; t.pairs_per_chunk = plan.pairs_per_chunk;
+    t.scale = d->softmax_scale;
+    t.scale_log2 = d->softmax_scale * 1.4426950408889634f;
+    return launched(launch_backward_tc(t, ctl, static_cast<cudaStream_t>(stream)));
+  }
   BwdParams p;
   p.q = q; p.k = k; p.v = v; p.out = out; p.dout = dout; p.lse = lse;
   p.ar = ar_mask; p.seg = segment_ids; p.mask_bs = d->mask_batch_stride;

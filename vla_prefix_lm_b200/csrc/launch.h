@@ -65,6 +65,47 @@ struct BwdParams {
 size_t bwd_workspace_bytes(int B, int S, int Hq);
 cudaError_t launch_backward(const BwdParams& p, cudaStream_t st);
 
+// Gradient of the prefill on tensor cores (bwd_tc.cu): bf16, Hkv = 1, d = 256.
+// Tensor maps are 4-D views (64, rows, column blocks, B) as for TcParams.
+struct BwdTcParams {
+  CUtensorMap map_q;    // q rows [B, S*Hq, 256], box (64, 128, 4, 1)
+  CUtensorMap map_do;   // dout rows, box (64, 128, 4, 1)
+  CUtensorMap map_k32;  // keys [B, S, 256], box (64, 32, 4, 1)
+  CUtensorMap map_v32;  // values, box (64, 32, 4, 1)
+  CUtensorMap map_kh;   // keys, box (64, 64, 2, 1): 64 keys x 128 columns
+  CUtensorMap map_qh;   // q rows, box (64, 64, 2, 1)
+  CUtensorMap map_doh;  // dout rows, box (64, 64, 2, 1)
+  CUtensorMap map_pT;   // P workspace [B, S*Hq, Skp] as (64, rows, Skp/64, B), box (64, 64, 2, 1)
+  CUtensorMap map_dsT;  // dS workspace, box (64, 64, 2, 1)
+  CUtensorMap map_ds;   // dS workspace, box (64, 128, 1, 1)
+  const uint8_t* ar;
+  const int32_t* seg;
+  long long mask_bs;
+  const void* out;      // forward output (bf16), for D
+  const void* dout;
+  const float* lse;     // [B, S*Hq] natural log
+  float* D;             // workspace [B, S*Hq]
+  __nv_bfloat16* P;     // workspace [B, S*Hq, Skp]
+  __nv_bfloat16* dS;    // workspace [B, S*Hq, Skp]
+  float* part;          // workspace: dK/dV partials per row chunk (n_chunks > 1)
+  float* dq;
+  float* dk;
+  float* dv;
+  int B, S, Hq, Skp, n_chunks, pairs_per_chunk;
+  float scale, scale_log2;
+};
+
+// Sizes of the tensor-core backward for a shape: row tiles, key groups, the
+// padded key count of the P / dS workspace, the dK/dV row chunks, and the
+// workspace layout (byte offsets, total).
+struct BwdTcPlan {
+  int n_pairs, n_sup, Skp, n_chunks, pairs_per_chunk;
+  size_t off_D, off_P, off_dS, off_part, bytes;
+};
+BwdTcPlan bwd_tc_plan(int B, int S, int Hq, int sms);
+cudaError_t launch_backward_tc(const BwdTcParams& p, const DevCtl& ctl, cudaStream_t st);
+int sm_count();
+
 cudaError_t launch_rope(const RopeParams& p, const DevCtl& ctl, cudaStream_t st);
 // Shared memory one RoPE CTA may use: (Hq + Hkv) * d * element size must fit.
 size_t rope_max_smem();

@@ -946,6 +946,8 @@ cudaError_t launch_mode(const TcParams& p, bool suffix_mode, const DevCtl& ctl, 
                        : launch_pair<true, false, L>(p, ctl, grid, st);
 }
 
+}  // namespace
+
 // SM count of the current device, looked up once per device (a process may
 // drive GPUs with different counts).
 int sm_count() {
@@ -963,8 +965,6 @@ int sm_count() {
   if (dev < kMaxDev) cache[dev].store(v, std::memory_order_relaxed);
   return v;
 }
-
-}  // namespace
 
 cudaError_t launch_tc_pair(const TcParams& p, bool suffix_mode, const DevCtl& ctl,
                            cudaStream_t st) {
