@@ -882,7 +882,8 @@ def run_reference(args, rank, ws):
 # ------------------------------------------------------------- profiling
 
 
-CASES = ("mmdit_prefill", "pi0_prefill", "pi05_prefill", "pi0_suffix_step", "decode_step")
+CASES = ("mmdit_prefill", "pi0_prefill", "pi05_prefill", "pi0_suffix_step", "decode_step",
+         "pi0_backward")
 
 
 def run_case(args):
@@ -898,7 +899,23 @@ def run_case(args):
     torch.cuda.set_device(dev)
     stream = torch.cuda.Stream(dev)
     name = args.case
-    if name.endswith("_prefill"):
+    if name == "pi0_backward":
+        w = W.workload(2)
+        q, k, v = (W.device_draw((w.B, w.Sq, h, w.d), 7_200_000 + j, w.d, w.dtype, dev)
+                   for j, h in enumerate((w.Hq, w.Hkv, w.Hkv)))
+        dout = W.device_draw(tuple(q.shape), 7_200_003, w.d, w.dtype, dev, 0.5)
+        ar = torch.tensor(w.ar, dtype=torch.uint8, device=dev)
+        lse = torch.empty((w.B, w.Sq, w.Hq), dtype=torch.float32, device=dev)
+        out = binding.pi_attn_prefill(q, k, v, ar, lse=lse, stream=stream)
+        wsb = torch.empty(binding.pi_attn_prefill_backward_workspace_bytes(q, k, ar),
+                          dtype=torch.uint8, device=dev)
+        grads = [torch.empty(t.shape, dtype=torch.float32, device=dev) for t in (q, k, v)]
+
+        def call():
+            binding.pi_attn_prefill_backward(q, k, v, ar, out, lse, dout, dq=grads[0],
+                                             dk=grads[1], dv=grads[2], workspace=wsb,
+                                             stream=stream)
+    elif name.endswith("_prefill"):
         w = W.workload({"mmdit_prefill": 5, "pi0_prefill": 2, "pi05_prefill": 4}[name])
         q, k, v = (W.device_draw((w.B, w.Sq, h, w.d), 7_000_000 + j, w.d, w.dtype, dev)
                    for j, h in enumerate((w.Hq, w.Hkv, w.Hkv)))

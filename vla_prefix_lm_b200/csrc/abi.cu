@@ -384,6 +384,7 @@ int pi_attn_prefill_backward(const pi_attn_desc* d, const void* q, const void* k
     t.dq = dq; t.dk = dk; t.dv = dv;
     t.B = d->B; t.S = d->Sq; t.Hq = d->Hq; t.Skp = plan.Skp;
     t.n_chunks = plan.n_chunks; t.pairs_per_chunk = plan.pairs_per_chunk;
+    t.ns1 = plan.ns1; t.clusters = plan.clusters;
     t.scale = d->softmax_scale;
     t.scale_log2 = d->softmax_scale * 1.4426950408889634f;
     return launched(launch_backward_tc(t, ctl, static_cast<cudaStream_t>(stream)));

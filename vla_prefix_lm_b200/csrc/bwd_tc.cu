@@ -17,23 +17,28 @@
 // once each, every one on tcgen05 pair MMAs (cta_group::2, M = 256 rows over a
 // cluster of two CTAs):
 //
-//   score pass  per 256-row tile (query-major): S = Q K^T and dP = dO V^T on
-//               64-key tiles into TMEM; one thread per row forms P and dS in
-//               fp32 and writes both as bf16 to the caller's workspace
-//               [B, rows, Skp] (Skp = S rounded up to 64).
-//   dK/dV pass  per 256-key tile (key-major): dV += P^T dO and dK += dS^T Q
+//   score pass  query-major: S = Q K^T and dP = dO V^T on 64-key tiles into
+//               TMEM; one thread per row forms P and dS in fp32 and writes
+//               both as bf16 to the caller's workspace [B, rows, Skp] (Skp = S
+//               rounded up to 64).  Persistent: each SM pair takes an equal,
+//               contiguous run of the (batch, 256-row tile, key tile) sequence
+//               and reloads Q and dO only when the row tile changes.
+//   dK/dV pass  key-major, per 256-key group: dV += P^T dO and dK += dS^T Q
 //               over 64-row steps, P^T and dS^T read MN-major from the
 //               workspace; small problems split the rows into chunks whose
 //               partial sums a reduction kernel adds in a fixed order.
 //   dQ pass     per 256-row tile: dQ += dS K over the same 64-key tiles.
+//               Persistent, with two TMEM accumulators so that one tile's
+//               epilogue overlaps the next tile's MMAs.
 //
 // Tiles are skipped by the forward's rule: a 256-key group is visited by a
 // 256-row tile unless no row of it sees any key of the group (block index,
 // expert <- FAST, padding).  The score pass writes all four 64-key tiles of a
 // visited group (exact zeros where masked), so the dK/dV pass, which reads
-// whole groups, never reads an unwritten block.  Everything is deterministic
-// (no atomics).  Every wait is bounded (DevCtl) and a timeout is reported in
-// the status word.
+// whole groups, never reads an unwritten block.  Rows go to global memory
+// through a per-warp shared-memory transpose, so every store instruction
+// writes whole 128-byte lines.  Everything is deterministic (no atomics).
+// Every wait is bounded (DevCtl) and a timeout is reported in the status word.
 #include <cfloat>
 
 #include "launch.h"
@@ -57,14 +62,15 @@ constexpr int kRowTile = kRows * kD * 2;       // [128 x 256]   64 KB (Q, dO in 
 constexpr int kItem32 = 32 * kD * 2;           // [32 x 256]    16 KB (this CTA's keys of a score tile)
 constexpr int kHalf64 = 64 * 128 * 2;          // [64 x 128]    16 KB (64 rows/keys x this CTA's d-half)
 constexpr int kDsTile = kRows * 64 * 2;        // [128 x 64]    16 KB (dS rows of a 64-key tile)
+constexpr int kWarpStage = 32 * 128;           // 4 KB per row warp: 32 rows x 128 B transpose
 
-constexpr int kNS1 = 2, kNS2 = 3, kNS3 = 4;    // ring stages per pass
+constexpr int kNS2 = 3, kNS3 = 4;              // ring stages of the dK/dV and dQ passes
 constexpr int kStage1 = 2 * kItem32;           // K, V items
 constexpr int kStage2 = 4 * kHalf64;           // P^T, dS^T, dO half, Q half
 constexpr int kStage3 = kDsTile + kHalf64;     // dS tile, K half
-constexpr int kOps1 = 2 * kRowTile + kNS1 * kStage1;   // 192 KB
-constexpr int kOps2 = kNS2 * kStage2;                  // 192 KB
-constexpr int kOps3 = kNS3 * kStage3;                  // 128 KB
+__host__ __device__ constexpr int ops1(int ns) { return 2 * kRowTile + ns * kStage1 + 4 * kWarpStage; }
+constexpr int kOps2 = kNS2 * kStage2;                        // 192 KB
+constexpr int kOps3 = kNS3 * kStage3 + 4 * kWarpStage;       // 144 KB
 
 constexpr uint32_t kIdescScore = idesc_bf16_f32(2 * kRows, kKT, false, false);
 constexpr uint32_t kIdescKV = idesc_bf16_f32(2 * kRows, kD, true, true);
@@ -73,10 +79,12 @@ constexpr uint32_t kIdescQ = idesc_bf16_f32(2 * kRows, kD, false, true);
 struct __align__(8) Ctl {
   uint64_t full[4];       // leader: a ring stage of both CTAs landed
   uint64_t empty[4];      // each CTA: its stage may be refilled
-  uint64_t rows_full;     // leader (score pass): Q and dO of both CTAs landed
+  uint64_t qd_full;       // leader (score pass): Q and dO of both CTAs landed
+  uint64_t qd_empty;      // each CTA (score pass): the row tile's last MMA read them
   uint64_t s_full[2];     // each CTA (score pass): S and dP of a tile in TMEM
   uint64_t s_free[2];     // leader (score pass): the pair's 8 row warps read them
-  uint64_t done;          // each CTA: the last accumulation finished
+  uint64_t done[2];       // each CTA: an accumulator is final
+  uint64_t acc_free[2];   // leader (dQ pass): the pair's 8 row warps read an accumulator
   uint64_t drain;         // leader: every MMA issued has completed
   uint32_t tmem_base;
   int abort;
@@ -88,8 +96,9 @@ struct __align__(8) Ctl {
 
 __host__ __device__ constexpr int ctl_bytes() { return ((int)sizeof(Ctl) + 127) / 128 * 128; }
 __host__ __device__ constexpr int pad128(int n) { return (n + 127) / 128 * 128; }
-__host__ __device__ constexpr int smem_need(int ops, int S) {
-  return ops + ctl_bytes() + pad128(S) * 2;
+// Operands, control block, `extra` bytes (rounded to 128), per-token codes.
+__host__ __device__ constexpr int smem_need(int ops, int S, int extra) {
+  return ops + ctl_bytes() + pad128(extra) + pad128(S) * 2;
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -123,15 +132,6 @@ __device__ __forceinline__ void commit_both(uint64_t* bar) {
   umma_commit_pair(mapa_shared(smem_u32(bar), 1));
 }
 
-// Warp-collective: 1 if every token of [tq0, tq1] is an expert (or padding)
-// token.
-__device__ __forceinline__ bool tokens_all_expert(const uint16_t* codes, int tq0, int tq1,
-                                                  int lane) {
-  int all_e = 1;
-  for (int t = tq0 + lane; t <= tq1; t += 32) all_e &= (codes[t] >> 1) & 1;
-  return __all_sync(0xffffffffu, all_e) != 0;
-}
-
 // Whether a 256-row tile whose last token has block index csq1 (all of whose
 // tokens are expert or padding if all_e) may see a key of the 256-key group
 // ks.  False only when no pair of the two can be visible: every key's block
@@ -150,14 +150,84 @@ __device__ __forceinline__ bool group_visible(const Ctl& c, uint32_t csq1, bool 
   return true;
 }
 
-// Common prologue: align the shared-memory base, scan the mask into packed
-// per-token codes and per-128-token summaries.  Returns nullptr (after
-// recording PI_ERR_UNSUPPORTED) if the layout does not fit.
-__device__ __forceinline__ uint8_t* bwd_smem(uint8_t* raw, int ops, int S, int smem_bytes,
-                                             const DevCtl& ctl) {
+// The visited 64-key tile after `kt` (-1: the first) of a row tile, or -1.
+__device__ __forceinline__ int next_tile(const Ctl& c, uint32_t csq1, bool all_e, int kt, int S,
+                                         int n_kt) {
+  int t = kt + 1;
+  while (t < n_kt) {
+    if ((t & 3) != 0) return t;                 // the rest of a visited group
+    if (group_visible(c, csq1, all_e, t >> 2, S)) return t;
+    t += 4;
+  }
+  return -1;
+}
+
+// 1 if every token of [tq0, tq1] is an expert (or padding) token.
+__device__ __forceinline__ bool tokens_all_expert_serial(const uint16_t* codes, int tq0, int tq1) {
+  for (int t = tq0; t <= tq1; ++t)
+    if (((codes[t] >> 1) & 1) == 0) return false;
+  return true;
+}
+
+// Warp-collective store of 32 rows x 128 bytes: lane t holds row t's bytes in
+// v[0..7] (16 bytes each) and row t goes to seg(t).  The rows pass through a
+// 4 KB shared-memory transpose (16-byte chunks XOR-swizzled by row, so both
+// directions are free of bank conflicts); each store instruction then writes
+// four whole rows (four 128-byte lines) instead of 32 scattered pieces.  Rows
+// whose bit in `valid` is clear are not written.
+template <class SegFn>
+__device__ __forceinline__ void store_rows128(uint8_t* stage, const uint4 (&v)[8], uint32_t valid,
+                                              int lane, SegFn seg) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<uint4*>(stage + lane * 128 + ((j ^ (lane & 7)) << 4)) = v[j];
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = 4 * i + (lane >> 3), j = lane & 7;
+    const uint4 x = *reinterpret_cast<const uint4*>(stage + r * 128 + ((j ^ (r & 7)) << 4));
+    if ((valid >> r) & 1u) *reinterpret_cast<uint4*>(seg(r) + 16 * j) = x;
+  }
+  __syncwarp();
+}
+
+// Warp-collective: 32 TMEM lanes (rows) x 256 fp32 columns from `taddr`,
+// times `mul`, to rows row_ptr(r) (256 fp32 each, 16-byte aligned), written
+// in 128-byte lines through `stage`; zeros (no TMEM read) when `zero`.
+template <class RowFn>
+__device__ __forceinline__ void tmem_rows_out(uint32_t taddr, float mul, uint8_t* stage,
+                                              uint32_t valid, int lane, bool zero, RowFn row_ptr) {
+#pragma unroll 1
+  for (int cc = 0; cc < kD / 32; ++cc) {
+    uint32_t o[32];
+    if (!zero) {
+      tmem_ld32(taddr + 32 * cc, o);
+      tmem_ld_wait();
+      reg_fence(o);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = 0u;
+    }
+    uint4 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      v[j] = make_uint4(__float_as_uint(__uint_as_float(o[4 * j]) * mul),
+                        __float_as_uint(__uint_as_float(o[4 * j + 1]) * mul),
+                        __float_as_uint(__uint_as_float(o[4 * j + 2]) * mul),
+                        __float_as_uint(__uint_as_float(o[4 * j + 3]) * mul));
+    store_rows128(stage, v, valid, lane, [&](int r) {
+      return reinterpret_cast<uint8_t*>(row_ptr(r) + 32 * cc);
+    });
+  }
+}
+
+// Common prologue: align the shared-memory base and check the layout fits.
+// Returns nullptr (after recording PI_ERR_UNSUPPORTED) if it does not.
+__device__ __forceinline__ uint8_t* bwd_smem(uint8_t* raw, int need, int smem_bytes,
+                                             const DevCtl& ctl, int S) {
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  if ((int)(smem - raw) + smem_need(ops, S) > smem_bytes || S > kMaxTokens) {
+  if ((int)(smem - raw) + need > smem_bytes || S > kMaxTokens) {
     if (threadIdx.x == 0) record_status(ctl, kStatusUnsupported);
     return nullptr;
   }
@@ -166,41 +236,84 @@ __device__ __forceinline__ uint8_t* bwd_smem(uint8_t* raw, int ops, int S, int s
 
 // ---------------------------------------------------------------- score pass
 
+// Position in a cluster's run of the (batch, row tile, visited key tile)
+// sequence.  Every role walks the same run with its own copy.
+struct TileWalk {
+  int b, pair, kt, left;
+  uint32_t csq1;
+  bool all_e;
+};
+
+__device__ __forceinline__ void walk_enter(TileWalk& w, const Ctl& c, const int* pinfo,
+                                           const uint16_t* codes, int j, int S, int n_kt,
+                                           int tok_per_pair) {
+  const int tq0 = w.pair * tok_per_pair, tq1 = min(tq0 + tok_per_pair, S) - 1;
+  w.csq1 = codes[tq1] >> 2;
+  w.all_e = ((pinfo[w.pair] >> 30) & 1) != 0;
+  w.kt = -1;
+  for (int i = 0; i <= j; ++i) w.kt = next_tile(c, w.csq1, w.all_e, w.kt, S, n_kt);
+}
+
+// Moves to the next tile of the run; returns true if the row tile changed.
+__device__ __forceinline__ bool walk_next(TileWalk& w, const Ctl& c, const int* pinfo,
+                                          const uint16_t* codes, int S, int n_kt, int n_pairs,
+                                          int tok_per_pair) {
+  if (--w.left <= 0) return false;
+  const int nk = next_tile(c, w.csq1, w.all_e, w.kt, S, n_kt);
+  if (nk >= 0) {
+    w.kt = nk;
+    return false;
+  }
+  do {
+    if (++w.pair == n_pairs) {
+      w.pair = 0;
+      ++w.b;
+    }
+  } while ((pinfo[w.pair] & 0x3FFFFFFF) == 0);
+  walk_enter(w, c, pinfo, codes, 0, S, n_kt, tok_per_pair);
+  return true;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     bwd_score_kernel(const __grid_constant__ BwdTcParams p, const DevCtl ctl, int smem_bytes) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = bwd_smem(smem_raw, kOps1, p.S, smem_bytes, ctl);
+  const int S = p.S, Hq = p.Hq, ns = p.ns1;
+  const int rows_per_b = S * Hq;
+  const int n_pairs = (rows_per_b + 2 * kRows - 1) / (2 * kRows);
+  const int ops = ops1(ns);
+  uint8_t* smem = bwd_smem(smem_raw, smem_need(ops, S, n_pairs * 4), smem_bytes, ctl, S);
   if (smem == nullptr) return;
-  Ctl& c = *reinterpret_cast<Ctl*>(smem + kOps1);
-  uint16_t* codes = reinterpret_cast<uint16_t*>(smem + kOps1 + ctl_bytes());
+  Ctl& c = *reinterpret_cast<Ctl*>(smem + ops);
+  int* pinfo = reinterpret_cast<int*>(smem + ops + ctl_bytes());
+  uint16_t* codes = reinterpret_cast<uint16_t*>(smem + ops + ctl_bytes() + pad128(n_pairs * 4));
   uint8_t* sQ = smem;
   uint8_t* sdO = smem + kRowTile;
   uint8_t* ring = smem + 2 * kRowTile;
+  uint8_t* stage = ring + ns * kStage1;
 
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int S = p.S, Hq = p.Hq;
-  const int rows_per_b = S * Hq;
-  const int n_pairs = (rows_per_b + 2 * kRows - 1) / (2 * kRows);
-  const int unit = blockIdx.x >> 1;
-  const int pair = unit % n_pairs, b = unit / n_pairs;
+  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
   const int tok_per_pair = 2 * kRows / Hq;
-  const int tq0 = pair * tok_per_pair, tq1 = min(tq0 + tok_per_pair, S) - 1;
-  const int row0 = pair * 2 * kRows + (int)rank * kRows;   // this CTA's first row
   const int n_sup = (S + kSup - 1) / kSup;
   const int n_kt = (S + kKT - 1) / kKT;
+  // A batch-shared mask: the clusters split the whole run evenly.  Per-batch
+  // masks: one cluster per (batch, row tile), scanning its own batch row.
+  const bool per_batch = p.mask_bs != 0;
+  const int b_mask = per_batch ? cluster / n_pairs : 0;
 
-  const uint8_t* ar_b = p.ar + (long long)b * p.mask_bs;
-  const int32_t* seg_b = p.seg ? p.seg + (long long)b * p.mask_bs : nullptr;
+  const uint8_t* ar_b = p.ar + (long long)b_mask * p.mask_bs;
+  const int32_t* seg_b = p.seg ? p.seg + (long long)b_mask * p.mask_bs : nullptr;
   const Flags32 flags0 = load_flags32(ar_b, seg_b, S, (int)threadIdx.x * 32);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kNS1; ++s) {
+    for (int s = 0; s < ns; ++s) {
       mbar_init(&c.full[s], 1);
       mbar_init(&c.empty[s], 1);
     }
-    mbar_init(&c.rows_full, 1);
+    mbar_init(&c.qd_full, 1);
+    mbar_init(&c.qd_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&c.s_full[s], 1);
       mbar_init(&c.s_free[s], 8);
@@ -214,53 +327,96 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     tma_prefetch_desc(&p.map_v32);
   }
   cluster_sync();
-  // Q and dO of this CTA's 128 rows load during the mask scan.
-  const uint32_t rows_full_l = mapa_shared(smem_u32(&c.rows_full), 0);
-  if (threadIdx.x == 0) {
-    if (leader) mbar_arrive_expect_tx(&c.rows_full, 4 * kRowTile);
-    tma_load_4d_pair(sQ, &p.map_q, rows_full_l, 0, row0, 0, b);
-    tma_load_4d_pair(sdO, &p.map_do, rows_full_l, 0, row0, 0, b);
-  }
   if (warp == 1) {
     tmem_alloc_pair(&c.tmem_base, 256);
     tmem_relinquish_pair();
   }
   build_codes_x32<kT>(ar_b, seg_b, S, pad128(S), codes, c.scan, flags0,
                       TileSums{c.cs_first, c.cs_last, c.flags});
+  // Per row tile: its visited key-tile count, and bit 30 if all its tokens
+  // are experts (or padding).
+  for (int pr = threadIdx.x; pr < n_pairs; pr += kT) {
+    const int tq0 = pr * tok_per_pair, tq1 = min(tq0 + tok_per_pair, S) - 1;
+    const bool all_e = tokens_all_expert_serial(codes, tq0, tq1);
+    const uint32_t csq1 = codes[tq1] >> 2;
+    int cnt = 0;
+    for (int ks = 0; ks < n_sup; ++ks)
+      if (group_visible(c, csq1, all_e, ks, S)) cnt += min(4 * ks + 4, n_kt) - 4 * ks;
+    pinfo[pr] = cnt | (all_e ? (1 << 30) : 0);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = c.tmem_base;
-  const uint32_t csq1 = codes[tq1] >> 2;
-  const bool all_e = tokens_all_expert(codes, tq0, tq1, lane);
+
+  // This cluster's run.
+  TileWalk w0{};
+  {
+    if (per_batch) {
+      w0.b = b_mask;
+      w0.pair = cluster % n_pairs;
+      w0.left = pinfo[w0.pair] & 0x3FFFFFFF;
+      if (w0.left > 0) walk_enter(w0, c, pinfo, codes, 0, S, n_kt, tok_per_pair);
+    } else {
+      long long Tb = 0;
+      for (int pr = 0; pr < n_pairs; ++pr) Tb += pinfo[pr] & 0x3FFFFFFF;
+      const long long T = Tb * p.B;
+      const long long lo = T * cluster / n_clusters, hi = T * (cluster + 1) / n_clusters;
+      w0.left = (int)(hi - lo);
+      if (w0.left > 0) {
+        w0.b = (int)(lo / Tb);
+        long long r = lo - (long long)w0.b * Tb;
+        w0.pair = 0;
+        while (r >= (pinfo[w0.pair] & 0x3FFFFFFF)) {
+          r -= pinfo[w0.pair] & 0x3FFFFFFF;
+          ++w0.pair;
+        }
+        walk_enter(w0, c, pinfo, codes, (int)r, S, n_kt, tok_per_pair);
+      }
+    }
+  }
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
-    uint32_t n = 0;
-    bool ok = true;
-    for (int ks = 0; ks < n_sup && ok; ++ks) {
-      if (!group_visible(c, csq1, all_e, ks, S)) continue;
-      for (int kt = 4 * ks; kt < min(4 * ks + 4, n_kt) && ok; ++kt, ++n) {
-        const int s = (int)(n % kNS1);
-        const uint32_t rel = n / kNS1;
-        if (rel > 0 && !warp_wait(&c.empty[s], (rel - 1) & 1, c, ctl)) { ok = false; break; }
+    TileWalk w = w0;
+    uint32_t n = 0, np = 0;
+    bool new_pair = true, ok = true;
+    const uint32_t qd_full_l = mapa_shared(smem_u32(&c.qd_full), 0);
+    while (w.left > 0 && ok) {
+      if (new_pair) {
+        // Q and dO of the row tile; the previous tile's last MMA read them.
+        if (np > 0 && !warp_wait(&c.qd_empty, (np - 1) & 1, c, ctl)) break;
         if (lane == 0) {
-          const uint32_t full_l = mapa_shared(smem_u32(&c.full[s]), 0);
-          if (leader) mbar_arrive_expect_tx(&c.full[s], 2 * kStage1);
-          uint8_t* st = ring + s * kStage1;
-          // this CTA's 32 keys of the tile, all 256 columns, of K and of V
-          tma_load_4d_pair(st, &p.map_k32, full_l, 0, kt * kKT + 32 * (int)rank, 0, b);
-          tma_load_4d_pair(st + kItem32, &p.map_v32, full_l, 0, kt * kKT + 32 * (int)rank, 0, b);
+          if (leader) mbar_arrive_expect_tx(&c.qd_full, 4 * kRowTile);
+          const int row0 = w.pair * 2 * kRows + (int)rank * kRows;
+          tma_load_4d_pair(sQ, &p.map_q, qd_full_l, 0, row0, 0, w.b);
+          tma_load_4d_pair(sdO, &p.map_do, qd_full_l, 0, row0, 0, w.b);
         }
         __syncwarp();
+        ++np;
       }
+      const int s = (int)(n % ns);
+      const uint32_t rel = n / ns;
+      if (rel > 0 && !warp_wait(&c.empty[s], (rel - 1) & 1, c, ctl)) break;
+      if (lane == 0) {
+        const uint32_t full_l = mapa_shared(smem_u32(&c.full[s]), 0);
+        if (leader) mbar_arrive_expect_tx(&c.full[s], 2 * kStage1);
+        uint8_t* st = ring + s * kStage1;
+        // this CTA's 32 keys of the tile, all 256 columns, of K and of V
+        tma_load_4d_pair(st, &p.map_k32, full_l, 0, w.kt * kKT + 32 * (int)rank, 0, w.b);
+        tma_load_4d_pair(st + kItem32, &p.map_v32, full_l, 0, w.kt * kKT + 32 * (int)rank, 0,
+                         w.b);
+      }
+      __syncwarp();
+      ++n;
+      new_pair = walk_next(w, c, pinfo, codes, S, n_kt, n_pairs, tok_per_pair);
     }
     // Loads complete on the leader's barriers: wait there (bounded) for the
     // last phase of each, so no copy is in flight when the cluster leaves.
     if (leader && lane == 0) {
-      (void)mbar_wait(&c.rows_full, 0, ctl);
-      for (int s = 0; s < kNS1; ++s) {
-        const uint32_t n_s = n > (uint32_t)s ? (n - (uint32_t)s + kNS1 - 1) / kNS1 : 0;
+      if (np > 0) (void)mbar_wait(&c.qd_full, (np - 1) & 1, ctl);
+      for (int s = 0; s < ns; ++s) {
+        const uint32_t n_s = n > (uint32_t)s ? (n - (uint32_t)s + ns - 1) / ns : 0;
         if (n_s > 0) (void)mbar_wait(&c.full[s], (n_s - 1) & 1, ctl);
       }
     }
@@ -271,45 +427,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
       const uint64_t qdesc = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dodesc = sdesc_sw128(smem_u32(sdO), 16, 1024);
       const uint64_t rdesc = sdesc_sw128(smem_u32(ring), 16, 1024);
-      uint32_t n = 0;
-      bool ok = warp_wait(&c.rows_full, 0, c, ctl);
-      for (int ks = 0; ks < n_sup && ok; ++ks) {
-        if (!group_visible(c, csq1, all_e, ks, S)) continue;
-        for (int kt = 4 * ks; kt < min(4 * ks + 4, n_kt) && ok; ++kt, ++n) {
-          const int s = (int)(n % kNS1);
-          if (!warp_wait(&c.full[s], (n / kNS1) & 1, c, ctl)) { ok = false; break; }
-          // S/dP buffer n % 2 was last read by the row warps at tile n - 2.
-          if (n >= 2 && !warp_wait(&c.s_free[n & 1], ((n - 2) >> 1) & 1, c, ctl)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (lane == 0) {
-            const uint64_t kd = rdesc + (uint64_t)((s * kStage1) >> 4);
-            const uint64_t vd = rdesc + (uint64_t)((s * kStage1 + kItem32) >> 4);
-            const uint32_t tS = tmem + 64 * (n & 1), tP = tmem + 128 + 64 * (n & 1);
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              // A: [128 rows x 16 d] of Q / dO; B: [32 keys x 16 d] of K / V; both
-              // K-major, 8-row groups 1024 B apart, a K step walks 32 B inside a
-              // 64-column block, then to the next block.
-              const uint32_t aoff = (uint32_t)((kk >> 2) * (kRows * 128) + (kk & 3) * 32);
-              const uint32_t boff = (uint32_t)((kk >> 2) * (32 * 128) + (kk & 3) * 32);
-              umma_pair_ss(tS, qdesc + (aoff >> 4), kd + (boff >> 4), kIdescScore,
-                           kk > 0 ? 1u : 0u);
-            }
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t aoff = (uint32_t)((kk >> 2) * (kRows * 128) + (kk & 3) * 32);
-              const uint32_t boff = (uint32_t)((kk >> 2) * (32 * 128) + (kk & 3) * 32);
-              umma_pair_ss(tP, dodesc + (aoff >> 4), vd + (boff >> 4), kIdescScore,
-                           kk > 0 ? 1u : 0u);
-            }
-            commit_both(&c.empty[s]);
-            commit_both(&c.s_full[n & 1]);
-          }
+      TileWalk w = w0;
+      uint32_t n = 0, np = 0;
+      bool new_pair = true, ok = true;
+      while (w.left > 0 && ok) {
+        if (new_pair) {
+          // Every MMA so far read the previous row tile's Q and dO.
+          if (np > 0 && lane == 0) commit_both(&c.qd_empty);
           __syncwarp();
+          if (!warp_wait(&c.qd_full, np & 1, c, ctl)) break;
+          ++np;
         }
+        const int s = (int)(n % ns);
+        if (!warp_wait(&c.full[s], (n / ns) & 1, c, ctl)) break;
+        // S/dP buffer n % 2 was last read by the row warps at tile n - 2.
+        if (n >= 2 && !warp_wait(&c.s_free[n & 1], ((n - 2) >> 1) & 1, c, ctl)) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint64_t kd = rdesc + (uint64_t)((s * kStage1) >> 4);
+          const uint64_t vd = rdesc + (uint64_t)((s * kStage1 + kItem32) >> 4);
+          const uint32_t tS = tmem + 64 * (n & 1), tP = tmem + 128 + 64 * (n & 1);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            // A: [128 rows x 16 d] of Q / dO; B: [32 keys x 16 d] of K / V; both
+            // K-major, 8-row groups 1024 B apart, a K step walks 32 B inside a
+            // 64-column block, then to the next block.
+            const uint32_t aoff = (uint32_t)((kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+            const uint32_t boff = (uint32_t)((kk >> 2) * (32 * 128) + (kk & 3) * 32);
+            umma_pair_ss(tS, qdesc + (aoff >> 4), kd + (boff >> 4), kIdescScore,
+                         kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t aoff = (uint32_t)((kk >> 2) * (kRows * 128) + (kk & 3) * 32);
+            const uint32_t boff = (uint32_t)((kk >> 2) * (32 * 128) + (kk & 3) * 32);
+            umma_pair_ss(tP, dodesc + (aoff >> 4), vd + (boff >> 4), kIdescScore,
+                         kk > 0 ? 1u : 0u);
+          }
+          commit_both(&c.empty[s]);
+          commit_both(&c.s_full[n & 1]);
+        }
+        __syncwarp();
+        ++n;
+        new_pair = walk_next(w, c, pinfo, codes, S, n_kt, n_pairs, tok_per_pair);
       }
       if (lane == 0) umma_commit_pair(smem_u32(&c.drain));
       __syncwarp();
@@ -320,97 +480,108 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const int rho = row0 + r;
-    const bool row_valid = rho < rows_per_b;
-    const int tok = row_valid ? rho / Hq : tq1;
-    const uint32_t cq = codes[tok];
-    const uint32_t csq = cq >> 2;
-    const bool row_expert = (cq & 2u) != 0;
-    const bool row_live = row_valid && !is_pad(cq);
-    const long long grow = (long long)b * rows_per_b + (row_valid ? rho : 0);
-    const float lse2 = row_live ? p.lse[grow] * kLog2e : 0.f;
-    const float Dv = row_live ? p.D[grow] : 0.f;
     const float cs = p.scale_log2;
-    __nv_bfloat16* prow = p.P + grow * p.Skp;
-    __nv_bfloat16* dsrow = p.dS + grow * p.Skp;
     const uint32_t s_free_l0 = mapa_shared(smem_u32(&c.s_free[0]), 0);
     const uint32_t s_free_l1 = mapa_shared(smem_u32(&c.s_free[1]), 0);
+    uint8_t* wstage = stage + quarter * kWarpStage;
+    const long long pitch = (long long)p.Skp * 2;          // bytes per workspace row
+    TileWalk w = w0;
     uint32_t n = 0;
-    bool ok = true;
-    for (int ks = 0; ks < n_sup && ok; ++ks) {
-      if (!group_visible(c, csq1, all_e, ks, S)) continue;
-      for (int kt = 4 * ks; kt < min(4 * ks + 4, n_kt) && ok; ++kt, ++n) {
-        const int bs = (int)(n & 1);
-        const int k0 = kt * kKT;
-        // Keys of this tile the row sees: a prefix (block index is
-        // non-decreasing), minus FAST keys for expert rows and padding keys.
-        int e = 0;
+    bool new_pair = true, ok = true;
+    // Per row tile: this thread's row and the warp's 32 rows.
+    uint32_t csq = 0, valid = 0;
+    bool row_expert = false, row_live = false;
+    float lse2 = 0.f, Dv = 0.f;
+    long long g0 = 0;                                       // global row of the warp's row 0
+    while (w.left > 0 && ok) {
+      if (new_pair) {
+        const int rho0 = w.pair * 2 * kRows + (int)rank * kRows + quarter * 32;
+        const int rho = rho0 + lane;
+        const bool row_valid = rho < rows_per_b;
+        const int tq1 = min(w.pair * tok_per_pair + tok_per_pair, S) - 1;
+        const uint32_t cq = codes[row_valid ? rho / Hq : tq1];
+        csq = cq >> 2;
+        row_expert = (cq & 2u) != 0;
+        row_live = row_valid && !is_pad(cq);
+        g0 = (long long)w.b * rows_per_b + rho0;
+        lse2 = row_live ? p.lse[g0 + lane] * kLog2e : 0.f;
+        Dv = row_live ? p.D[g0 + lane] : 0.f;
+        valid = __ballot_sync(0xffffffffu, row_valid);
+      }
+      const int bs = (int)(n & 1);
+      const int k0 = w.kt * kKT;
+      // Keys of this tile the row sees: a prefix (block index is
+      // non-decreasing), minus FAST keys for expert rows and padding keys.
+      int e = 0;
 #pragma unroll
-        for (int step = kKT; step >= 1; step >>= 1) {
-          const int probe = e + step;
-          if (probe <= kKT && (uint32_t)(codes[k0 + probe - 1] >> 2) <= csq) e = probe;
-        }
-        e = row_live ? min(e, S - k0) : 0;
-        const uint32_t tf = c.flags[kt >> 1];
-        const bool hole = ((tf & 1u) && row_expert) || (tf & 4u);
-        if (!warp_wait(&c.s_full[bs], (n >> 1) & 1, c, ctl)) { ok = false; break; }
-        tc_fence_after();
-        uint32_t s0[32], s1[32], d0[32], d1[32];
-        tmem_ld32(tmem + lane_off + 64 * bs, s0);
-        tmem_ld32(tmem + lane_off + 64 * bs + 32, s1);
-        tmem_ld32(tmem + lane_off + 128 + 64 * bs, d0);
-        tmem_ld32(tmem + lane_off + 128 + 64 * bs + 32, d1);
-        tmem_ld_wait();
-        reg_fence(s0);
-        reg_fence(s1);
-        reg_fence(d0);
-        reg_fence(d1);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(bs ? s_free_l1 : s_free_l0);
-        uint32_t hid0 = 0u, hid1 = 0u;   // bit j: key j of the tile hidden by the hole rule
-        if (hole) {
-          const uint4* kc = reinterpret_cast<const uint4*>(codes + k0);
+      for (int step = kKT; step >= 1; step >>= 1) {
+        const int probe = e + step;
+        if (probe <= kKT && (uint32_t)(codes[k0 + probe - 1] >> 2) <= csq) e = probe;
+      }
+      e = row_live ? min(e, S - k0) : 0;
+      const uint32_t tf = c.flags[w.kt >> 1];
+      const bool hole = ((tf & 1u) && row_expert) || (tf & 4u);
+      if (!warp_wait(&c.s_full[bs], (n >> 1) & 1, c, ctl)) break;
+      tc_fence_after();
+      uint32_t s0[32], s1[32], d0[32], d1[32];
+      tmem_ld32(tmem + lane_off + 64 * bs, s0);
+      tmem_ld32(tmem + lane_off + 64 * bs + 32, s1);
+      tmem_ld32(tmem + lane_off + 128 + 64 * bs, d0);
+      tmem_ld32(tmem + lane_off + 128 + 64 * bs + 32, d1);
+      tmem_ld_wait();
+      reg_fence(s0);
+      reg_fence(s1);
+      reg_fence(d0);
+      reg_fence(d1);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(bs ? s_free_l1 : s_free_l0);
+      uint32_t hid0 = 0u, hid1 = 0u;   // bit j: key j of the tile hidden by the hole rule
+      if (hole) {
+        const uint4* kc = reinterpret_cast<const uint4*>(codes + k0);
 #pragma unroll
-          for (int q8 = 0; q8 < kKT / 8; ++q8) {
-            const uint4 v4 = kc[q8];
-            const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+        for (int q8 = 0; q8 < kKT / 8; ++q8) {
+          const uint4 v4 = kc[q8];
+          const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
-            for (int h = 0; h < 8; ++h) {
-              const int j = 8 * q8 + h;
-              const uint32_t ck = (wv[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
-              const uint32_t hide = ((row_expert && (ck & 1u)) || is_pad(ck)) ? 1u : 0u;
-              if (j < 32) hid0 |= hide << j;
-              else hid1 |= hide << (j - 32);
-            }
-          }
-        }
-        uint32_t pk[32], dk[32];
-#pragma unroll
-        for (int j = 0; j < kKT; j += 2) {
-          float sv0 = __uint_as_float(j < 32 ? s0[j] : s1[j - 32]);
-          float sv1 = __uint_as_float(j + 1 < 32 ? s0[j + 1] : s1[j - 31]);
-          const float dv0 = __uint_as_float(j < 32 ? d0[j] : d1[j - 32]);
-          const float dv1 = __uint_as_float(j + 1 < 32 ? d0[j + 1] : d1[j - 31]);
-          const uint32_t h0 = j < 32 ? (hid0 >> j) & 1u : (hid1 >> (j - 32)) & 1u;
-          const uint32_t h1 = j + 1 < 32 ? (hid0 >> (j + 1)) & 1u : (hid1 >> (j - 31)) & 1u;
-          const float2 t = ffma2(make_float2(sv0, sv1), make_float2(cs, cs),
-                                 make_float2(-lse2, -lse2));
-          const float p0 = (j < e && !h0) ? ex2(t.x) : 0.f;
-          const float p1 = (j + 1 < e && !h1) ? ex2(t.y) : 0.f;
-          pk[j >> 1] = cvt_bf16x2(p0, p1);
-          dk[j >> 1] = cvt_bf16x2(p0 * (dv0 - Dv), p1 * (dv1 - Dv));
-        }
-        if (row_valid) {
-          uint4* pd = reinterpret_cast<uint4*>(prow + k0);
-          uint4* dd = reinterpret_cast<uint4*>(dsrow + k0);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            pd[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-            dd[q] = make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
+          for (int h = 0; h < 8; ++h) {
+            const int j = 8 * q8 + h;
+            const uint32_t ck = (wv[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+            const uint32_t hide = ((row_expert && (ck & 1u)) || is_pad(ck)) ? 1u : 0u;
+            if (j < 32) hid0 |= hide << j;
+            else hid1 |= hide << (j - 32);
           }
         }
       }
+      uint32_t pk[32], dk[32];
+#pragma unroll
+      for (int j = 0; j < kKT; j += 2) {
+        const float sv0 = __uint_as_float(j < 32 ? s0[j] : s1[j - 32]);
+        const float sv1 = __uint_as_float(j + 1 < 32 ? s0[j + 1] : s1[j - 31]);
+        const float dv0 = __uint_as_float(j < 32 ? d0[j] : d1[j - 32]);
+        const float dv1 = __uint_as_float(j + 1 < 32 ? d0[j + 1] : d1[j - 31]);
+        const uint32_t h0 = j < 32 ? (hid0 >> j) & 1u : (hid1 >> (j - 32)) & 1u;
+        const uint32_t h1 = j + 1 < 32 ? (hid0 >> (j + 1)) & 1u : (hid1 >> (j - 31)) & 1u;
+        const float2 t = ffma2(make_float2(sv0, sv1), make_float2(cs, cs),
+                               make_float2(-lse2, -lse2));
+        const float p0 = (j < e && !h0) ? ex2(t.x) : 0.f;
+        const float p1 = (j + 1 < e && !h1) ? ex2(t.y) : 0.f;
+        pk[j >> 1] = cvt_bf16x2(p0, p1);
+        dk[j >> 1] = cvt_bf16x2(p0 * (dv0 - Dv), p1 * (dv1 - Dv));
+      }
+      {
+        uint4 v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        uint8_t* pbase = reinterpret_cast<uint8_t*>(p.P) + g0 * pitch + k0 * 2;
+        store_rows128(wstage, v, valid, lane, [&](int rr) { return pbase + rr * pitch; });
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
+        uint8_t* dbase = reinterpret_cast<uint8_t*>(p.dS) + g0 * pitch + k0 * 2;
+        store_rows128(wstage, v, valid, lane, [&](int rr) { return dbase + rr * pitch; });
+      }
+      ++n;
+      new_pair = walk_next(w, c, pinfo, codes, S, n_kt, n_pairs, tok_per_pair);
     }
   }
 
@@ -424,40 +595,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
   }
 }
 
-// ----------------------------------------------------- epilogue helpers
-
-// Warp-collective: this thread's TMEM row (256 fp32 columns from `col`) times
-// `mul` to dst[0..255] (fp32, 16-byte aligned) when `store`; zeros when `zero`
-// (no TMEM read then).
-__device__ __forceinline__ void tmem_row_out(uint32_t taddr, float mul, float* dst, bool store,
-                                             bool zero) {
-#pragma unroll 1
-  for (int cc = 0; cc < kD / 32; ++cc) {
-    uint32_t o[32];
-    if (!zero) {
-      tmem_ld32(taddr + 32 * cc, o);
-      tmem_ld_wait();
-      reg_fence(o);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 32; ++e) o[e] = 0u;
-    }
-    if (store) {
-#pragma unroll
-      for (int e = 0; e < 32; e += 4)
-        *reinterpret_cast<float4*>(dst + 32 * cc + e) =
-            make_float4(__uint_as_float(o[e]) * mul, __uint_as_float(o[e + 1]) * mul,
-                        __uint_as_float(o[e + 2]) * mul, __uint_as_float(o[e + 3]) * mul);
-    }
-  }
-}
-
 // ------------------------------------------------------------- dK/dV pass
+
+// Warp-collective: 1 if every token of [tq0, tq1] is an expert (or padding)
+// token.
+__device__ __forceinline__ bool tokens_all_expert(const uint16_t* codes, int tq0, int tq1,
+                                                  int lane) {
+  int all_e = 1;
+  for (int t = tq0 + lane; t <= tq1; t += 32) all_e &= (codes[t] >> 1) & 1;
+  return __all_sync(0xffffffffu, all_e) != 0;
+}
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     bwd_dkdv_tc_kernel(const __grid_constant__ BwdTcParams p, const DevCtl ctl, int smem_bytes) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = bwd_smem(smem_raw, kOps2, p.S, smem_bytes, ctl);
+  uint8_t* smem = bwd_smem(smem_raw, smem_need(kOps2, p.S, 0), smem_bytes, ctl, p.S);
   if (smem == nullptr) return;
   Ctl& c = *reinterpret_cast<Ctl*>(smem + kOps2);
   uint16_t* codes = reinterpret_cast<uint16_t*>(smem + kOps2 + ctl_bytes());
@@ -487,7 +639,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
       mbar_init(&c.full[s], 1);
       mbar_init(&c.empty[s], 1);
     }
-    mbar_init(&c.done, 1);
+    mbar_init(&c.done[0], 1);
     mbar_init(&c.drain, 1);
     c.abort = 0;
     fence_barrier_init();
@@ -582,7 +734,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
                          (n > 0 || k4 > 0) ? 1u : 0u);
           }
           commit_both(&c.empty[s]);
-          if (n + 1 == n_total) commit_both(&c.done);
+          if (n + 1 == n_total) commit_both(&c.done[0]);
         }
         __syncwarp();
       }
@@ -594,33 +746,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     // ------------------------------------ epilogue warps (both CTAs)
     for (int pt = p_begin; pt < p_end; ++pt) n_total += (uint32_t)tile_steps(pt);
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const int key = ks * kSup + (int)rank * kRows + r;
+    const int key0 = ks * kSup + (int)rank * kRows + quarter * 32;   // the warp's first key
     const bool have = n_total > 0;
     bool ok = true;
     if (have) {
-      ok = warp_wait(&c.done, 0, c, ctl);
+      ok = warp_wait(&c.done[0], 0, c, ctl);
       tc_fence_after();
     }
     if (ok) {
-      float* dkdst;
-      float* dvdst;
-      bool store;
+      // Every MMA has completed, so the ring is free: each warp transposes
+      // its rows through its own 4 KB of it.
+      uint8_t* wstage = ring + quarter * kWarpStage;
+      float* dkbase;
+      float* dvbase;
+      uint32_t valid;
       if (p.n_chunks == 1) {
-        store = key < S;
-        const long long o = ((long long)b * S + (store ? key : 0)) * kD;
-        dkdst = p.dk + o;
-        dvdst = p.dv + o;
+        valid = __ballot_sync(0xffffffffu, key0 + lane < S);
+        const long long o = ((long long)b * S + key0) * kD;
+        dkbase = p.dk + o;
+        dvbase = p.dv + o;
       } else {
-        store = true;
+        valid = 0xffffffffu;
         const long long kpad = (long long)n_sup * kSup;
-        const long long o = (((long long)chunk * p.B + b) * kpad + key) * kD;
-        dkdst = p.part + o;
-        dvdst = p.part + (long long)p.n_chunks * p.B * kpad * kD + o;
+        const long long o = (((long long)chunk * p.B + b) * kpad + key0) * kD;
+        dkbase = p.part + o;
+        dvbase = p.part + (long long)p.n_chunks * p.B * kpad * kD + o;
       }
-      tmem_row_out(tdK + lane_off, p.scale, dkdst, store, !have);
-      tmem_row_out(tdV + lane_off, 1.f, dvdst, store, !have);
+      tmem_rows_out(tdK + lane_off, p.scale, wstage, valid, lane, !have,
+                    [&](int rr) { return dkbase + (long long)rr * kD; });
+      tmem_rows_out(tdV + lane_off, 1.f, wstage, valid, lane, !have,
+                    [&](int rr) { return dvbase + (long long)rr * kD; });
     }
   }
 
@@ -639,11 +795,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     bwd_dq_tc_kernel(const __grid_constant__ BwdTcParams p, const DevCtl ctl, int smem_bytes) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = bwd_smem(smem_raw, kOps3, p.S, smem_bytes, ctl);
+  uint8_t* smem = bwd_smem(smem_raw, smem_need(kOps3, p.S, 0), smem_bytes, ctl, p.S);
   if (smem == nullptr) return;
   Ctl& c = *reinterpret_cast<Ctl*>(smem + kOps3);
   uint16_t* codes = reinterpret_cast<uint16_t*>(smem + kOps3 + ctl_bytes());
   uint8_t* ring = smem;
+  uint8_t* stage = smem + kNS3 * kStage3;
 
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -651,16 +808,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
   const int S = p.S, Hq = p.Hq;
   const int rows_per_b = S * Hq;
   const int n_pairs = (rows_per_b + 2 * kRows - 1) / (2 * kRows);
-  const int unit = blockIdx.x >> 1;
-  const int pair = unit % n_pairs, b = unit / n_pairs;
+  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+  const int n_units = p.B * n_pairs;
   const int tok_per_pair = 2 * kRows / Hq;
-  const int tq0 = pair * tok_per_pair, tq1 = min(tq0 + tok_per_pair, S) - 1;
-  const int row0 = pair * 2 * kRows + (int)rank * kRows;
   const int n_sup = (S + kSup - 1) / kSup;
   const int n_kt = (S + kKT - 1) / kKT;
+  // A batch-shared mask: clusters walk units c, c + C, ...; per-batch masks:
+  // one unit per cluster, which scans that unit's batch row.
+  const bool per_batch = p.mask_bs != 0;
+  const int b_mask = per_batch ? cluster / n_pairs : 0;
 
-  const uint8_t* ar_b = p.ar + (long long)b * p.mask_bs;
-  const int32_t* seg_b = p.seg ? p.seg + (long long)b * p.mask_bs : nullptr;
+  const uint8_t* ar_b = p.ar + (long long)b_mask * p.mask_bs;
+  const int32_t* seg_b = p.seg ? p.seg + (long long)b_mask * p.mask_bs : nullptr;
   const Flags32 flags0 = load_flags32(ar_b, seg_b, S, (int)threadIdx.x * 32);
 
   if (threadIdx.x == 0) {
@@ -668,7 +827,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
       mbar_init(&c.full[s], 1);
       mbar_init(&c.empty[s], 1);
     }
-    mbar_init(&c.done, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&c.done[a], 1);
+      mbar_init(&c.acc_free[a], 8);
+    }
     mbar_init(&c.drain, 1);
     c.abort = 0;
     fence_barrier_init();
@@ -677,7 +839,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
   }
   cluster_sync();
   if (warp == 1) {
-    tmem_alloc_pair(&c.tmem_base, 256);
+    tmem_alloc_pair(&c.tmem_base, 512);
     tmem_relinquish_pair();
   }
   build_codes_x32<kT>(ar_b, seg_b, S, pad128(S), codes, c.scan, flags0,
@@ -686,18 +848,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = c.tmem_base;
-  const uint32_t csq1 = codes[tq1] >> 2;
-  const bool all_e = tokens_all_expert(codes, tq0, tq1, lane);
-  uint32_t n_total = 0;
-  for (int ks = 0; ks < n_sup; ++ks)
-    if (group_visible(c, csq1, all_e, ks, S)) n_total += (uint32_t)(min(4 * ks + 4, n_kt) - 4 * ks);
+
+  // Visited key tiles of row tile `pair`: kt = first, then next_tile.
+  auto pair_info = [&](int pair, uint32_t& csq1, bool& all_e) {
+    const int tq0 = pair * tok_per_pair, tq1 = min(tq0 + tok_per_pair, S) - 1;
+    csq1 = codes[tq1] >> 2;
+    all_e = tokens_all_expert(codes, tq0, tq1, lane);
+  };
+  const int u_first = cluster, u_step = per_batch ? n_units : n_clusters;
 
   if (warp == 0) {
     uint32_t n = 0;
     bool ok = true;
-    for (int ks = 0; ks < n_sup && ok; ++ks) {
-      if (!group_visible(c, csq1, all_e, ks, S)) continue;
-      for (int kt = 4 * ks; kt < min(4 * ks + 4, n_kt) && ok; ++kt, ++n) {
+    for (int u = u_first; u < n_units && ok; u += u_step) {
+      const int pair = u % n_pairs, b = u / n_pairs;
+      const int row0 = pair * 2 * kRows + (int)rank * kRows;
+      uint32_t csq1;
+      bool all_e;
+      pair_info(pair, csq1, all_e);
+      for (int kt = next_tile(c, csq1, all_e, -1, S, n_kt); kt >= 0 && ok;
+           kt = next_tile(c, csq1, all_e, kt, S, n_kt), ++n) {
         const int s = (int)(n % kNS3);
         const uint32_t rel = n / kNS3;
         if (rel > 0 && !warp_wait(&c.empty[s], (rel - 1) & 1, c, ctl)) { ok = false; break; }
@@ -722,25 +892,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     if (leader) {
       const uint64_t adesc = sdesc_sw128(smem_u32(ring), 16, 1024);
       const uint64_t bdesc = sdesc_sw128(smem_u32(ring), kHalf64 / 2, 1024);
-      uint32_t n = 0;
+      uint32_t n = 0, i = 0;
       bool ok = true;
-      for (; n < n_total && ok; ++n) {
-        const int s = (int)(n % kNS3);
-        if (!warp_wait(&c.full[s], (n / kNS3) & 1, c, ctl)) { ok = false; break; }
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t base = (uint32_t)(s * kStage3);
+      for (int u = u_first; u < n_units && ok; u += u_step, ++i) {
+        const int a = (int)(i & 1);
+        // Accumulator a was last read by the epilogue of unit i - 2.
+        if (i >= 2 && !warp_wait(&c.acc_free[a], ((i - 2) >> 1) & 1, c, ctl)) break;
+        const int pair = u % n_pairs;
+        uint32_t csq1;
+        bool all_e;
+        pair_info(pair, csq1, all_e);
+        uint32_t t = 0;
+        for (int kt = next_tile(c, csq1, all_e, -1, S, n_kt); kt >= 0;
+             kt = next_tile(c, csq1, all_e, kt, S, n_kt), ++n, ++t) {
+          const int s = (int)(n % kNS3);
+          if (!warp_wait(&c.full[s], (n / kNS3) & 1, c, ctl)) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t base = (uint32_t)(s * kStage3);
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            // A = dS [128 rows x 16 keys] K-major (a K step walks 32 B of the
-            // 128-byte line); B = K [16 keys x (128 columns per CTA)] MN-major.
-            umma_pair_ss(tmem, adesc + ((base + k4 * 32) >> 4),
-                         bdesc + ((base + kDsTile + k4 * 2048) >> 4), kIdescQ,
-                         (n > 0 || k4 > 0) ? 1u : 0u);
+            for (int k4 = 0; k4 < 4; ++k4) {
+              // A = dS [128 rows x 16 keys] K-major (a K step walks 32 B of
+              // the 128-byte line); B = K [16 keys x (128 columns per CTA)]
+              // MN-major.
+              umma_pair_ss(tmem + 256 * a, adesc + ((base + k4 * 32) >> 4),
+                           bdesc + ((base + kDsTile + k4 * 2048) >> 4), kIdescQ,
+                           (t > 0 || k4 > 0) ? 1u : 0u);
+            }
+            commit_both(&c.empty[s]);
           }
-          commit_both(&c.empty[s]);
-          if (n + 1 == n_total) commit_both(&c.done);
+          __syncwarp();
         }
+        if (!ok) break;
+        // A unit without tiles still completes a phase of done[a].
+        if (lane == 0) commit_both(&c.done[a]);
         __syncwarp();
       }
       if (lane == 0) umma_commit_pair(smem_u32(&c.drain));
@@ -749,19 +934,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     }
   } else {
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const int rho = row0 + r;
-    const bool row_valid = rho < rows_per_b;
-    const bool have = n_total > 0;
-    bool ok = true;
-    if (have) {
-      ok = warp_wait(&c.done, 0, c, ctl);
+    uint8_t* wstage = stage + quarter * kWarpStage;
+    const uint32_t acc_free_l0 = mapa_shared(smem_u32(&c.acc_free[0]), 0);
+    const uint32_t acc_free_l1 = mapa_shared(smem_u32(&c.acc_free[1]), 0);
+    uint32_t i = 0;
+    for (int u = u_first; u < n_units; u += u_step, ++i) {
+      const int a = (int)(i & 1);
+      const int pair = u % n_pairs, b = u / n_pairs;
+      uint32_t csq1;
+      bool all_e;
+      pair_info(pair, csq1, all_e);
+      const bool have = next_tile(c, csq1, all_e, -1, S, n_kt) >= 0;
+      if (!warp_wait(&c.done[a], (i >> 1) & 1, c, ctl)) break;
       tc_fence_after();
-    }
-    if (ok) {
-      float* dst = p.dq + ((long long)b * rows_per_b + (row_valid ? rho : 0)) * kD;
-      tmem_row_out(tmem + lane_off, p.scale, dst, row_valid, !have);
+      const int rho0 = pair * 2 * kRows + (int)rank * kRows + quarter * 32;
+      const uint32_t valid = __ballot_sync(0xffffffffu, rho0 + lane < rows_per_b);
+      float* base = p.dq + ((long long)b * rows_per_b + rho0) * kD;
+      tmem_rows_out(tmem + 256 * a + lane_off, p.scale, wstage, valid, lane, !have,
+                    [&](int rr) { return base + (long long)rr * kD; });
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(a ? acc_free_l1 : acc_free_l0);
     }
   }
 
@@ -771,7 +965,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
   cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem, 256);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -830,10 +1024,10 @@ __global__ void __launch_bounds__(256)
 }
 
 template <typename K>
-cudaError_t launch_cluster_kernel(K kernel, int clusters, int ops, const BwdTcParams& p,
+cudaError_t launch_cluster_kernel(K kernel, int clusters, int need, const BwdTcParams& p,
                                   const DevCtl& ctl, cudaStream_t st) {
   static_assert(sizeof(BwdTcParams) <= 4096, "kernel parameters too large");
-  const int smem = min(smem_need(ops, p.S) + 1024, kSmemLimit);
+  const int smem = min(need + 1024, kSmemLimit);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemLimit);
   if (e != cudaSuccess) return e;
@@ -849,16 +1043,18 @@ BwdTcPlan bwd_tc_plan(int B, int S, int Hq, int sms) {
   pl.n_pairs = (rows + 2 * kRows - 1) / (2 * kRows);
   pl.n_sup = (S + kSup - 1) / kSup;
   pl.Skp = (S + kKT - 1) / kKT * kKT;
+  pl.clusters = max(sms / 2, 1);
+  // Two K/V stages in the score pass when they fit beside the codes.
+  pl.ns1 = smem_need(ops1(2), S, pl.n_pairs * 4) + 1024 <= kSmemLimit ? 2 : 1;
   // Row chunks of the dK/dV pass: the fewest that keep the SM pairs as busy
   // as any larger count would (whole waves of clusters).
-  const int clusters = max(sms / 2, 1);
   const long long units = (long long)B * pl.n_sup;
   int best = 1;
   double best_t = 1e30;
   for (int c = 1; c <= pl.n_pairs && c <= 64; ++c) {
     const int ppc = (pl.n_pairs + c - 1) / c;
     const int cc = (pl.n_pairs + ppc - 1) / ppc;                  // chunks actually used
-    const double waves = (double)((units * cc + clusters - 1) / clusters);
+    const double waves = (double)((units * cc + pl.clusters - 1) / pl.clusters);
     const double t = waves * ppc;
     if (t < best_t - 1e-9) {
       best_t = t;
@@ -890,9 +1086,13 @@ cudaError_t launch_backward_tc(const BwdTcParams& p, const DevCtl& ctl, cudaStre
   if (e != cudaSuccess) return e;
   const int n_pairs = (p.S * p.Hq + 2 * kRows - 1) / (2 * kRows);
   const int n_sup = (p.S + kSup - 1) / kSup;
-  e = launch_cluster_kernel(bwd_score_kernel, p.B * n_pairs, kOps1, p, ctl, st);
+  const int units = p.B * n_pairs;
+  const int persistent = p.mask_bs == 0 ? min(units, p.clusters) : units;
+  e = launch_cluster_kernel(bwd_score_kernel, persistent,
+                            smem_need(ops1(p.ns1), p.S, n_pairs * 4), p, ctl, st);
   if (e != cudaSuccess) return e;
-  e = launch_cluster_kernel(bwd_dkdv_tc_kernel, p.B * n_sup * p.n_chunks, kOps2, p, ctl, st);
+  e = launch_cluster_kernel(bwd_dkdv_tc_kernel, p.B * n_sup * p.n_chunks,
+                            smem_need(kOps2, p.S, 0), p, ctl, st);
   if (e != cudaSuccess) return e;
   if (p.n_chunks > 1) {
     const long long n4 = (long long)p.B * p.S * (kD / 4);
@@ -902,7 +1102,8 @@ cudaError_t launch_backward_tc(const BwdTcParams& p, const DevCtl& ctl, cudaStre
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  return launch_cluster_kernel(bwd_dq_tc_kernel, p.B * n_pairs, kOps3, p, ctl, st);
+  return launch_cluster_kernel(bwd_dq_tc_kernel, persistent, smem_need(kOps3, p.S, 0), p, ctl,
+                               st);
 }
 
 }  // namespace piattn

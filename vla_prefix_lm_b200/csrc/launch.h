@@ -92,6 +92,8 @@ struct BwdTcParams {
   float* dk;
   float* dv;
   int B, S, Hq, Skp, n_chunks, pairs_per_chunk;
+  int ns1;              // K/V stages of the score pass (1 or 2, by shared memory)
+  int clusters;         // SM pairs the persistent passes use
   float scale, scale_log2;
 };
 
@@ -99,7 +101,7 @@ struct BwdTcParams {
 // padded key count of the P / dS workspace, the dK/dV row chunks, and the
 // workspace layout (byte offsets, total).
 struct BwdTcPlan {
-  int n_pairs, n_sup, Skp, n_chunks, pairs_per_chunk;
+  int n_pairs, n_sup, Skp, n_chunks, pairs_per_chunk, ns1, clusters;
   size_t off_D, off_P, off_dS, off_part, bytes;
 };
 BwdTcPlan bwd_tc_plan(int B, int S, int Hq, int sms);
