@@ -191,6 +191,12 @@ int pi_attn_prefill_backward(const pi_attn_desc* desc, const void* q, const void
  *   pi_attn_suffix_workspace_bytes(desc) bytes (may be NULL when that is 0);
  *   its contents need no initialisation and are garbage afterwards.  Calls
  *   that may overlap on the GPU need distinct workspaces.
+ * Two kernels serve this call.  A suffix of at most 8 query rows (Sq * Hq <=
+ * 8, e.g. the single-token decode of "Pi0-FAST 模型架构", 4.1) streams the cache
+ * through the CUDA cores of a cluster of 8 CTAs per batch element and merges
+ * on chip: it needs no workspace.  Larger suffixes run on the tensor cores;
+ * batches too small to fill the GPU split the cache over several CTA pairs
+ * and need a workspace for the partial results.
  */
 int pi_attn_suffix(const pi_attn_desc* desc, const void* q_suf, const void* k_suf,
                    const void* v_suf, const void* k_cache, const void* v_cache,
@@ -229,6 +235,26 @@ int pi_attn_suffix_masked(const pi_attn_desc* desc, const void* q_suf, const voi
  */
 int pi_attn_debug_mask(const pi_attn_desc* desc, int mode, const uint8_t* ar_mask,
                        const int32_t* segment_ids, uint8_t* mask_out, pi_stream_t stream);
+
+/*
+ * pi_attn_debug_tiles -- writes the tile classes the bf16 prefill kernel uses
+ * to skip work, for comparison with a brute-force scan of the explicit mask.
+ * The kernel walks 256-row query tiles (256 / Hq tokens x Hq heads) against
+ * 128-key tiles; for each pair it decides from the block indices, the FAST /
+ * expert tags and the padding flags of the tokens (the rule of "π0.5 vs
+ * MM-DiT joint attention", π0.5:三段,两处看不到) that no row sees any key
+ * (skipped), that every row sees every key (full) or neither (partial, masked
+ * per element).  This call runs the same scan and classification.
+ *   desc         B, Sq (= S), Hq and mask_batch_stride are read; P must be 0;
+ *                Hq in {1, 2, 4, 8, 16}
+ *   ar_mask, segment_ids   as pi_attn_prefill (device memory)
+ *   classes_out  device uint8 [B][ceil(S*Hq/256)][ceil(S/128)]: 0 skipped,
+ *                1 full, 2 partial
+ * Errors: PI_ERR_ARG, PI_ERR_ALIGN, PI_ERR_UNSUPPORTED before any launch;
+ * PI_ERR_CUDA if the launch fails.
+ */
+int pi_attn_debug_tiles(const pi_attn_desc* desc, const uint8_t* ar_mask,
+                        const int32_t* segment_ids, uint8_t* classes_out, pi_stream_t stream);
 
 /*
  * pi_attn_read_status -- synchronises `stream`, returns the device status word

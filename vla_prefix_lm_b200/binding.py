@@ -39,6 +39,7 @@ EXPORTED = (
     "pi_attn_prefill_backward",
     "pi_attn_prefill_backward_workspace_bytes",
     "pi_attn_suffix_noalloc_capacity",
+    "pi_attn_debug_tiles",
 )
 
 
@@ -104,6 +105,8 @@ def lib() -> ctypes.CDLL:
         L.pi_attn_status_string.restype = ctypes.c_char_p
         L.pi_attn_set_wait_limit.argtypes = [ctypes.c_uint64]
         L.pi_attn_set_wait_limit.restype = ctypes.c_uint64
+        L.pi_attn_debug_tiles.argtypes = [dp, vp, vp, vp, vp]
+        L.pi_attn_debug_tiles.restype = i32
         L.pi_attn_selftest_wait.argtypes = [vp]
         L.pi_attn_selftest_wait.restype = i32
         L.pi_attn_suffix_masked.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -399,6 +402,26 @@ def pi_attn_debug_mask(ar_mask, segment_ids=None, B=None, P=0, mode=0, stream=No
                                   _ptr(out), ctypes.c_void_p(_stream(stream)))
     if rc != PI_OK:
         raise PiAttnError(rc, "pi_attn_debug_mask")
+    return out
+
+
+def pi_attn_debug_tiles(ar_mask, segment_ids=None, B=None, Hq=8, stream=None):
+    """The bf16 prefill kernel's tile classes: uint8 [B, ceil(S*Hq/256),
+    ceil(S/128)], 0 = skipped, 1 = full, 2 = partial."""
+    _need(ar_mask, "ar_mask", torch.uint8)
+    S = ar_mask.shape[-1]
+    if B is None:
+        B = ar_mask.shape[0] if ar_mask.dim() == 2 else 1
+    mbs = _mask_stride(ar_mask, B, S)
+    if segment_ids is not None:
+        _need(segment_ids, "segment_ids", torch.int32)
+    n_pairs = (S * Hq + 255) // 256
+    out = torch.empty((B, n_pairs, (S + 127) // 128), dtype=torch.uint8, device=ar_mask.device)
+    desc = PiAttnDesc(B, S, 0, Hq, 1, 256, PI_BF16, 1.0, mbs)
+    rc = lib().pi_attn_debug_tiles(ctypes.byref(desc), _ptr(ar_mask), _ptr(segment_ids),
+                                   _ptr(out), ctypes.c_void_p(_stream(stream)))
+    if rc != PI_OK:
+        raise PiAttnError(rc, "pi_attn_debug_tiles")
     return out
 
 

@@ -202,6 +202,7 @@ int pi_attn_prefill(const pi_attn_desc* d, const void* q, const void* k, const v
 size_t pi_attn_suffix_workspace_bytes(const pi_attn_desc* d) {
   if (check_desc(d, true) != PI_OK) return 0;
   if (d->dtype != PI_BF16 || d->B == 0 || d->Sq == 0) return 0;
+  if (decode_applies(d->Sq, d->Hq)) return 0;
   return tc_suffix_workspace_bytes(d->B, d->Sq, d->P, d->Hq);
 }
 
@@ -239,6 +240,32 @@ int pi_attn_suffix_masked(const pi_attn_desc* d, const void* q_suf, const void* 
     p.B = d->B; p.Sq = d->Sq; p.P = d->P; p.Hq = d->Hq; p.Hkv = d->Hkv; p.d = d->d;
     p.scale = d->softmax_scale;
     return launched(launch_simt_f32(p, ctl, st));
+  }
+  if (decode_applies(d->Sq, d->Hq)) {
+    // Few query rows: the cache is spread over a cluster of CTAs per batch
+    // element and merged on chip (no workspace).
+    DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (!encode_rows(&p.map_k, k_suf, d->Sq, d->B, 32) ||
+        !encode_rows(&p.map_v, v_suf, d->Sq, d->B, 32))
+      return PI_ERR_CUDA;
+    if (d->P > 0) {
+      if (!encode_rows(&p.map_kc, k_cache, d->P, d->B, 32) ||
+          !encode_rows(&p.map_vc, v_cache, d->P, d->B, 32))
+        return PI_ERR_CUDA;
+    } else {
+      p.map_kc = p.map_k;
+      p.map_vc = p.map_v;
+    }
+    p.q = static_cast<const __nv_bfloat16*>(q_suf);
+    p.ar = ar_mask_suf;
+    p.seg = segment_ids_suf;
+    p.mask_bs = d->mask_batch_stride;
+    p.cache_valid = cache_valid;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.B = d->B; p.Sq = d->Sq; p.P = d->P; p.Hq = d->Hq;
+    p.scale_log2 = d->softmax_scale * 1.4426950408889634f;
+    return launched(launch_decode(p, ctl, st));
   }
   const int splits = tc_suffix_splits(d->B, d->Sq, d->P, d->Hq);
   const size_t need = tc_suffix_workspace_bytes(d->B, d->Sq, d->P, d->Hq);
@@ -416,6 +443,21 @@ int pi_attn_debug_mask(const pi_attn_desc* d, int mode, const uint8_t* ar_mask,
   return launched(launch_debug_mask(mode, d->B, d->Sq, d->P, ar_mask, segment_ids,
                                     d->mask_batch_stride, mask_out,
                                     static_cast<cudaStream_t>(stream)));
+}
+
+int pi_attn_debug_tiles(const pi_attn_desc* d, const uint8_t* ar_mask,
+                        const int32_t* segment_ids, uint8_t* classes_out, pi_stream_t stream) {
+  if (!d || !ar_mask || !classes_out) return PI_ERR_ARG;
+  if (d->B < 0 || d->Sq < 0 || d->P != 0) return PI_ERR_ARG;
+  if (d->mask_batch_stride < 0 || (d->mask_batch_stride != 0 && d->mask_batch_stride < d->Sq))
+    return PI_ERR_ARG;
+  if (d->Sq > kMaxTokens) return PI_ERR_UNSUPPORTED;
+  if (!(d->Hq == 1 || d->Hq == 2 || d->Hq == 4 || d->Hq == 8 || d->Hq == 16))
+    return PI_ERR_UNSUPPORTED;
+  if (segment_ids && (reinterpret_cast<uintptr_t>(segment_ids) & 3u)) return PI_ERR_ALIGN;
+  if (d->B == 0 || d->Sq == 0) return PI_OK;
+  return launched(launch_debug_tiles(ar_mask, segment_ids, d->mask_batch_stride, d->B, d->Sq,
+                                     d->Hq, classes_out, static_cast<cudaStream_t>(stream)));
 }
 
 int pi_attn_read_status(pi_stream_t stream) {

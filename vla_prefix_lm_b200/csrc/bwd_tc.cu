@@ -478,7 +478,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
   } else {
     // ------------------------------------------ row warps (both CTAs)
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float cs = p.scale_log2;
     const uint32_t s_free_l0 = mapa_shared(smem_u32(&c.s_free[0]), 0);
@@ -811,7 +810,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
   const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
   const int n_units = p.B * n_pairs;
   const int tok_per_pair = 2 * kRows / Hq;
-  const int n_sup = (S + kSup - 1) / kSup;
   const int n_kt = (S + kKT - 1) / kKT;
   // A batch-shared mask: clusters walk units c, c + C, ...; per-batch masks:
   // one unit per cluster, which scans that unit's batch row.

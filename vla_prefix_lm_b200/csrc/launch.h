@@ -35,6 +35,10 @@ cudaError_t launch_debug_mask(int mode, int B, int Sq, int P, const uint8_t* ar,
 
 cudaError_t launch_selftest_wait(const DevCtl& ctl, cudaStream_t st);
 
+// Tile classes of the bf16 prefill kernel (tests): out [B][ceil(S*Hq/256)][ceil(S/128)].
+cudaError_t launch_debug_tiles(const uint8_t* ar, const int32_t* seg, long long mask_bs, int B,
+                               int S, int Hq, uint8_t* out, cudaStream_t st);
+
 // Rotary embedding of q (and k) in place at positions cumsum(tmask) - 1
 // (+ the valid prefix count when pmask is given).
 struct RopeParams {
@@ -147,5 +151,30 @@ cudaError_t launch_tc_pair(const TcParams& p, bool suffix_mode, const DevCtl& ct
 
 size_t tc_suffix_workspace_bytes(int B, int Sq, int P, int Hq);
 int tc_suffix_splits(int B, int Sq, int P, int Hq);
+
+// Merges split partials (unnormalised O [splits][rows][256] fp32, then (m, l)
+// [splits][rows][2] in the exp2 domain) into bf16 rows.
+cudaError_t launch_combine(const float* ws, __nv_bfloat16* out, int n_splits, long long n_rows,
+                           cudaStream_t st);
+
+// Suffix pass with at most 8 query rows per batch element (decode.cu): bf16,
+// one KV head, d = 256.  Needs no workspace.  Cache and suffix K/V as 4-D
+// views, box (64, 32, 4, 1).
+struct DecodeParams {
+  CUtensorMap map_kc;
+  CUtensorMap map_vc;
+  CUtensorMap map_k;
+  CUtensorMap map_v;
+  const __nv_bfloat16* q;       // [B, Sq, Hq, 256]
+  const uint8_t* ar;            // suffix ar_mask rows
+  const int32_t* seg;           // suffix segment ids (may be null)
+  long long mask_bs;
+  const uint8_t* cache_valid;   // [B, P] (may be null)
+  __nv_bfloat16* out;
+  int B, Sq, P, Hq;
+  float scale_log2;
+};
+bool decode_applies(int Sq, int Hq);
+cudaError_t launch_decode(const DecodeParams& p, const DevCtl& ctl, cudaStream_t st);
 
 }  // namespace piattn

@@ -946,7 +946,57 @@ cudaError_t launch_mode(const TcParams& p, bool suffix_mode, const DevCtl& ctl, 
                        : launch_pair<true, false, L>(p, ctl, grid, st);
 }
 
+// The tile classes build_tile_list gives, exported for tests: one CTA per
+// (256-row tile, batch element) scans the mask like the attention kernel and
+// writes out[b][pair][key tile] = 0 (skipped), 1 (full) or 2 (partial).
+struct DbgTileSmem {
+  int scan[kThreads / 32];
+  uint16_t list[kMaxTokens / kBN + 2];
+  uint16_t tile_cs_first[kMaxTokens / kBN + 2];
+  uint16_t tile_cs_last[kMaxTokens / kBN + 2];
+  uint8_t tile_fast[kMaxTokens / kBN + 2];
+};
+
+__global__ void __launch_bounds__(kThreads)
+    debug_tiles_kernel(const uint8_t* ar, const int32_t* seg, long long mask_bs, int S, int Hq,
+                       uint8_t* out) {
+  extern __shared__ __align__(16) uint8_t dbg_raw[];
+  DbgTileSmem& sm = *reinterpret_cast<DbgTileSmem*>(dbg_raw);
+  uint16_t* codes = reinterpret_cast<uint16_t*>(dbg_raw + ((sizeof(DbgTileSmem) + 127) / 128) * 128);
+  const int pair = blockIdx.x, b = blockIdx.y, n_pairs = gridDim.x;
+  const int n_kt = (S + kBN - 1) / kBN;
+  const uint8_t* ar_b = ar + (long long)b * mask_bs;
+  const int32_t* seg_b = seg ? seg + (long long)b * mask_bs : nullptr;
+  const Flags32 f0 = load_flags32(ar_b, seg_b, S, (int)threadIdx.x * 32);
+  build_codes_x32<kThreads>(ar_b, seg_b, S, pad_tokens(S), codes, sm.scan, f0,
+                            TileSums{sm.tile_cs_first, sm.tile_cs_last, sm.tile_fast});
+  uint8_t* o = out + ((long long)b * n_pairs + pair) * n_kt;
+  for (int t = threadIdx.x; t < n_kt; t += blockDim.x) o[t] = 0;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int tok_per_pair = 2 * kBM / Hq;
+    const int tq0 = pair * tok_per_pair, tq1 = min(tq0 + tok_per_pair, S) - 1;
+    const int n = build_tile_list(sm, codes, tq0, tq1, S, sm.list, lane);
+    for (int i = lane; i < n; i += 32) {
+      const uint16_t e = sm.list[i];
+      o[e & kTileIndex] = (e & kTilePartial) ? 2 : 1;
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_debug_tiles(const uint8_t* ar, const int32_t* seg, long long mask_bs, int B,
+                               int S, int Hq, uint8_t* out, cudaStream_t st) {
+  const int n_pairs = (S * Hq + 2 * kBM - 1) / (2 * kBM);
+  const int smem = (int)((sizeof(DbgTileSmem) + 127) / 128 * 128) + pad_tokens(S) * 2;
+  static const cudaError_t attr = cudaFuncSetAttribute(
+      debug_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+  if (attr != cudaSuccess) return attr;
+  debug_tiles_kernel<<<dim3(n_pairs, B), kThreads, smem, st>>>(ar, seg, mask_bs, S, Hq, out);
+  return cudaGetLastError();
+}
 
 // SM count of the current device, looked up once per device (a process may
 // drive GPUs with different counts).
@@ -982,6 +1032,12 @@ cudaError_t launch_tc_pair(const TcParams& p, bool suffix_mode, const DevCtl& ct
   const long long n_rows = (long long)p.B * rows;
   combine_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, st>>>(
       p.ws, reinterpret_cast<__nv_bfloat16*>(p.out_ptr), p.n_splits, n_rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const float* ws, __nv_bfloat16* out, int n_splits, long long n_rows,
+                           cudaStream_t st) {
+  combine_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, st>>>(ws, out, n_splits, n_rows);
   return cudaGetLastError();
 }
 
