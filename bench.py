@@ -710,7 +710,8 @@ def decode_steps(args, dev, stream, rank):
         "gb_per_s_algorithmic": bytes_step / (us / 1e6) / 1e9,
         "hbm_frac": bytes_step / (us / 1e6) / 1e9 / P_["hbm_gbs"],
         "algorithmic_bytes_per_step": bytes_step,
-        "splits": binding.pi_attn_suffix_workspace_bytes(q, k, kc, ar) > 0,
+        "kernel": "decode_kernel: a cluster of 8 CTAs per batch element, mma.sync, on-chip merge",
+        "timing": "median of 20 single-call graph replays, L2 flushed before each",
     }
 
 
