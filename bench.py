@@ -509,6 +509,37 @@ def _cold_graph_us(fn, stream, reps=20):
     return float(np.median(t))
 
 
+def _rotating_us(calls, stream, reps=10):
+    """Device time per call of ``calls`` (one per input set, the sets together
+    larger than twice the L2), captured as one CUDA graph and replayed ``reps``
+    times after one untimed replay: every call reads its inputs from HBM, and
+    the L2 holds only the earlier calls' own data."""
+    import torch
+
+    with torch.cuda.stream(stream):
+        for c in calls:
+            c()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for c in calls:
+            c()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g.replay()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / (reps * len(calls))
+
+
+def _n_sets(set_bytes):
+    return max(3, int(np.ceil(2 * L2_BYTES / set_bytes)) + 1)
+
+
 def prepost_steps(args, dev, stream, rank):
     """RoPE and the Euler update around the attention, each timed alone (cold
     L2), and the whole pi0 sampling loop -- per step RoPE of the suffix q/k at
@@ -523,17 +554,21 @@ def prepost_steps(args, dev, stream, rank):
     res = {}
     # prefill: q [8, 611, 8, 256], k [8, 611, 1, 256] bf16, all tokens valid
     B, S, Hq, d = 8, 611, 8, 256
-    q, _ = W.draw((B, S, Hq, d), 9101 + rank, d, "bf16")
-    k, _ = W.draw((B, S, 1, d), 9102 + rank, d, "bf16")
-    q, k = q.to(dev), k.to(dev)
+    set_bytes = B * S * (Hq + 1) * d * 2
+    n = _n_sets(set_bytes)
+    qk = [(W.device_draw((B, S, Hq, d), 9100 + 10 * i + rank, d, "bf16", dev),
+           W.device_draw((B, S, 1, d), 9101 + 10 * i + rank, d, "bf16", dev)) for i in range(n)]
     tm = torch.ones((B, S), dtype=torch.uint8, device=dev)
-    us = dist.max_over_ranks(_cold_graph_us(
-        lambda: binding.pi_rope_inplace(q, k, tm, stream=stream), stream))
-    nb = 2 * (q.numel() + k.numel()) * 2 + tm.numel()
-    res["rope_prefill"] = {"shape": "q [8,611,8,256], k [8,611,1,256] bf16", "us_cold_l2": us,
+    us = dist.max_over_ranks(_rotating_us(
+        [lambda q=q, k=k: binding.pi_rope_inplace(q, k, tm, stream=stream) for q, k in qk],
+        stream))
+    nb = 2 * set_bytes + tm.numel()
+    res["rope_prefill"] = {"shape": "q [8,611,8,256], k [8,611,1,256] bf16", "us_cold": us,
                            "algorithmic_bytes": nb, "gb_per_s": nb / us / 1e3,
-                           "hbm_frac": nb / us / 1e3 / hbm}
-    del q, k, tm
+                           "hbm_frac": nb / us / 1e3 / hbm,
+                           "timing": f"graph over {n} input sets ({n * set_bytes / 2**20:.0f} "
+                                     "MiB > 2 x L2): every call reads HBM"}
+    del qk, tm
 
     # suffix loop of the pi0 workload: B=32, 51 suffix tokens, cache 816, 10 steps
     w = W.workload(3)
@@ -550,18 +585,28 @@ def prepost_steps(args, dev, stream, rank):
     need = binding.pi_attn_suffix_workspace_bytes(ins[0][0], ins[0][1], kc, ins[0][3])
     wsb = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
 
-    q0, k0 = ins[0][0], ins[0][1]
-    us = dist.max_over_ranks(_cold_graph_us(
-        lambda: binding.pi_rope_inplace(q0, k0, sm_, prefix_mask=pm, stream=stream), stream))
-    nb = 2 * (q0.numel() + k0.numel()) * 2 + sm_.numel() + pm.numel()
+    set_bytes = w.B * w.Sq * (w.Hq + 1) * w.d * 2
+    n = _n_sets(set_bytes)
+    qk = [(W.device_draw((w.B, w.Sq, w.Hq, w.d), 9200 + 10 * i + rank, w.d, "bf16", dev),
+           W.device_draw((w.B, w.Sq, 1, w.d), 9201 + 10 * i + rank, w.d, "bf16", dev))
+          for i in range(n)]
+    us = dist.max_over_ranks(_rotating_us(
+        [lambda q=q, k=k: binding.pi_rope_inplace(q, k, sm_, prefix_mask=pm, stream=stream)
+         for q, k in qk], stream))
+    nb = 2 * set_bytes + sm_.numel() + pm.numel()
     res["rope_suffix"] = {"shape": "q [32,51,8,256], k [32,51,1,256] bf16, prefix mask [32,816]",
-                          "us_cold_l2": us, "algorithmic_bytes": nb, "gb_per_s": nb / us / 1e3,
-                          "hbm_frac": nb / us / 1e3 / hbm}
+                          "us_cold": us, "algorithmic_bytes": nb, "gb_per_s": nb / us / 1e3,
+                          "hbm_frac": nb / us / 1e3 / hbm,
+                          "timing": f"graph over {n} input sets ({n * set_bytes / 2**20:.0f} "
+                                    "MiB > 2 x L2): every call reads HBM"}
+    del qk
     us = dist.max_over_ranks(_cold_graph_us(
         lambda: binding.pi_euler_update(x, vel[0], -0.1, stream=stream), stream))
     nb = 3 * x.numel() * 4
     res["euler"] = {"shape": "x, v [32,50,32] fp32", "us_cold_l2": us, "algorithmic_bytes": nb,
-                    "gb_per_s": nb / us / 1e3}
+                    "gb_per_s": nb / us / 1e3,
+                    "timing": "median of 20 single-call graph replays, L2 flushed before each "
+                              "(launch-bound: 0.6 MB)"}
 
     def ctrl():
         for s, (q, k, v, ar) in enumerate(ins):
@@ -662,8 +707,9 @@ def backward_steps(args, dev, stream, rank):
 
 def decode_steps(args, dev, stream, rank):
     """FAST-style single-token decode: B=32 queries of one token (8 heads)
-    against a cache of 880 tokens (816 prefix + 64 generated), cold L2.  Each
-    step reads the whole cache once: HBM-bound."""
+    against a cache of 880 tokens (816 prefix + 64 generated).  Each step reads
+    the whole cache once: HBM-bound.  Timed over rotating caches larger than
+    twice the L2, so every step reads HBM."""
     import torch
 
     from vla_prefix_lm_b200 import binding, dist
@@ -671,47 +717,36 @@ def decode_steps(args, dev, stream, rank):
 
     B, P, Hq, d = 32, 880, 8, 256
     P_ = peaks()
-    kc, _ = W.draw((B, P, 1, d), 9001 + rank, d, "bf16")
-    vc, _ = W.draw((B, P, 1, d), 9002 + rank, d, "bf16")
-    q, _ = W.draw((B, 1, Hq, d), 9003 + rank, d, "bf16")
-    k, _ = W.draw((B, 1, 1, d), 9004 + rank, d, "bf16")
-    v, _ = W.draw((B, 1, 1, d), 9005 + rank, d, "bf16")
-    kc, vc, q, k, v = (t.to(dev) for t in (kc, vc, q, k, v))
+    set_bytes = 2 * B * P * d * 2
+    n = _n_sets(set_bytes)
+    sets = []
+    for i in range(n):
+        s0 = 9000 + 10 * i + 1000 * rank
+        sets.append((W.device_draw((B, 1, Hq, d), s0, d, "bf16", dev),
+                     W.device_draw((B, 1, 1, d), s0 + 1, d, "bf16", dev),
+                     W.device_draw((B, 1, 1, d), s0 + 2, d, "bf16", dev),
+                     W.device_draw((B, P, 1, d), s0 + 3, d, "bf16", dev),
+                     W.device_draw((B, P, 1, d), s0 + 4, d, "bf16", dev)))
     ar = torch.ones(1, dtype=torch.uint8, device=dev)
-    out = torch.empty_like(q)
-    need = binding.pi_attn_suffix_workspace_bytes(q, k, kc, ar)
+    outs = [torch.empty_like(x[0]) for x in sets]
+    need = binding.pi_attn_suffix_workspace_bytes(sets[0][0], sets[0][1], sets[0][3], ar)
     wsb = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            binding.pi_attn_suffix(q, k, v, kc, vc, ar, out=out, workspace=wsb, stream=stream)
-    torch.cuda.synchronize()
-    g1 = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g1, stream=stream):
-        binding.pi_attn_suffix(q, k, v, kc, vc, ar, out=out, workspace=wsb, stream=stream)
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    cold = []
     dist.barrier()
-    for _ in range(20):
-        with torch.cuda.stream(stream):
-            flush.fill_(1.0)
-            e0.record(stream)
-            g1.replay()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        cold.append(e0.elapsed_time(e1) * 1e3)
-    us = dist.max_over_ranks(float(np.median(cold)))
-    del flush
+    us = dist.max_over_ranks(_rotating_us(
+        [lambda x=x, o=o: binding.pi_attn_suffix(x[0], x[1], x[2], x[3], x[4], ar, out=o,
+                                                 workspace=wsb, stream=stream)
+         for x, o in zip(sets, outs)], stream, reps=20))
     assert binding.pi_attn_read_status(stream) == binding.PI_OK
     bytes_step = 2 * B * P * d * 2 + 2 * B * Hq * d * 2 + 2 * B * d * 2
     return {
         "workload": "single-token decode: B=32, Hq=8, d=256, cache 880 (pi_attn_suffix, Sq=1)",
-        "us_per_step_cold_l2": us,
+        "us_per_step_cold": us,
         "gb_per_s_algorithmic": bytes_step / (us / 1e6) / 1e9,
         "hbm_frac": bytes_step / (us / 1e6) / 1e9 / P_["hbm_gbs"],
         "algorithmic_bytes_per_step": bytes_step,
         "kernel": "decode_kernel: a cluster of 8 CTAs per batch element, mma.sync, on-chip merge",
-        "timing": "median of 20 single-call graph replays, L2 flushed before each",
+        "timing": f"graph over {n} caches ({n * set_bytes / 2**20:.0f} MiB > 2 x L2), "
+                  "replayed 20x: every step reads HBM",
     }
 
 
@@ -757,23 +792,25 @@ def suffix_control(args, dev, stream, rank):
     torch.cuda.synchronize()
     us_ctrl = dist.max_over_ranks(e0.elapsed_time(e1) * 1e3 / reps)
 
-    # cold-L2 per step: flush (write > L2) before each single-step graph, outside the events
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-    g1 = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g1, stream=stream):
-        q, k, v, ar = ins[0]
-        binding.pi_attn_suffix(q, k, v, kc, vc, ar, out=outs[0], workspace=wsb, stream=stream)
-    cold = []
-    for _ in range(20):
-        with torch.cuda.stream(stream):
-            flush.fill_(1.0)
-            e0.record(stream)
-            g1.replay()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        cold.append(e0.elapsed_time(e1) * 1e3)
-    us_cold = dist.max_over_ranks(float(np.median(cold)))
-    del flush
+    # cold: one step per input set (its own cache, suffix q/k/v and output), the
+    # sets together larger than twice the L2, so every step reads HBM
+    set_bytes = 2 * w.B * w.P * w.d * 2 + 2 * w.B * w.Sq * w.Hq * w.d * 2 + 2 * w.B * w.Sq * w.d * 2
+    n = _n_sets(set_bytes)
+    cold_sets = []
+    for i in range(n):
+        s0 = 9500 + 10 * i + 1000 * rank
+        cold_sets.append((W.device_draw((w.B, w.Sq, w.Hq, w.d), s0, w.d, "bf16", dev),
+                          W.device_draw((w.B, w.Sq, 1, w.d), s0 + 1, w.d, "bf16", dev),
+                          W.device_draw((w.B, w.Sq, 1, w.d), s0 + 2, w.d, "bf16", dev),
+                          W.device_draw((w.B, w.P, 1, w.d), s0 + 3, w.d, "bf16", dev),
+                          W.device_draw((w.B, w.P, 1, w.d), s0 + 4, w.d, "bf16", dev)))
+    cold_outs = [torch.empty_like(x[0]) for x in cold_sets]
+    ar0 = ins[0][3]
+    us_cold = dist.max_over_ranks(_rotating_us(
+        [lambda x=x, o=o: binding.pi_attn_suffix(x[0], x[1], x[2], x[3], x[4], ar0, out=o,
+                                                 workspace=wsb, stream=stream)
+         for x, o in zip(cold_sets, cold_outs)], stream, reps=20))
+    del cold_sets, cold_outs
     assert binding.pi_attn_read_status(stream) == binding.PI_OK
 
     pairs = visible_pairs_per_bh(w.ar, P=w.P) * w.B * w.Hq
@@ -784,14 +821,16 @@ def suffix_control(args, dev, stream, rank):
         "workload": "pi0_euler_suffix: B=32, Hq=8, d=256, prefix cache 816, 10 steps x 51 tokens",
         "us_per_ctrl": us_ctrl,
         "us_per_step_warm": us_step,
-        "us_per_step_cold_l2": us_cold,
+        "us_per_step_cold": us_cold,
         "pairs_per_s": pairs / (us_step / 1e6),
         "tflops": 4 * w.d * pairs / (us_step / 1e6) / 1e12,
         "gb_per_s_algorithmic_cold": bytes_step / (us_cold / 1e6) / 1e9,
         "hbm_frac_cold": bytes_step / (us_cold / 1e6) / 1e9 / P["hbm_gbs"],
         "algorithmic_bytes_per_step": bytes_step,
         "gpu_launches_per_ctrl": w.calls,
-        "timing": f"graph of 10 steps replayed {reps}x (warm); cold: L2 flushed before each step",
+        "timing": f"warm: graph of 10 steps against one cache replayed {reps}x; cold: graph "
+                  f"over {n} input sets ({n * set_bytes / 2**20:.0f} MiB > 2 x L2, each with "
+                  "its own cache) replayed 20x, every step reading HBM",
     }
 
 
@@ -884,7 +923,7 @@ def run_reference(args, rank, ws):
 
 
 CASES = ("mmdit_prefill", "pi0_prefill", "pi05_prefill", "pi0_suffix_step", "decode_step",
-         "pi0_backward")
+         "pi0_backward", "rope_prefill")
 
 
 def run_case(args):
@@ -900,7 +939,14 @@ def run_case(args):
     torch.cuda.set_device(dev)
     stream = torch.cuda.Stream(dev)
     name = args.case
-    if name == "pi0_backward":
+    if name == "rope_prefill":
+        q = W.device_draw((8, 611, 8, 256), 7_300_000, 256, "bf16", dev)
+        k = W.device_draw((8, 611, 1, 256), 7_300_001, 256, "bf16", dev)
+        tm = torch.ones((8, 611), dtype=torch.uint8, device=dev)
+
+        def call():
+            binding.pi_rope_inplace(q, k, tm, stream=stream)
+    elif name == "pi0_backward":
         w = W.workload(2)
         q, k, v = (W.device_draw((w.B, w.Sq, h, w.d), 7_200_000 + j, w.d, w.dtype, dev)
                    for j, h in enumerate((w.Hq, w.Hkv, w.Hkv)))

@@ -329,9 +329,7 @@ size_t pi_attn_suffix_noalloc_capacity(void);
  * d must be a multiple of 16 and at most 256, B at most 65535, and one
  * token's heads, (Hq + Hkv) * d * element size (Hkv counted only when k is
  * given), at most 160 KiB (else PI_ERR_UNSUPPORTED); base > 1 (10000 for
- * Gemma).  A chunk of tokens whose copy into shared memory does not complete
- * within the wait bound is left unrotated, with PI_ERR_TIMEOUT in the status
- * word (pi_attn_read_status).
+ * Gemma).  The kernel has no device-side waits.
  * Errors as the attention calls (host-side checks, PI_ERR_ALIGN for pointers
  * not 16-byte aligned).
  */

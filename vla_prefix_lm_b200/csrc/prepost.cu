@@ -11,18 +11,20 @@
 //
 // Both kernels are HBM-bound elementwise passes.
 //
-// RoPE: one CTA per (batch, chunk of tokens).  The chunk's q rows and k rows
-// are each one contiguous range of [B, S, H, d], so one bulk asynchronous copy
-// apiece brings them into shared memory; while they are in flight the CTA
-// forms the chunk's positions (a block count of the mask bytes before the
-// chunk, a ballot over its own) and the inverse frequencies base^(-2i/d) in
-// fp64.  A thread then owns one (token, N-column slice of the first half) and
-// the matching slice of the second half: it forms that slice's angles once
-// (the product pos * inv_freq reduced modulo 2*pi in fp64, so that large
-// positions keep fp32-level accuracy), rotates every head of q and k in
-// shared memory, and two bulk stores write the chunk back.  Chunks hold about
-// 32 KB, so several CTAs share an SM and the whole pass is one wave at the
-// pages' sizes.
+// RoPE: one CTA per (batch, run of tokens); a thread owns one (token, 16-byte
+// column slice of the first half of the head) and the matching slice of the
+// second half.  The CTA first forms its tokens' positions (a block count of
+// the mask bytes before the run -- and of the valid prefix tokens -- plus one
+// ballot over the run's own bytes) and the inverse frequencies
+// base^(-2i/d) in fp64.  Each thread then forms its slice's angles once (the
+// product pos * inv_freq reduced modulo 2*pi in fp64, so that positions in
+// the thousands keep fp32 accuracy, then sincosf) and rotates that slice of
+// every head of q and k in place, straight from and to global memory: each
+// warp access is a contiguous run of 16-byte vectors, and with the heads'
+// loads issued together many requests are in flight per SM, which the pass
+// needs to stream at HBM rate.  (A form that staged each run through
+// shared memory with one bulk copy per CTA kept DRAM at a fifth of its
+// bandwidth: too few bytes in flight per SM.)
 #include <algorithm>
 #include <cstdint>
 
@@ -33,9 +35,8 @@ namespace piattn {
 namespace {
 
 constexpr int kRopeThreads = 128;
-constexpr int kRopeMaxTok = 32;                  // one ballot covers a chunk
-constexpr int kRopeChunkBytes = 32 * 1024;       // q + k bytes a chunk aims at
-constexpr int kRopeMaxSmem = 160 * 1024;         // one token's heads must fit
+constexpr int kRopeMaxTok = 32;                  // one ballot covers a CTA's tokens
+constexpr int kRopeMaxSmem = 160 * 1024;         // bound on one token's heads (ABI limit)
 
 template <typename T> struct Vec;
 template <> struct Vec<__nv_bfloat16> { static constexpr int N = 8; };   // 16 B
@@ -62,30 +63,12 @@ __device__ __forceinline__ uint4 pack(const float (&f)[4], float*) {
                     __float_as_uint(f[3]));
 }
 
-// Bulk (untiled) copies: 16-byte aligned addresses, size a multiple of 16.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
-                                         uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                   reinterpret_cast<uint64_t>(dst)),
-               "r"(smem_u32(src)), "r"(bytes)
-               : "memory");
-}
-
 template <typename T>
 __global__ void __launch_bounds__(kRopeThreads)
     rope_kernel(T* q, T* k, const uint8_t* tmask, long long tmask_bs, const uint8_t* pmask,
                 long long pmask_bs, int S, int P, int Hq, int Hkv, int d, int tok,
-                double log2_base, int32_t* pos_out, const DevCtl ctl) {
+                double log2_base, int32_t* pos_out) {
   constexpr int N = Vec<T>::N;
-  extern __shared__ __align__(128) uint8_t rope_smem[];   // q chunk | k chunk
-  __shared__ __align__(8) uint64_t bar;
   __shared__ double s_inv[128];                 // base^(-2i/d), i < d/2 <= 128
   __shared__ int s_count[kRopeThreads / 32];
   __shared__ uint32_t s_bits;
@@ -95,28 +78,10 @@ __global__ void __launch_bounds__(kRopeThreads)
   const int half = d / 2;
   const int vpr = half / N;                     // vectors per half row
   const int Hk = k ? Hkv : 0;
-  const long long bt0 = (long long)b * S + t0;
-  T* gq = q + bt0 * Hq * d;
-  T* gk = k ? k + bt0 * Hkv * d : nullptr;
-  const uint32_t qbytes = (uint32_t)(nt * Hq * d) * sizeof(T);
-  const uint32_t kbytes = (uint32_t)(nt * Hk * d) * sizeof(T);
-  T* sq = reinterpret_cast<T*>(rope_smem);
-  T* sk = reinterpret_cast<T*>(rope_smem + qbytes);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-  if (threadIdx.x == 0) {
-    mbar_init(&bar, 1);
-    fence_barrier_init();
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(&bar, qbytes + kbytes);
-    bulk_g2s(sq, gq, qbytes, &bar);
-    if (kbytes) bulk_g2s(sk, gk, kbytes, &bar);
-  }
-
-  // Positions: valid tokens before the chunk (and valid prefix tokens) by a
-  // block count, the chunk's own mask bits by one ballot.
+  // Positions: valid tokens before the run (and valid prefix tokens) by a
+  // block count, the run's own mask bits by one ballot.
   const uint8_t* tm = tmask + (long long)b * tmask_bs;
   int cnt = 0;
   for (int t = threadIdx.x * 4; t < t0; t += kRopeThreads * 4) {
@@ -145,50 +110,51 @@ __global__ void __launch_bounds__(kRopeThreads)
   for (int w = 0; w < kRopeThreads / 32; ++w) base += s_count[w];
   const uint32_t bits = s_bits;
 
-  const bool ok = __syncthreads_and(mbar_wait(&bar, 0, ctl));
-  if (!ok) {
-    // The status word holds the timeout; give the copies a second bounded
-    // wait so that none is still writing this CTA's shared memory at exit.
-    if (threadIdx.x == 0) mbar_wait(&bar, 0, ctl);
-    return;
-  }
-
+  const int tl = threadIdx.x / vpr, vi = threadIdx.x % vpr;
+  if (tl >= nt) return;
+  const int pos = base + __popc(bits & (0xFFFFFFFFu >> (31 - tl)));
+  const long long bt = (long long)b * S + t0 + tl;
+  if (pos_out && vi == 0) pos_out[bt] = pos;
   const double two_pi = 6.283185307179586476925286766559;
   const double inv_two_pi = 0.15915494309189533576888376337251;
-  for (int idx = threadIdx.x; idx < nt * vpr; idx += kRopeThreads) {
-    const int tl = idx / vpr, vi = idx % vpr;
-    const int pos = base + __popc(bits & (0xFFFFFFFFu >> (31 - tl)));
-    if (pos_out && vi == 0) pos_out[bt0 + tl] = pos;
-    float cs[N], sn[N];
+  float cs[N], sn[N];
 #pragma unroll
-    for (int e = 0; e < N; ++e) {
-      double ang = (double)pos * s_inv[vi * N + e];
-      ang -= two_pi * rint(ang * inv_two_pi);
-      sincosf((float)ang, &sn[e], &cs[e]);
-    }
-    for (int h = 0; h < Hq + Hk; ++h) {
-      T* row = h < Hq ? sq + (tl * Hq + h) * d : sk + (tl * Hk + (h - Hq)) * d;
-      uint4* p1 = reinterpret_cast<uint4*>(row + vi * N);
-      uint4* p2 = reinterpret_cast<uint4*>(row + half + vi * N);
-      float a[N], c[N], o1[N], o2[N];
-      unpack(*p1, a, (T*)nullptr);
-      unpack(*p2, c, (T*)nullptr);
-#pragma unroll
-      for (int e = 0; e < N; ++e) {
-        o1[e] = a[e] * cs[e] - c[e] * sn[e];
-        o2[e] = c[e] * cs[e] + a[e] * sn[e];
-      }
-      *p1 = pack(o1, (T*)nullptr);
-      *p2 = pack(o2, (T*)nullptr);
-    }
+  for (int e = 0; e < N; ++e) {
+    double ang = (double)pos * s_inv[vi * N + e];
+    ang -= two_pi * rint(ang * inv_two_pi);
+    sincosf((float)ang, &sn[e], &cs[e]);
   }
-  fence_proxy_async_smem();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    bulk_s2g(gq, sq, qbytes);
-    if (kbytes) bulk_s2g(gk, sk, kbytes);
-    tma_store_commit();
-    tma_store_wait_read();
+  T* gq = q + bt * Hq * d + vi * N;
+  T* gk = k ? k + bt * Hkv * d + vi * N : nullptr;
+  constexpr int kU = 4;                          // heads whose loads are in flight together
+  for (int h0 = 0; h0 < Hq + Hk; h0 += kU) {
+    uint4 x1[kU], x2[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int h = h0 + u;
+      if (h < Hq + Hk) {
+        T* row = h < Hq ? gq + (long long)h * d : gk + (long long)(h - Hq) * d;
+        x1[u] = *reinterpret_cast<const uint4*>(row);
+        x2[u] = *reinterpret_cast<const uint4*>(row + half);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int h = h0 + u;
+      if (h < Hq + Hk) {
+        T* row = h < Hq ? gq + (long long)h * d : gk + (long long)(h - Hq) * d;
+        float a[N], c[N], o1[N], o2[N];
+        unpack(x1[u], a, (T*)nullptr);
+        unpack(x2[u], c, (T*)nullptr);
+#pragma unroll
+        for (int e = 0; e < N; ++e) {
+          o1[e] = a[e] * cs[e] - c[e] * sn[e];
+          o2[e] = c[e] * cs[e] + a[e] * sn[e];
+        }
+        *reinterpret_cast<uint4*>(row) = pack(o1, (T*)nullptr);
+        *reinterpret_cast<uint4*>(row + half) = pack(o2, (T*)nullptr);
+      }
+    }
   }
 }
 
@@ -227,37 +193,28 @@ __global__ void __launch_bounds__(256)
 
 }  // namespace
 
-int rope_tokens_per_cta(int Hq, int Hkv_used, int d, bool f32) {
-  const int per_tok = (Hq + Hkv_used) * d * (f32 ? 4 : 2);
-  return std::max(1, std::min(kRopeMaxTok, kRopeChunkBytes / per_tok));
+// Tokens per CTA: one thread per (token, 16-byte slice of a half row), at most
+// 32 tokens (one ballot).
+int rope_tokens_per_cta(int d, bool f32) {
+  const int vpr = (d / 2) / (f32 ? 4 : 8);
+  return std::max(1, std::min(kRopeMaxTok, kRopeThreads / std::max(vpr, 1)));
 }
 
 size_t rope_max_smem() { return kRopeMaxSmem; }
 
 cudaError_t launch_rope(const RopeParams& p, const DevCtl& ctl, cudaStream_t st) {
-  const int hk = p.k ? p.Hkv : 0;
-  const int tok = rope_tokens_per_cta(p.Hq, hk, p.d, p.f32);
-  const size_t smem = (size_t)tok * (p.Hq + hk) * p.d * (p.f32 ? 4 : 2);
-  if (smem > (size_t)kRopeMaxSmem) return cudaErrorInvalidValue;
+  (void)ctl;   // no waits in this kernel
+  const int tok = rope_tokens_per_cta(p.d, p.f32);
   dim3 grid((p.S + tok - 1) / tok, p.B);
   const double log2_base = log2((double)p.base);
-  cudaError_t e = cudaSuccess;
   if (p.f32) {
-    if (smem > 48 * 1024)
-      e = cudaFuncSetAttribute(rope_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kRopeMaxSmem);
-    if (e != cudaSuccess) return e;
-    rope_kernel<float><<<grid, kRopeThreads, smem, st>>>(
+    rope_kernel<float><<<grid, kRopeThreads, 0, st>>>(
         static_cast<float*>(p.q), static_cast<float*>(p.k), p.tmask, p.tmask_bs, p.pmask,
-        p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, tok, log2_base, p.pos_out, ctl);
+        p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, tok, log2_base, p.pos_out);
   } else {
-    if (smem > 48 * 1024)
-      e = cudaFuncSetAttribute(rope_kernel<__nv_bfloat16>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, kRopeMaxSmem);
-    if (e != cudaSuccess) return e;
-    rope_kernel<__nv_bfloat16><<<grid, kRopeThreads, smem, st>>>(
+    rope_kernel<__nv_bfloat16><<<grid, kRopeThreads, 0, st>>>(
         static_cast<__nv_bfloat16*>(p.q), static_cast<__nv_bfloat16*>(p.k), p.tmask, p.tmask_bs,
-        p.pmask, p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, tok, log2_base, p.pos_out, ctl);
+        p.pmask, p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, tok, log2_base, p.pos_out);
   }
   return cudaGetLastError();
 }
