@@ -251,8 +251,10 @@ __device__ int build_tile_list(const SmemT& sm, const uint16_t* codes, int tq0, 
 }
 
 // Warp-collective: the unit with index u and this warp's tile list for it.
+// Not inlined: every warp role calls it, and one copy keeps the kernel's code
+// (which far exceeds an SM's instruction cache) smaller.
 template <bool kSuffix, class SmemT>
-__device__ __forceinline__ Unit make_unit(int u, const TcParams& p, int n_pairs, int n_cache,
+__device__ __noinline__ Unit make_unit(int u, const TcParams& p, int n_pairs, int n_cache,
                                           const SmemT& sm, const uint16_t* codes, uint16_t* list,
                                           int lane) {
   Unit x;
@@ -358,12 +360,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // With a single split every unit visits at least one key tile (a valid
   // query sees its own token; a unit of padding rows gets one masked tile),
   // so the first unit's Q can load during the mask scan.
+  // Without segment ids (or in a suffix pass with a cache, whose cached tiles
+  // come first) the unit's first key tile is also known: tile 0, since every
+  // query sees key 0 by the block-index rule.  Its K and V then load during the
+  // scan as well.  (Segment ids can hide tile 0 -- FAST keys from expert rows,
+  // padding -- so those launches wait for the scan.)
   const bool early_q = p.n_splits == 1;
+  const bool early_kv = early_q && (p.seg == nullptr || (kSuffix && p.P > 0));
   if (early_q && threadIdx.x == 0) {
     const int pair0 = cluster % n_pairs, b0 = cluster / n_pairs;
     if (leader) mbar_arrive_expect_tx(&sm.q_full, 2 * kQBytes);
     tma_load_4d_pair(sQ, &p.map_q, mapa_shared(smem_u32(&sm.q_full), 0), 0,
                      pair0 * 2 * kBM + (int)rank * kBM, 0, b0);
+  }
+  if (early_kv && threadIdx.x == 0) {
+    const int b0 = cluster / n_pairs;
+    if (leader) {
+      mbar_arrive_expect_tx(&sm.k_full[0], 2 * kKItem);
+      mbar_arrive_expect_tx(&sm.v_full[0], 2 * kVItem);
+      mbar_arrive_expect_tx(&sm.v_full[1], 2 * kVItem);
+    }
+    const bool cache0 = kSuffix && p.P > 0;
+    const CUtensorMap* mk = cache0 ? &p.map_kc : &p.map_k;
+    const CUtensorMap* mv = cache0 ? &p.map_vch : &p.map_vh;
+    tma_load_4d_pair(kring, mk, mapa_shared(smem_u32(&sm.k_full[0]), 0), 0, 64 * (int)rank, 0,
+                     b0);
+    tma_load_4d_pair(vring, mv, mapa_shared(smem_u32(&sm.v_full[0]), 0), 0, 0, 2 * (int)rank,
+                     b0);
+    tma_load_4d_pair(vring + kVItem, mv, mapa_shared(smem_u32(&sm.v_full[1]), 0), 0, 64,
+                     2 * (int)rank, b0);
   }
   if (warp == 1) {
     tmem_alloc_pair(&sm.tmem_base, 512);
@@ -401,11 +426,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       }
+      const bool first_unit = nq == 0;
       ++nq;
       auto load_k = [&](int idx) -> bool {
         const KvTile kt = kv_tile_at<kSuffix>(list, idx, n_cache, p.P, cache_masked);
         const int s = (int)(uk % kK);
         const uint32_t rel = uk / kK;
+        if (early_kv && first_unit && uk == 0) {  // tile 0's K was issued before the scan
+          ++uk;
+          return true;
+        }
         if (rel > 0 && !warp_wait(&sm.k_empty[s], (rel - 1) & 1, sm, ctl)) return false;
         if (lane == 0) {
           if (leader) mbar_arrive_expect_tx(&sm.k_full[s], 2 * kKItem);
@@ -422,6 +452,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const KvTile kt = kv_tile_at<kSuffix>(list, idx, n_cache, p.P, cache_masked);
         const int s = (int)(uv % kV);
         const uint32_t rel = uv / kV;
+        if (early_kv && first_unit && uv < 2) {   // tile 0's V was issued before the scan
+          ++uv;
+          return true;
+        }
         if (rel > 0 && !warp_wait(&sm.v_empty[s], (rel - 1) & 1, sm, ctl)) return false;
         if (lane == 0) {
           if (leader) mbar_arrive_expect_tx(&sm.v_full[s], 2 * kVItem);
@@ -587,8 +621,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool store_pending = false;    // this warp's output stores may still read P
     bool ok = true;
 
+    // The next unit's tile list is built while the current unit's last PV
+    // runs (the list of the current unit is no longer read then).
+    Unit nx = make_unit<kSuffix>(cluster, p, n_pairs, n_cache, sm, codes, list, lane);
     for (int unit = cluster; unit < n_units && ok; unit += n_clusters) {
-      const Unit x = make_unit<kSuffix>(unit, p, n_pairs, n_cache, sm, codes, list, lane);
+      const Unit x = nx;
       const int row0 = x.pair * 2 * kBM + (int)rank * kBM;
       const bool row_valid = row0 + r < rows_per_b;
       const long long slot = ((long long)x.split * p.B + x.b) * rows_per_b + row0 + r;
@@ -598,6 +635,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           wml[0] = -INFINITY;
           wml[1] = 0.f;
         }
+        if (unit + n_clusters < n_units)
+          nx = make_unit<kSuffix>(unit + n_clusters, p, n_pairs, n_cache, sm, codes, list, lane);
         continue;
       }
       const int tok = min(x.tq0 + ((int)rank * kBM + r) / p.Hq, x.tq1);
@@ -649,56 +688,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(bs ? s_free_l1 : s_free_l0);
-        if (kt.partial) {
-          const int k0 = kt.tile * kBN;
-          int e;
-          bool hole = false;
-          if (kSuffix && kt.src == 1) {
-            e = min(kBN, p.P - k0);
-            if (cache_masked) {
-              // Padded prefix keys: bit j of vb[j / 32] set iff key j is valid.
-              uint32_t vb[4];
+        // Partial tiles and padding rows: one 128-bit visibility mask per row
+        // (bit j of vm[j / 32] = key j visible), applied in a single pass.
+        // The keys a row sees in a partial tile are a prefix (the block index
+        // is non-decreasing), minus the FAST keys for expert rows and the
+        // padding keys for every row; a cached tile with a validity mask keeps
+        // the valid keys of its ragged prefix.
+        if (kt.partial || __any_sync(0xffffffffu, row_pad)) {
+          uint32_t vm[4] = {~0u, ~0u, ~0u, ~0u};
+          if (kt.partial) {
+            const int k0 = kt.tile * kBN;
+            int e;
+            if (kSuffix && kt.src == 1) {
+              e = min(kBN, p.P - k0);
+              if (cache_masked) {
 #pragma unroll
-              for (int w = 0; w < 4; ++w) vb[w] = __ballot_sync(0xffffffffu, vraw[w] != 0u);
+                for (int w = 0; w < 4; ++w) vm[w] = __ballot_sync(0xffffffffu, vraw[w] != 0u);
+              }
+            } else {
+              e = 0;
 #pragma unroll
-              for (int j = 0; j < kBN; ++j)
-                xs[j] = (j < e && ((vb[j >> 5] >> (j & 31)) & 1u)) ? xs[j] : -INFINITY;
-              e = kBN;                              // applied above
-            }
-          } else {
-            e = 0;
+              for (int step = kBN; step >= 1; step >>= 1) {
+                const int probe = e + step;
+                if (probe <= kBN && (uint32_t)(codes[k0 + probe - 1] >> 2) <= csq) e = probe;
+              }
+              e = min(e, n_key_tok - k0);
+              if (kt.any_fast || kt.any_pad) {
+                // FAST bit (padding keys carry it too) and padding, per key.
 #pragma unroll
-            for (int step = kBN; step >= 1; step >>= 1) {
-              const int probe = e + step;
-              if (probe <= kBN && (uint32_t)(codes[k0 + probe - 1] >> 2) <= csq) e = probe;
-            }
-            e = min(e, n_key_tok - k0);
-            hole = (row_expert && kt.any_fast) || kt.any_pad;
-          }
-          if (hole) {
-            // Per key: FAST keys are hidden from expert rows, padding keys
-            // from every row (padding also carries the FAST bit).
-            const uint4* kc = reinterpret_cast<const uint4*>(codes + k0);
-#pragma unroll
-            for (int q8 = 0; q8 < kBN / 8; ++q8) {
-              const uint4 v4 = kc[q8];
-              const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-              for (int h = 0; h < 8; ++h) {
-                const int j = 8 * q8 + h;
-                const uint32_t ck = (wv[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
-                const bool hide = (row_expert && (ck & 1u)) || is_pad(ck);
-                xs[j] = (j < e && !hide) ? xs[j] : -INFINITY;
+                for (int w = 0; w < 4; ++w) {
+                  const uint32_t ck = codes[k0 + 32 * w + lane];
+                  const uint32_t fw = __ballot_sync(0xffffffffu, (ck & 1u) != 0u);
+                  const uint32_t pw = __ballot_sync(0xffffffffu, is_pad(ck));
+                  vm[w] &= ~(row_expert ? fw : pw);
+                }
               }
             }
-          } else {
 #pragma unroll
-            for (int j = 0; j < kBN; ++j) xs[j] = j < e ? xs[j] : -INFINITY;
+            for (int w = 0; w < 4; ++w) {
+              const int lo = 32 * w;
+              vm[w] &= e >= lo + 32 ? ~0u : (e <= lo ? 0u : ((1u << (e - lo)) - 1u));
+            }
           }
-        }
-        if (row_pad) {
+          if (row_pad) vm[0] = vm[1] = vm[2] = vm[3] = 0u;
 #pragma unroll
-          for (int j = 0; j < kBN; ++j) xs[j] = -INFINITY;
+          for (int j = 0; j < kBN; ++j) xs[j] = ((vm[j >> 5] >> (j & 31)) & 1u) ? xs[j] : -INFINITY;
         }
         // Row maximum: eight independent chains of three-input max.
         float m8[8];
@@ -781,6 +815,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------- epilogue
       const uint32_t g_last = g + (uint32_t)x.n_it - 1;
       g += (uint32_t)x.n_it;
+      if (unit + n_clusters < n_units)
+        nx = make_unit<kSuffix>(unit + n_clusters, p, n_pairs, n_cache, sm, codes, list, lane);
       if (!warp_wait(&sm.o_done, g_last & 1, sm, ctl)) { ok = false; break; }
       tc_fence_after();
       const long long grow = (long long)x.b * rows_per_b + row0 + r;
