@@ -97,6 +97,24 @@ bool encode_view(CUtensorMap* map, const void* base, uint64_t rows, uint64_t blo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A [batch][rows][cols] bf16 tensor (row pitch `pitch` bytes) viewed as 3-D
+// (cols, rows, batch), box (32, 32, 1) with the 64-byte swizzle: 32-row by
+// 32-column boxes whose 64-byte rows carry their 16-byte chunks at
+// chunk ^ ((row / 2) % 4); rows past `rows` of a batch element are clipped.
+bool encode_rows64b(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                    uint64_t batch, uint64_t pitch) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, rows, batch};
+  cuuint64_t strides[2] = {pitch, pitch * rows};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // The backward runs on tensor cores for the forward's tensor-core geometry
@@ -404,7 +422,9 @@ int pi_attn_prefill_backward(const pi_attn_desc* d, const void* q, const void* k
         !encode_rows(&t.map_doh, dout, rows, d->B, 64, 2) ||
         !encode_view(&t.map_pT, t.P, rows, plan.Skp / 64, d->B, pitch, 64, 2) ||
         !encode_view(&t.map_dsT, t.dS, rows, plan.Skp / 64, d->B, pitch, 64, 2) ||
-        !encode_view(&t.map_ds, t.dS, rows, plan.Skp / 64, d->B, pitch, 128, 1))
+        !encode_view(&t.map_ds, t.dS, rows, plan.Skp / 64, d->B, pitch, 128, 1) ||
+        !encode_rows64b(&t.map_pw, t.P, plan.Skp, rows, d->B, pitch) ||
+        !encode_rows64b(&t.map_dsw, t.dS, plan.Skp, rows, d->B, pitch))
       return PI_ERR_CUDA;
     t.ar = ar_mask; t.seg = segment_ids; t.mask_bs = d->mask_batch_stride;
     t.out = out; t.dout = dout; t.lse = lse;

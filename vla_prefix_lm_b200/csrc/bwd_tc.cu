@@ -49,6 +49,7 @@ namespace piattn {
 namespace {
 
 constexpr int kT = 192;          // warp 0 TMA, warp 1 TMEM + MMA issue, warps 2..5 rows
+constexpr int kT1 = 320;         // score pass: warps 2..9 rows, two per TMEM lane quarter
 constexpr int kRows = 128;       // rows per CTA (256 per pair)
 constexpr int kD = 256;
 constexpr int kKT = 64;          // keys per score tile (32 per CTA)
@@ -82,13 +83,13 @@ struct __align__(8) Ctl {
   uint64_t qd_full;       // leader (score pass): Q and dO of both CTAs landed
   uint64_t qd_empty;      // each CTA (score pass): the row tile's last MMA read them
   uint64_t s_full[2];     // each CTA (score pass): S and dP of a tile in TMEM
-  uint64_t s_free[2];     // leader (score pass): the pair's 8 row warps read them
+  uint64_t s_free[2];     // leader (score pass): the pair's 16 row warps read them
   uint64_t done[2];       // each CTA: an accumulator is final
   uint64_t acc_free[2];   // leader (dQ pass): the pair's 8 row warps read an accumulator
   uint64_t drain;         // leader: every MMA issued has completed
   uint32_t tmem_base;
   int abort;
-  int scan[kT / 32];
+  int scan[kT1 / 32];
   uint16_t cs_first[kMaxTiles128];
   uint16_t cs_last[kMaxTiles128];
   uint8_t flags[kMaxTiles128];
@@ -274,7 +275,7 @@ __device__ __forceinline__ bool walk_next(TileWalk& w, const Ctl& c, const int* 
   return true;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
     bwd_score_kernel(const __grid_constant__ BwdTcParams p, const DevCtl ctl, int smem_bytes) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int S = p.S, Hq = p.Hq, ns = p.ns1;
@@ -316,7 +317,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     mbar_init(&c.qd_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&c.s_full[s], 1);
-      mbar_init(&c.s_free[s], 8);
+      mbar_init(&c.s_free[s], 16);
     }
     mbar_init(&c.drain, 1);
     c.abort = 0;
@@ -325,17 +326,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     tma_prefetch_desc(&p.map_do);
     tma_prefetch_desc(&p.map_k32);
     tma_prefetch_desc(&p.map_v32);
+    tma_prefetch_desc(&p.map_pw);
+    tma_prefetch_desc(&p.map_dsw);
   }
   cluster_sync();
   if (warp == 1) {
     tmem_alloc_pair(&c.tmem_base, 256);
     tmem_relinquish_pair();
   }
-  build_codes_x32<kT>(ar_b, seg_b, S, pad128(S), codes, c.scan, flags0,
+  build_codes_x32<kT1>(ar_b, seg_b, S, pad128(S), codes, c.scan, flags0,
                       TileSums{c.cs_first, c.cs_last, c.flags});
   // Per row tile: its visited key-tile count, and bit 30 if all its tokens
   // are experts (or padding).
-  for (int pr = threadIdx.x; pr < n_pairs; pr += kT) {
+  for (int pr = threadIdx.x; pr < n_pairs; pr += kT1) {
     const int tq0 = pr * tok_per_pair, tq1 = min(tq0 + tok_per_pair, S) - 1;
     const bool all_e = tokens_all_expert_serial(codes, tq0, tq1);
     const uint32_t csq1 = codes[tq1] >> 2;
@@ -382,6 +385,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     uint32_t n = 0, np = 0;
     bool new_pair = true, ok = true;
     const uint32_t qd_full_l = mapa_shared(smem_u32(&c.qd_full), 0);
+    // K and V are read by every row tile: keep them in L2 against the P and dS
+    // stream this pass writes.
+    const uint64_t keep = l2_policy_evict_last();
     while (w.left > 0 && ok) {
       if (new_pair) {
         // Q and dO of the row tile; the previous tile's last MMA read them.
@@ -403,9 +409,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
         if (leader) mbar_arrive_expect_tx(&c.full[s], 2 * kStage1);
         uint8_t* st = ring + s * kStage1;
         // this CTA's 32 keys of the tile, all 256 columns, of K and of V
-        tma_load_4d_pair(st, &p.map_k32, full_l, 0, w.kt * kKT + 32 * (int)rank, 0, w.b);
-        tma_load_4d_pair(st + kItem32, &p.map_v32, full_l, 0, w.kt * kKT + 32 * (int)rank, 0,
-                         w.b);
+        tma_load_4d_pair_hint(st, &p.map_k32, full_l, 0, w.kt * kKT + 32 * (int)rank, 0, w.b,
+                              keep);
+        tma_load_4d_pair_hint(st + kItem32, &p.map_v32, full_l, 0, w.kt * kKT + 32 * (int)rank,
+                              0, w.b, keep);
       }
       __syncwarp();
       ++n;
@@ -477,24 +484,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     }
   } else {
     // ------------------------------------------ row warps (both CTAs)
+    // A warp reaches only the TMEM lanes of quarter warp % 4; two warps share
+    // each quarter's 32 rows, warp 2 + q + 4h taking keys [32h, 32h + 32) of
+    // every tile.  P = exp2(S c - lse) needs no running maximum, so the halves
+    // never exchange anything.
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float cs = p.scale_log2;
     const uint32_t s_free_l0 = mapa_shared(smem_u32(&c.s_free[0]), 0);
     const uint32_t s_free_l1 = mapa_shared(smem_u32(&c.s_free[1]), 0);
-    uint8_t* wstage = stage + quarter * kWarpStage;
-    const long long pitch = (long long)p.Skp * 2;          // bytes per workspace row
+    // The warp's 32 x 32 P and dS boxes leave by TMA bulk stores from a 2 KB
+    // stage, laid out as the tensor map's 64-byte swizzle expects.
+    uint8_t* wstage = stage + (warp - 2) * (kWarpStage / 2);
+    const uint64_t stream = l2_policy_evict_first();
     TileWalk w = w0;
     uint32_t n = 0;
     bool new_pair = true, ok = true;
-    // Per row tile: this thread's row and the warp's 32 rows.
-    uint32_t csq = 0, valid = 0;
+    bool store_pending = false;   // lane 0's bulk stores may still read the stage
+    // Per row tile: this thread's row.
+    uint32_t csq = 0;
     bool row_expert = false, row_live = false;
     float lse2 = 0.f, Dv = 0.f;
-    long long g0 = 0;                                       // global row of the warp's row 0
+    int rho0 = 0;                                           // the warp's row 0 in its batch element
     while (w.left > 0 && ok) {
       if (new_pair) {
-        const int rho0 = w.pair * 2 * kRows + (int)rank * kRows + quarter * 32;
+        rho0 = w.pair * 2 * kRows + (int)rank * kRows + quarter * 32;
         const int rho = rho0 + lane;
         const bool row_valid = rho < rows_per_b;
         const int tq1 = min(w.pair * tok_per_pair + tok_per_pair, S) - 1;
@@ -502,86 +517,95 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
         csq = cq >> 2;
         row_expert = (cq & 2u) != 0;
         row_live = row_valid && !is_pad(cq);
-        g0 = (long long)w.b * rows_per_b + rho0;
+        const long long g0 = (long long)w.b * rows_per_b + rho0;
         lse2 = row_live ? p.lse[g0 + lane] * kLog2e : 0.f;
         Dv = row_live ? p.D[g0 + lane] : 0.f;
-        valid = __ballot_sync(0xffffffffu, row_valid);
       }
       const int bs = (int)(n & 1);
       const int k0 = w.kt * kKT;
+      const int kh = k0 + 32 * half;                        // this warp's first key
       // Keys of this tile the row sees: a prefix (block index is
       // non-decreasing), minus FAST keys for expert rows and padding keys.
-      int e = 0;
+      // The tile's last key visible means every key is (most tiles).
+      int e = kKT;
+      if ((uint32_t)(codes[min(k0 + kKT, S) - 1] >> 2) > csq) {
+        e = 0;
 #pragma unroll
-      for (int step = kKT; step >= 1; step >>= 1) {
-        const int probe = e + step;
-        if (probe <= kKT && (uint32_t)(codes[k0 + probe - 1] >> 2) <= csq) e = probe;
+        for (int step = kKT; step >= 1; step >>= 1) {
+          const int probe = e + step;
+          if (probe <= kKT && (uint32_t)(codes[k0 + probe - 1] >> 2) <= csq) e = probe;
+        }
       }
-      e = row_live ? min(e, S - k0) : 0;
+      e = row_live ? min(e, S - k0) - 32 * half : 0;       // visible keys of this half
       const uint32_t tf = c.flags[w.kt >> 1];
       const bool hole = ((tf & 1u) && row_expert) || (tf & 4u);
       if (!warp_wait(&c.s_full[bs], (n >> 1) & 1, c, ctl)) break;
       tc_fence_after();
-      uint32_t s0[32], s1[32], d0[32], d1[32];
-      tmem_ld32(tmem + lane_off + 64 * bs, s0);
-      tmem_ld32(tmem + lane_off + 64 * bs + 32, s1);
-      tmem_ld32(tmem + lane_off + 128 + 64 * bs, d0);
-      tmem_ld32(tmem + lane_off + 128 + 64 * bs + 32, d1);
+      uint32_t s0[32], d0[32];
+      tmem_ld32(tmem + lane_off + 64 * bs + 32 * half, s0);
+      tmem_ld32(tmem + lane_off + 128 + 64 * bs + 32 * half, d0);
       tmem_ld_wait();
       reg_fence(s0);
-      reg_fence(s1);
       reg_fence(d0);
-      reg_fence(d1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(bs ? s_free_l1 : s_free_l0);
-      uint32_t hid0 = 0u, hid1 = 0u;   // bit j: key j of the tile hidden by the hole rule
+      uint32_t hid = 0u;               // bit j: key kh + j hidden by the hole rule
       if (hole) {
-        const uint4* kc = reinterpret_cast<const uint4*>(codes + k0);
+        const uint4* kc = reinterpret_cast<const uint4*>(codes + kh);
 #pragma unroll
-        for (int q8 = 0; q8 < kKT / 8; ++q8) {
+        for (int q8 = 0; q8 < 4; ++q8) {
           const uint4 v4 = kc[q8];
           const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
           for (int h = 0; h < 8; ++h) {
-            const int j = 8 * q8 + h;
             const uint32_t ck = (wv[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
             const uint32_t hide = ((row_expert && (ck & 1u)) || is_pad(ck)) ? 1u : 0u;
-            if (j < 32) hid0 |= hide << j;
-            else hid1 |= hide << (j - 32);
+            hid |= hide << (8 * q8 + h);
           }
         }
       }
-      uint32_t pk[32], dk[32];
+      uint32_t pk[16], dk[16];
 #pragma unroll
-      for (int j = 0; j < kKT; j += 2) {
-        const float sv0 = __uint_as_float(j < 32 ? s0[j] : s1[j - 32]);
-        const float sv1 = __uint_as_float(j + 1 < 32 ? s0[j + 1] : s1[j - 31]);
-        const float dv0 = __uint_as_float(j < 32 ? d0[j] : d1[j - 32]);
-        const float dv1 = __uint_as_float(j + 1 < 32 ? d0[j + 1] : d1[j - 31]);
-        const uint32_t h0 = j < 32 ? (hid0 >> j) & 1u : (hid1 >> (j - 32)) & 1u;
-        const uint32_t h1 = j + 1 < 32 ? (hid0 >> (j + 1)) & 1u : (hid1 >> (j - 31)) & 1u;
-        const float2 t = ffma2(make_float2(sv0, sv1), make_float2(cs, cs),
-                               make_float2(-lse2, -lse2));
-        const float p0 = (j < e && !h0) ? ex2(t.x) : 0.f;
-        const float p1 = (j + 1 < e && !h1) ? ex2(t.y) : 0.f;
+      for (int j = 0; j < 32; j += 2) {
+        const float2 t = ffma2(make_float2(__uint_as_float(s0[j]), __uint_as_float(s0[j + 1])),
+                               make_float2(cs, cs), make_float2(-lse2, -lse2));
+        const float p0 = (j < e && !((hid >> j) & 1u)) ? ex2(t.x) : 0.f;
+        const float p1 = (j + 1 < e && !((hid >> (j + 1)) & 1u)) ? ex2(t.y) : 0.f;
         pk[j >> 1] = cvt_bf16x2(p0, p1);
-        dk[j >> 1] = cvt_bf16x2(p0 * (dv0 - Dv), p1 * (dv1 - Dv));
+        dk[j >> 1] = cvt_bf16x2(p0 * (__uint_as_float(d0[j]) - Dv),
+                                p1 * (__uint_as_float(d0[j + 1]) - Dv));
       }
-      {
-        uint4 v[8];
+      if (rho0 < rows_per_b) {
+        // Row `lane` of each box: its 16-byte chunk j at j ^ ((lane / 2) % 4).
+        // Rows past the batch element's end are clipped by the tensor map.
+        uint8_t* const line = wstage + lane * 64;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        uint8_t* pbase = reinterpret_cast<uint8_t*>(p.P) + g0 * pitch + k0 * 2;
-        store_rows128(wstage, v, valid, lane, [&](int rr) { return pbase + rr * pitch; });
+        for (int m = 0; m < 2; ++m) {
+          const uint32_t* src = m == 0 ? pk : dk;
+          if (store_pending) {   // the previous box has been read out of the stage
+            if (lane == 0) tma_store_wait_read();
+            __syncwarp();
+          }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
-        uint8_t* dbase = reinterpret_cast<uint8_t*>(p.dS) + g0 * pitch + k0 * 2;
-        store_rows128(wstage, v, valid, lane, [&](int rr) { return dbase + rr * pitch; });
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(line + ((j ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(src[4 * j], src[4 * j + 1], src[4 * j + 2], src[4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d_hint(m == 0 ? &p.map_pw : &p.map_dsw, wstage, kh, rho0, w.b, stream);
+            tma_store_commit();
+          }
+          __syncwarp();
+          store_pending = true;
+        }
       }
       ++n;
       new_pair = walk_next(w, c, pinfo, codes, S, n_kt, n_pairs, tok_per_pair);
     }
+    if (store_pending && lane == 0) tma_store_wait_all();
+    __syncwarp();
   }
 
   __syncwarp();
@@ -1023,13 +1047,13 @@ __global__ void __launch_bounds__(256)
 
 template <typename K>
 cudaError_t launch_cluster_kernel(K kernel, int clusters, int need, const BwdTcParams& p,
-                                  const DevCtl& ctl, cudaStream_t st) {
+                                  const DevCtl& ctl, cudaStream_t st, int threads = kT) {
   static_assert(sizeof(BwdTcParams) <= 4096, "kernel parameters too large");
   const int smem = min(need + 1024, kSmemLimit);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemLimit);
   if (e != cudaSuccess) return e;
-  kernel<<<2 * clusters, kT, smem, st>>>(p, ctl, smem);
+  kernel<<<2 * clusters, threads, smem, st>>>(p, ctl, smem);
   return cudaGetLastError();
 }
 
@@ -1087,7 +1111,7 @@ cudaError_t launch_backward_tc(const BwdTcParams& p, const DevCtl& ctl, cudaStre
   const int units = p.B * n_pairs;
   const int persistent = p.mask_bs == 0 ? min(units, p.clusters) : units;
   e = launch_cluster_kernel(bwd_score_kernel, persistent,
-                            smem_need(ops1(p.ns1), p.S, n_pairs * 4), p, ctl, st);
+                            smem_need(ops1(p.ns1), p.S, n_pairs * 4), p, ctl, st, kT1);
   if (e != cudaSuccess) return e;
   e = launch_cluster_kernel(bwd_dkdv_tc_kernel, p.B * n_sup * p.n_chunks,
                             smem_need(kOps2, p.S, 0), p, ctl, st);

@@ -82,6 +82,8 @@ struct BwdTcParams {
   CUtensorMap map_pT;   // P workspace [B, S*Hq, Skp] as (64, rows, Skp/64, B), box (64, 64, 2, 1)
   CUtensorMap map_dsT;  // dS workspace, box (64, 64, 2, 1)
   CUtensorMap map_ds;   // dS workspace, box (64, 128, 1, 1)
+  CUtensorMap map_pw;   // P workspace as (Skp, S*Hq, B), box (32, 32, 1), 64-byte swizzle
+  CUtensorMap map_dsw;  // dS workspace, the same view (the score pass's stores)
   const uint8_t* ar;
   const int32_t* seg;
   long long mask_bs;
