@@ -127,6 +127,19 @@ __device__ __forceinline__ void tma_store_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with launch_pdl may start
+// while the previous kernel in its stream is still running: it does only
+// work that touches no global memory (barrier set-up, TMEM allocation) before
+// pdl_wait(), which returns once the previous kernel has completed and its
+// writes are visible; pdl_launch_dependents() then lets the next kernel start
+// its own prologue on SMs as they free up.  Without a previous kernel launched
+// this way both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

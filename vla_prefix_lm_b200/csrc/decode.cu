@@ -146,6 +146,10 @@ __global__ void __cluster_dims__(kDecCluster, 1, 1) __launch_bounds__(kDecThread
       tma_load_4d(kt + kTileBytes, &p.map_v, &sm.full[s], 0, 0, 0, b);
     }
   };
+  // Nothing above touched global memory: it may overlap the previous kernel
+  // in the stream, whose results are visible from here on.
+  pdl_wait();
+  pdl_launch_dependents();
   if (t == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[s], 1);
     sm.timed_out = 0;
@@ -371,8 +375,7 @@ cudaError_t launch_decode(const DecodeParams& p, const DevCtl& ctl, cudaStream_t
       decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmemBytes);
   if (attr != cudaSuccess) return attr;
   dim3 grid(kDecCluster, (unsigned)p.B);
-  decode_kernel<<<grid, kDecThreads, kDecSmemBytes, st>>>(p, ctl);
-  return cudaGetLastError();
+  return launch_pdl(decode_kernel, grid, dim3(kDecThreads), kDecSmemBytes, st, p, ctl);
 }
 
 }  // namespace piattn

@@ -8,6 +8,25 @@
 
 namespace piattn {
 
+// Launches `kernel` so that it may begin while the previous kernel in `st` is
+// still running (programmatic stream serialization): the kernel must call
+// pdl_wait() before its first global memory access (common.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // Inputs of the fp32 SIMT path (both modes).  Prefill: k/v hold the S keys,
 // kc/vc are null and P = 0.  Suffix: k/v hold the Sq suffix keys and kc/vc the
 // P cached prefix keys.

@@ -72,6 +72,8 @@ __global__ void __launch_bounds__(kRopeThreads)
   __shared__ double s_inv[128];                 // base^(-2i/d), i < d/2 <= 128
   __shared__ int s_count[kRopeThreads / 32];
   __shared__ uint32_t s_bits;
+  pdl_wait();                                   // q and k may come from the kernel before
+  pdl_launch_dependents();
   const int b = blockIdx.y;
   const int t0 = blockIdx.x * tok;
   const int nt = min(tok, S - t0);
@@ -161,6 +163,8 @@ __global__ void __launch_bounds__(kRopeThreads)
 template <typename T>
 __global__ void __launch_bounds__(256)
     euler_kernel(float* __restrict__ x, const T* __restrict__ v, float dt, long long n) {
+  pdl_wait();                                   // v comes from the attention pass before
+  pdl_launch_dependents();
   const long long n4 = n / 4;
   const long long stride = (long long)gridDim.x * blockDim.x;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
@@ -207,16 +211,15 @@ cudaError_t launch_rope(const RopeParams& p, const DevCtl& ctl, cudaStream_t st)
   const int tok = rope_tokens_per_cta(p.d, p.f32);
   dim3 grid((p.S + tok - 1) / tok, p.B);
   const double log2_base = log2((double)p.base);
-  if (p.f32) {
-    rope_kernel<float><<<grid, kRopeThreads, 0, st>>>(
-        static_cast<float*>(p.q), static_cast<float*>(p.k), p.tmask, p.tmask_bs, p.pmask,
-        p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, tok, log2_base, p.pos_out);
-  } else {
-    rope_kernel<__nv_bfloat16><<<grid, kRopeThreads, 0, st>>>(
-        static_cast<__nv_bfloat16*>(p.q), static_cast<__nv_bfloat16*>(p.k), p.tmask, p.tmask_bs,
-        p.pmask, p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, tok, log2_base, p.pos_out);
-  }
-  return cudaGetLastError();
+  if (p.f32)
+    return launch_pdl(rope_kernel<float>, grid, dim3(kRopeThreads), 0, st,
+                      static_cast<float*>(p.q), static_cast<float*>(p.k), p.tmask, p.tmask_bs,
+                      p.pmask, p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, tok, log2_base,
+                      p.pos_out);
+  return launch_pdl(rope_kernel<__nv_bfloat16>, grid, dim3(kRopeThreads), 0, st,
+                    static_cast<__nv_bfloat16*>(p.q), static_cast<__nv_bfloat16*>(p.k), p.tmask,
+                    p.tmask_bs, p.pmask, p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, tok, log2_base,
+                    p.pos_out);
 }
 
 cudaError_t launch_euler(float* x, const void* v, bool v_f32, float dt, long long n,
@@ -225,13 +228,11 @@ cudaError_t launch_euler(float* x, const void* v, bool v_f32, float dt, long lon
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long blocks_needed = (n / 4 + 255) / 256 + 1;
   const int grid = (int)std::min<long long>(blocks_needed, (long long)sms * 8);
-  if (v_f32) {
-    euler_kernel<float><<<grid, 256, 0, st>>>(x, static_cast<const float*>(v), dt, n);
-  } else {
-    euler_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(x, static_cast<const __nv_bfloat16*>(v),
-                                                      dt, n);
-  }
-  return cudaGetLastError();
+  if (v_f32)
+    return launch_pdl(euler_kernel<float>, dim3(grid), dim3(256), 0, st, x,
+                      static_cast<const float*>(v), dt, n);
+  return launch_pdl(euler_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, x,
+                    static_cast<const __nv_bfloat16*>(v), dt, n);
 }
 
 }  // namespace piattn

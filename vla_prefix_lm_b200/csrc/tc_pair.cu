@@ -291,6 +291,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   // Both CTAs see the same base offset, so both leave here or neither does.
   if ((int)(smem - smem_raw) + layout_bytes<L>(p.Sq) > smem_bytes || p.Sq > L::kMaxTok) {
+    pdl_wait();
     if (threadIdx.x == 0) record_status(ctl, kStatusUnsupported);
     return;
   }
@@ -314,14 +315,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // unmasked suffix pass pays nothing for it.
   constexpr bool cache_masked = kSuffix && kCacheMask;
 
-  // The mask bytes are the first global reads: issue them before anything
-  // else so their latency hides behind the barrier and TMEM set-up.  With a
-  // batch-shared mask (the persistent case) every unit uses row 0; otherwise
-  // this cluster runs exactly one unit and scans that unit's batch row.
+  // With a batch-shared mask (the persistent case) every unit uses row 0;
+  // otherwise this cluster runs exactly one unit and scans that unit's batch
+  // row.
   const int b_codes = (cluster / p.n_splits) / n_pairs;
   const uint8_t* ar_b = p.ar + (long long)b_codes * p.mask_bs;
   const int32_t* seg_b = p.seg ? p.seg + (long long)b_codes * p.mask_bs : nullptr;
-  const Flags32 flags0 = load_flags32(ar_b, seg_b, n_key_tok, (int)threadIdx.x * 32);
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
@@ -357,6 +356,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   // Both CTAs' barriers must exist before either side signals the other.
   cluster_sync();
+  if (warp == 1) {
+    tmem_alloc_pair(&sm.tmem_base, 512);
+    tmem_relinquish_pair();
+  }
+  // Everything above touches no global memory, so it may overlap the previous
+  // kernel in the stream; from here on its results are visible.
+  pdl_wait();
+  pdl_launch_dependents();
+  // The mask bytes are the first global reads; their latency hides behind
+  // the early TMA issue below.
+  const Flags32 flags0 = load_flags32(ar_b, seg_b, n_key_tok, (int)threadIdx.x * 32);
   // With a single split every unit visits at least one key tile (a valid
   // query sees its own token; a unit of padding rows gets one masked tile),
   // so the first unit's Q can load during the mask scan.
@@ -389,10 +399,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                      b0);
     tma_load_4d_pair(vring + kVItem, mv, mapa_shared(smem_u32(&sm.v_full[1]), 0), 0, 64,
                      2 * (int)rank, b0);
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(&sm.tmem_base, 512);
-    tmem_relinquish_pair();
   }
   build_codes_x32<kThreads>(ar_b, seg_b, n_key_tok, pad_tokens(n_key_tok), codes, sm.scan,
                             flags0, TileSums{sm.tile_cs_first, sm.tile_cs_last, sm.tile_fast});
@@ -927,6 +933,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 __global__ void __launch_bounds__(256)
     combine_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ out, int n_splits,
                    long long n_rows) {
+  pdl_wait();                  // the partials come from the kernel before
+  pdl_launch_dependents();
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= n_rows) return;
@@ -970,8 +978,8 @@ cudaError_t launch_pair(const TcParams& p, const DevCtl& ctl, dim3 grid, cudaStr
       kSmemLimit);
   if (attr_err != cudaSuccess) return attr_err;
   const int smem = pair_smem_bytes<L>(p.Sq);
-  tc_pair_kernel<kSuffix, kCacheMask, L><<<grid, kThreads, smem, st>>>(p, ctl, smem);
-  return cudaGetLastError();
+  return launch_pdl(tc_pair_kernel<kSuffix, kCacheMask, L>, grid, dim3(kThreads), smem, st, p,
+                    ctl, smem);
 }
 
 template <class L>
@@ -1066,15 +1074,15 @@ cudaError_t launch_tc_pair(const TcParams& p, bool suffix_mode, const DevCtl& ct
                           : launch_mode<LayoutLong>(p, suffix_mode, ctl, grid, st);
   if (e != cudaSuccess || p.n_splits <= 1) return e;
   const long long n_rows = (long long)p.B * rows;
-  combine_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, st>>>(
-      p.ws, reinterpret_cast<__nv_bfloat16*>(p.out_ptr), p.n_splits, n_rows);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3((unsigned)((n_rows + 7) / 8)), dim3(256), 0, st,
+                    static_cast<const float*>(p.ws), reinterpret_cast<__nv_bfloat16*>(p.out_ptr),
+                    p.n_splits, n_rows);
 }
 
 cudaError_t launch_combine(const float* ws, __nv_bfloat16* out, int n_splits, long long n_rows,
                            cudaStream_t st) {
-  combine_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, st>>>(ws, out, n_splits, n_rows);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3((unsigned)((n_rows + 7) / 8)), dim3(256), 0, st, ws, out,
+                    n_splits, n_rows);
 }
 
 int tc_suffix_splits(int B, int Sq, int P, int Hq) {
