@@ -229,6 +229,7 @@ __device__ __forceinline__ uint8_t* bwd_smem(uint8_t* raw, int need, int smem_by
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(raw) + 1023) & ~static_cast<uintptr_t>(1023));
   if ((int)(smem - raw) + need > smem_bytes || S > kMaxTokens) {
+    pdl_wait();
     if (threadIdx.x == 0) record_status(ctl, kStatusUnsupported);
     return nullptr;
   }
@@ -306,7 +307,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
 
   const uint8_t* ar_b = p.ar + (long long)b_mask * p.mask_bs;
   const int32_t* seg_b = p.seg ? p.seg + (long long)b_mask * p.mask_bs : nullptr;
-  const Flags32 flags0 = load_flags32(ar_b, seg_b, S, (int)threadIdx.x * 32);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ns; ++s) {
@@ -334,6 +334,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
     tmem_alloc_pair(&c.tmem_base, 256);
     tmem_relinquish_pair();
   }
+  // Nothing above touched global memory (it may overlap the previous kernel);
+  // its results are visible from here on.
+  pdl_wait();
+  pdl_launch_dependents();
+  const Flags32 flags0 = load_flags32(ar_b, seg_b, S, (int)threadIdx.x * 32);
   build_codes_x32<kT1>(ar_b, seg_b, S, pad128(S), codes, c.scan, flags0,
                       TileSums{c.cs_first, c.cs_last, c.flags});
   // Per row tile: its visited key-tile count, and bit 30 if all its tokens
@@ -655,7 +660,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
 
   const uint8_t* ar_b = p.ar + (long long)b * p.mask_bs;
   const int32_t* seg_b = p.seg ? p.seg + (long long)b * p.mask_bs : nullptr;
-  const Flags32 flags0 = load_flags32(ar_b, seg_b, S, (int)threadIdx.x * 32);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNS2; ++s) {
@@ -676,6 +680,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     tmem_alloc_pair(&c.tmem_base, 512);
     tmem_relinquish_pair();
   }
+  // Nothing above touched global memory (it may overlap the previous kernel);
+  // its results are visible from here on.
+  pdl_wait();
+  pdl_launch_dependents();
+  const Flags32 flags0 = load_flags32(ar_b, seg_b, S, (int)threadIdx.x * 32);
   build_codes_x32<kT>(ar_b, seg_b, S, pad128(S), codes, c.scan, flags0,
                       TileSums{c.cs_first, c.cs_last, c.flags});
   tc_fence_before();
@@ -842,7 +851,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
 
   const uint8_t* ar_b = p.ar + (long long)b_mask * p.mask_bs;
   const int32_t* seg_b = p.seg ? p.seg + (long long)b_mask * p.mask_bs : nullptr;
-  const Flags32 flags0 = load_flags32(ar_b, seg_b, S, (int)threadIdx.x * 32);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNS3; ++s) {
@@ -864,6 +872,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     tmem_alloc_pair(&c.tmem_base, 512);
     tmem_relinquish_pair();
   }
+  // Nothing above touched global memory (it may overlap the previous kernel);
+  // its results are visible from here on.
+  pdl_wait();
+  pdl_launch_dependents();
+  const Flags32 flags0 = load_flags32(ar_b, seg_b, S, (int)threadIdx.x * 32);
   build_codes_x32<kT>(ar_b, seg_b, S, pad128(S), codes, c.scan, flags0,
                       TileSums{c.cs_first, c.cs_last, c.flags});
   tc_fence_before();
@@ -999,6 +1012,8 @@ __global__ void __launch_bounds__(256)
     bwd_rowdot_kernel(const __nv_bfloat16* __restrict__ out,
                       const __nv_bfloat16* __restrict__ dout, float* __restrict__ D,
                       long long n_rows) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
   for (long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -1025,6 +1040,8 @@ __global__ void __launch_bounds__(256)
 __global__ void __launch_bounds__(256)
     bwd_chunk_sum_kernel(const float* __restrict__ part, float* __restrict__ dk,
                          float* __restrict__ dv, int n_chunks, int B, int S, int kpad) {
+  pdl_wait();                 // the partials come from the dK/dV pass before
+  pdl_launch_dependents();
   const long long n4 = (long long)B * S * (kD / 4);
   const long long stride = (long long)gridDim.x * blockDim.x;
   const long long per_chunk = (long long)B * kpad * kD;
@@ -1053,8 +1070,7 @@ cudaError_t launch_cluster_kernel(K kernel, int clusters, int need, const BwdTcP
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemLimit);
   if (e != cudaSuccess) return e;
-  kernel<<<2 * clusters, threads, smem, st>>>(p, ctl, smem);
-  return cudaGetLastError();
+  return launch_pdl(kernel, dim3(2 * clusters), dim3(threads), smem, st, p, ctl, smem);
 }
 
 }  // namespace
@@ -1101,10 +1117,10 @@ BwdTcPlan bwd_tc_plan(int B, int S, int Hq, int sms) {
 cudaError_t launch_backward_tc(const BwdTcParams& p, const DevCtl& ctl, cudaStream_t st) {
   const long long rows = (long long)p.B * p.S * p.Hq;
   const int rd_blocks = (int)min((rows + 7) / 8, (long long)148 * 16);
-  bwd_rowdot_kernel<<<rd_blocks, 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(p.out), static_cast<const __nv_bfloat16*>(p.dout),
-      const_cast<float*>(p.D), rows);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(bwd_rowdot_kernel, dim3(rd_blocks), dim3(256), 0, st,
+                             static_cast<const __nv_bfloat16*>(p.out),
+                             static_cast<const __nv_bfloat16*>(p.dout), const_cast<float*>(p.D),
+                             rows);
   if (e != cudaSuccess) return e;
   const int n_pairs = (p.S * p.Hq + 2 * kRows - 1) / (2 * kRows);
   const int n_sup = (p.S + kSup - 1) / kSup;
@@ -1119,9 +1135,9 @@ cudaError_t launch_backward_tc(const BwdTcParams& p, const DevCtl& ctl, cudaStre
   if (p.n_chunks > 1) {
     const long long n4 = (long long)p.B * p.S * (kD / 4);
     const int blocks = (int)min((n4 + 255) / 256, (long long)148 * 8);
-    bwd_chunk_sum_kernel<<<blocks, 256, 0, st>>>(p.part, p.dk, p.dv, p.n_chunks, p.B, p.S,
-                                                 n_sup * kSup);
-    e = cudaGetLastError();
+    e = launch_pdl(bwd_chunk_sum_kernel, dim3(blocks), dim3(256), 0, st,
+                   static_cast<const float*>(p.part), p.dk, p.dv, p.n_chunks, p.B, p.S,
+                   n_sup * kSup);
     if (e != cudaSuccess) return e;
   }
   return launch_cluster_kernel(bwd_dq_tc_kernel, persistent, smem_need(kOps3, p.S, 0), p, ctl,
