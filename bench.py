@@ -161,6 +161,17 @@ def gpu_id(dev) -> str:
 # ------------------------------------------------------------------ our arm
 
 
+def _prefill_ws(q, k, ar):
+    """Scratch that lets the prefill split its last round of query tiles over
+    idle SM pairs (None if this geometry takes none)."""
+    import torch
+
+    from vla_prefix_lm_b200 import binding
+
+    n = binding.pi_attn_prefill_workspace_bytes(q, k, ar)
+    return torch.empty(n, dtype=torch.uint8, device=q.device) if n else None
+
+
 def _mmdit_sets(w, dev, n, seed0):
     """``n`` fresh MM-DiT input sets (q, k, v, ar) drawn on the device."""
     import torch
@@ -231,9 +242,11 @@ def run_ours(args, rank, ws, local):
     outs = [torch.empty_like(s_[0]) for s_ in sets]
     set_bytes = sum(t.nbytes for t in sets[0][:3]) + outs[0].nbytes
 
+    pws = _prefill_ws(sets[0][0], sets[0][1], sets[0][3])
+
     def workload_calls():
         for i, (q, k, v, ar) in enumerate(sets):
-            binding.pi_attn_prefill(q, k, v, ar, out=outs[i], stream=stream)
+            binding.pi_attn_prefill(q, k, v, ar, out=outs[i], stream=stream, workspace=pws)
 
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 1)):
@@ -354,6 +367,7 @@ def e2e_mmdit(args, w, dev, stream, rank, ws, dev_sets):
     hout = [torch.empty(dev_sets[0][0].shape, dtype=torch.bfloat16, pin_memory=True)
             for _ in range(2)]
     din = [tuple(torch.empty_like(t) for t in dev_sets[0]) for _ in range(2)]
+    pws = _prefill_ws(dev_sets[0][0], dev_sets[0][1], dev_sets[0][3])
     dout = [torch.empty_like(dev_sets[0][0]) for _ in range(2)]
     h2d_bytes = sum(t.nbytes for t in host[0])
     d2h_bytes = hout[0].nbytes
@@ -376,7 +390,7 @@ def e2e_mmdit(args, w, dev, stream, rank, ws, dev_sets):
                 stream.wait_event(ev_out[j])           # output slot j copied out
             if compute:
                 q, k, v, ar = din[j]
-                binding.pi_attn_prefill(q, k, v, ar, out=dout[j], stream=stream)
+                binding.pi_attn_prefill(q, k, v, ar, out=dout[j], stream=stream, workspace=pws)
             ev_done[j].record(stream)
             s_out.wait_event(ev_done[j])
             with torch.cuda.stream(s_out):
@@ -435,11 +449,12 @@ def prefill_config(cfg, dev, stream, rank, n_sets, reps):
         ins.append(tuple(W.device_draw((w.B, w.Sq, h, w.d), s + j, w.d, w.dtype, dev)
                          for j, h in enumerate((w.Hq, w.Hkv, w.Hkv))))
     outs = [torch.empty_like(t[0]) for t in ins]
+    pws = _prefill_ws(ins[0][0], ins[0][1], ar)
 
     def call(i):
         q, k, v = ins[i % n_sets]
         binding.pi_attn_prefill(q, k, v, ar, segment_ids=seg, out=outs[i % n_sets],
-                                softmax_scale=w.scale, stream=stream)
+                                softmax_scale=w.scale, stream=stream, workspace=pws)
 
     with torch.cuda.stream(stream):
         for i in range(max(3, n_sets)):
@@ -969,9 +984,11 @@ def run_case(args):
         ar = torch.tensor(w.ar, dtype=torch.uint8, device=dev)
         seg = None if w.seg is None else torch.tensor(w.seg, dtype=torch.int32, device=dev)
         out = torch.empty_like(q)
+        pws = _prefill_ws(q, k, ar)
 
         def call():
-            binding.pi_attn_prefill(q, k, v, ar, segment_ids=seg, out=out, stream=stream)
+            binding.pi_attn_prefill(q, k, v, ar, segment_ids=seg, out=out, stream=stream,
+                                    workspace=pws)
     else:
         if name == "pi0_suffix_step":
             w = W.workload(3)

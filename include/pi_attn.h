@@ -144,6 +144,31 @@ int pi_attn_prefill(const pi_attn_desc* desc, const void* q, const void* k, cons
                     pi_stream_t stream);
 
 /*
+ * pi_attn_prefill_ws -- pi_attn_prefill with scratch for a split last round.
+ * The bf16 kernel hands whole 256-row query tiles to the SM pairs in rounds;
+ * when the last round would leave at least half the pairs idle (MM-DiT: 532
+ * tiles on 74 pairs leave 14 for the 8th round), the full rounds run whole
+ * and each remaining tile is split over several pairs by key tiles (pieces
+ * of at least 6 of the S / 128 key tiles, so short sequences stay whole), its
+ * fp32 partials merged by a second kernel (log-sum-exp rule).  Same results
+ * up to the rounding order of fp32 sums.
+ *   desc ... lse   as pi_attn_prefill
+ *   workspace  device scratch of pi_attn_prefill_workspace_bytes(desc) bytes,
+ *              16-byte aligned, caller-owned, contents ignored; one call at a
+ *              time per workspace.  NULL: as pi_attn_prefill.
+ *   ws_bytes   its size
+ * Only bf16 with a batch-shared mask (mask_batch_stride == 0) uses it (the
+ * size is 0 otherwise).  The size depends on the device's SM count.
+ * Errors: as pi_attn_prefill, plus PI_ERR_ARG for a workspace smaller than
+ * required and PI_ERR_ALIGN for a misaligned one, before anything is
+ * enqueued.
+ */
+size_t pi_attn_prefill_workspace_bytes(const pi_attn_desc* desc);
+int pi_attn_prefill_ws(const pi_attn_desc* desc, const void* q, const void* k, const void* v,
+                       const uint8_t* ar_mask, const int32_t* segment_ids, void* out, float* lse,
+                       void* workspace, size_t ws_bytes, pi_stream_t stream);
+
+/*
  * pi_attn_prefill_backward -- gradient of pi_attn_prefill with respect to q,
  * k and v, for training.
  * Source: "VLA 代码精读 - OpenPI & StarVLA", 1.5 Pi0.compute_loss runs the

@@ -40,6 +40,8 @@ EXPORTED = (
     "pi_attn_prefill_backward_workspace_bytes",
     "pi_attn_suffix_noalloc_capacity",
     "pi_attn_debug_tiles",
+    "pi_attn_prefill_ws",
+    "pi_attn_prefill_workspace_bytes",
 )
 
 
@@ -93,6 +95,10 @@ def lib() -> ctypes.CDLL:
         dp = ctypes.POINTER(PiAttnDesc)
         L.pi_attn_prefill.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.pi_attn_prefill.restype = i32
+        L.pi_attn_prefill_ws.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.pi_attn_prefill_ws.restype = i32
+        L.pi_attn_prefill_workspace_bytes.argtypes = [dp]
+        L.pi_attn_prefill_workspace_bytes.restype = sz
         L.pi_attn_suffix.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.pi_attn_suffix.restype = i32
         L.pi_attn_suffix_workspace_bytes.argtypes = [dp]
@@ -172,10 +178,21 @@ def _dtype_code(t):
     raise ValueError(f"unsupported dtype {t.dtype}")
 
 
+def pi_attn_prefill_workspace_bytes(q, k, ar_mask, softmax_scale=1.0):
+    """Bytes of the scratch pi_attn_prefill takes as ``workspace`` (0: this
+    geometry does not use one)."""
+    B, S, Hq, d = q.shape
+    desc = PiAttnDesc(B, S, 0, Hq, k.shape[2], d, _dtype_code(q), float(softmax_scale),
+                      _mask_stride(ar_mask, B, S))
+    return int(lib().pi_attn_prefill_workspace_bytes(ctypes.byref(desc)))
+
+
 def pi_attn_prefill(q, k, v, ar_mask, segment_ids=None, out=None, lse=None,
-                    softmax_scale=1.0, stream=None):
+                    softmax_scale=1.0, stream=None, workspace=None):
     """Joint prefill.  q [B,S,Hq,d]; k, v [B,S,Hkv,d]; ar_mask uint8 [S] or [B,S];
-    segment_ids int32 like ar_mask or None.  Returns ``out`` (allocated if None)."""
+    segment_ids int32 like ar_mask or None.  Returns ``out`` (allocated if None).
+    ``workspace``: a CUDA byte tensor of pi_attn_prefill_workspace_bytes bytes
+    (lets a sparse last round of query tiles split over idle SM pairs), or None."""
     _need(q, "q", dims=4)
     _need(k, "k", q.dtype, 4)
     _need(v, "v", q.dtype, 4)
@@ -194,9 +211,16 @@ def pi_attn_prefill(q, k, v, ar_mask, segment_ids=None, out=None, lse=None,
     if lse is not None:
         _need(lse, "lse", torch.float32)
     desc = PiAttnDesc(B, S, 0, Hq, k.shape[2], d, _dtype_code(q), float(softmax_scale), mbs)
-    rc = lib().pi_attn_prefill(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(ar_mask),
-                               _ptr(segment_ids), _ptr(out), _ptr(lse),
-                               ctypes.c_void_p(_stream(stream)))
+    if workspace is None:
+        rc = lib().pi_attn_prefill(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v),
+                                   _ptr(ar_mask), _ptr(segment_ids), _ptr(out), _ptr(lse),
+                                   ctypes.c_void_p(_stream(stream)))
+    else:
+        _need(workspace, "workspace", torch.uint8)
+        rc = lib().pi_attn_prefill_ws(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v),
+                                      _ptr(ar_mask), _ptr(segment_ids), _ptr(out), _ptr(lse),
+                                      _ptr(workspace), workspace.numel(),
+                                      ctypes.c_void_p(_stream(stream)))
     if rc != PI_OK:
         raise PiAttnError(rc, "pi_attn_prefill")
     return out

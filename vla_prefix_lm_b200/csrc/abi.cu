@@ -167,11 +167,20 @@ int check_backward_desc(const pi_attn_desc* d) {
 
 extern "C" {
 
-int pi_attn_prefill(const pi_attn_desc* d, const void* q, const void* k, const void* v,
-                    const uint8_t* ar_mask, const int32_t* segment_ids, void* out, float* lse,
-                    pi_stream_t stream) {
+namespace {
+bool tail_split_applies(const pi_attn_desc* d) {
+  return d->dtype == PI_BF16 && d->mask_batch_stride == 0;
+}
+
+int prefill_impl(const pi_attn_desc* d, const void* q, const void* k, const void* v,
+                 const uint8_t* ar_mask, const int32_t* segment_ids, void* out, float* lse,
+                 void* workspace, size_t ws_bytes, pi_stream_t stream) {
   int rc = check_desc(d, false);
   if (rc != PI_OK) return rc;
+  if (workspace != nullptr && tail_split_applies(d)) {
+    if (!aligned16(workspace)) return PI_ERR_ALIGN;
+    if (ws_bytes < tc_prefill_tail_bytes()) return PI_ERR_ARG;
+  }
   if (d->B == 0 || d->Sq == 0) return PI_OK;
   if (!q || !k || !v || !ar_mask || !out) return PI_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return PI_ERR_ALIGN;
@@ -208,13 +217,31 @@ int pi_attn_prefill(const pi_attn_desc* d, const void* q, const void* k, const v
   p.seg = segment_ids;
   p.mask_bs = d->mask_batch_stride;
   p.lse = lse;
-  p.ws = nullptr;
+  p.ws = tail_split_applies(d) ? static_cast<float*>(workspace) : nullptr;
   p.out_ptr = out;
   p.B = d->B; p.Sq = d->Sq; p.P = 0; p.Hq = d->Hq;
   p.n_splits = 1;
   p.scale = d->softmax_scale;
   p.scale_log2 = d->softmax_scale * 1.4426950408889634f;
   return launched(launch_tc_pair(p, false, ctl, st));
+}
+}  // namespace
+
+int pi_attn_prefill(const pi_attn_desc* d, const void* q, const void* k, const void* v,
+                    const uint8_t* ar_mask, const int32_t* segment_ids, void* out, float* lse,
+                    pi_stream_t stream) {
+  return prefill_impl(d, q, k, v, ar_mask, segment_ids, out, lse, nullptr, 0, stream);
+}
+
+size_t pi_attn_prefill_workspace_bytes(const pi_attn_desc* d) {
+  if (check_desc(d, false) != PI_OK || !tail_split_applies(d)) return 0;
+  return tc_prefill_tail_bytes();
+}
+
+int pi_attn_prefill_ws(const pi_attn_desc* d, const void* q, const void* k, const void* v,
+                       const uint8_t* ar_mask, const int32_t* segment_ids, void* out, float* lse,
+                       void* workspace, size_t ws_bytes, pi_stream_t stream) {
+  return prefill_impl(d, q, k, v, ar_mask, segment_ids, out, lse, workspace, ws_bytes, stream);
 }
 
 size_t pi_attn_suffix_workspace_bytes(const pi_attn_desc* d) {

@@ -160,6 +160,11 @@ struct TcParams {
   void* out_ptr;        // bf16 output rows (written by the combine kernel under split-K)
   int B, Sq, P, Hq;
   int n_splits;         // KV splits per query tile (1 = write final output)
+  // Prefill tail split: units [0, n_main) run whole (full rounds of the
+  // clusters); each later unit runs as tail_splits pieces whose fp32 partials
+  // go to ws ([piece][256 rows] O, then (m, l)) and tail_combine_kernel merges.
+  int n_main;           // B * query tiles when there is no tail split
+  int tail_splits;      // 1: no tail split
   float scale_log2;     // softmax_scale * log2(e)
   float scale;          // softmax_scale
 };
@@ -171,6 +176,10 @@ cudaError_t launch_tc_pair(const TcParams& p, bool suffix_mode, const DevCtl& ct
                            cudaStream_t st);
 
 size_t tc_suffix_workspace_bytes(int B, int Sq, int P, int Hq);
+
+// Scratch of the prefill tail split on the current device: at most one round
+// of pieces (one per SM pair) of 256 rows, fp32 O and (m, l).
+size_t tc_prefill_tail_bytes();
 int tc_suffix_splits(int B, int Sq, int P, int Hq);
 
 // Merges split partials (unnormalised O [splits][rows][256] fp32, then (m, l)

@@ -199,6 +199,7 @@ struct Unit {
   int b, pair, split;
   int tq0, tq1;        // first / last valid query token of the pair tile
   int it_begin, n_it;  // this split's slice of the visited key tiles
+  int piece;           // prefill tail split: the piece's index, else -1
 };
 
 // Warp-collective: classifies every key tile for the unit's query tokens
@@ -258,8 +259,19 @@ __device__ __noinline__ Unit make_unit(int u, const TcParams& p, int n_pairs, in
                                           const SmemT& sm, const uint16_t* codes, uint16_t* list,
                                           int lane) {
   Unit x;
-  x.split = u % p.n_splits;
-  const int t = u / p.n_splits;
+  int splits = p.n_splits, t;
+  if (!kSuffix && u >= p.n_main) {
+    // A tail unit: piece u - n_main of the units after the full rounds.
+    const int v = u - p.n_main;
+    splits = p.tail_splits;
+    x.split = v % splits;
+    t = p.n_main + v / splits;
+    x.piece = v;
+  } else {
+    x.split = u % p.n_splits;
+    t = u / p.n_splits;
+    x.piece = -1;
+  }
   x.pair = t % n_pairs;
   x.b = t / n_pairs;
   const int tok_per_pair = 2 * kBM / p.Hq;
@@ -275,7 +287,7 @@ __device__ __noinline__ Unit make_unit(int u, const TcParams& p, int n_pairs, in
     n_list = 1;
   }
   const int n_total = n_cache + n_list;
-  const int per = (n_total + p.n_splits - 1) / p.n_splits;
+  const int per = (n_total + splits - 1) / splits;
   x.it_begin = min(x.split * per, n_total);
   x.n_it = min(x.it_begin + per, n_total) - x.it_begin;
   return x;
@@ -307,7 +319,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows_per_b = p.Sq * p.Hq;
   const int n_pairs = (rows_per_b + 2 * kBM - 1) / (2 * kBM);
-  const int n_units = p.B * n_pairs * p.n_splits;
+  // Prefill: units [0, n_main) whole, then tail_splits pieces of each later one.
+  const int n_units = kSuffix ? p.B * n_pairs * p.n_splits
+                              : p.n_main + (p.B * n_pairs - p.n_main) * p.tail_splits;
+  const int n_tail_pieces = n_units - p.n_main;
   const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
   const int n_key_tok = p.Sq;
   const int n_cache = kSuffix ? (p.P + kBN - 1) / kBN : 0;
@@ -634,12 +649,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const Unit x = nx;
       const int row0 = x.pair * 2 * kBM + (int)rank * kBM;
       const bool row_valid = row0 + r < rows_per_b;
-      const long long slot = ((long long)x.split * p.B + x.b) * rows_per_b + row0 + r;
+      // Where a partial result of this row goes: split-K over the cache
+      // (suffix: [split][batch][row]) or a prefill tail piece ([piece][256
+      // rows]); unnormalised O rows, then (m, l) pairs.
+      float* po = nullptr;
+      float* pml = nullptr;
+      if (p.n_splits > 1) {
+        const long long slot = ((long long)x.split * p.B + x.b) * rows_per_b + row0 + r;
+        po = p.ws + slot * kD;
+        pml = p.ws + (long long)p.n_splits * p.B * rows_per_b * kD + slot * 2;
+      } else if (x.piece >= 0) {
+        const long long ts = (long long)x.piece * (2 * kBM) + (int)rank * kBM + r;
+        po = p.ws + ts * kD;
+        pml = p.ws + (long long)n_tail_pieces * (2 * kBM) * kD + ts * 2;
+      }
       if (x.n_it == 0) {
-        if (p.n_splits > 1 && row_valid) {
-          float* wml = p.ws + (long long)p.n_splits * p.B * rows_per_b * kD + slot * 2;
-          wml[0] = -INFINITY;
-          wml[1] = 0.f;
+        if (pml != nullptr && row_valid) {
+          pml[0] = -INFINITY;
+          pml[1] = 0.f;
         }
         if (unit + n_clusters < n_units)
           nx = make_unit<kSuffix>(unit + n_clusters, p, n_pairs, n_cache, sm, codes, list, lane);
@@ -826,7 +853,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!warp_wait(&sm.o_done, g_last & 1, sm, ctl)) { ok = false; break; }
       tc_fence_after();
       const long long grow = (long long)x.b * rows_per_b + row0 + r;
-      if (p.n_splits == 1) {
+      if (po == nullptr) {
         // A row that saw no key (a padding query) writes 0, lse = -inf.
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
         // The P buffer is free once the last PV has finished: each warp stages
@@ -882,10 +909,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!kSuffix && p.lse && row_valid)
           p.lse[grow] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
       } else {
-        // Split-K partial: unnormalised O and (m, l) for the combine kernel.
+        // Split partial: unnormalised O and (m, l) for a combine kernel.
         // tcgen05.ld is warp-collective (.sync.aligned): every lane loads,
         // only lanes holding a real row store.
-        float* wo = p.ws + slot * kD;
+        float* wo = po;
 #pragma unroll 1
         for (int cc = 0; cc < kD / 32; ++cc) {
           uint32_t o[32];
@@ -904,9 +931,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(o_free_l);
         if (row_valid) {
-          float* wml = p.ws + (long long)p.n_splits * p.B * rows_per_b * kD + slot * 2;
-          wml[0] = m_run;
-          wml[1] = l_run;
+          pml[0] = m_run;
+          pml[1] = l_run;
         }
       }
     }
@@ -961,6 +987,58 @@ __global__ void __launch_bounds__(256)
   pk.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
   pk.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
   *reinterpret_cast<uint4*>(out + row * kD + lane * 8) = pk;
+}
+
+// Merges the prefill tail pieces: for each row of a tail unit (units from
+// n_main on, each split into `splits` pieces over its key tiles), out = sum_k
+// 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k with M = max_k m_k (the log-sum-exp
+// rule), and lse.  One warp per row, 8 columns per lane; pieces with l = 0
+// (no visible key) drop out; a row with none writes 0 and lse = -inf.
+__global__ void __launch_bounds__(256)
+    tail_combine_kernel(const float* __restrict__ ws, __nv_bfloat16* __restrict__ out,
+                        float* __restrict__ lse, int n_main, int n_tail_units, int splits,
+                        int n_pairs, int rows_per_b) {
+  pdl_wait();                  // the partials come from the kernel before
+  pdl_launch_dependents();
+  const long long tr = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);   // tail row
+  const int lane = threadIdx.x & 31;
+  if (tr >= (long long)n_tail_units * 2 * kBM) return;
+  const int unit = n_main + (int)(tr / (2 * kBM));
+  const int rr = (int)(tr % (2 * kBM));                // row of the 256-row tile
+  const int b = unit / n_pairs, pair = unit % n_pairs;
+  const int row = pair * 2 * kBM + rr;
+  if (row >= rows_per_b) return;
+  const long long n_rows_ws = (long long)n_tail_units * splits * 2 * kBM;
+  const long long ts0 = (long long)(unit - n_main) * splits * 2 * kBM + rr;  // piece 0's row
+  const float2* ml = reinterpret_cast<const float2*>(ws + n_rows_ws * kD);
+  float M = -INFINITY;
+  for (int k = 0; k < splits; ++k) {
+    const float2 v = ml[ts0 + (long long)k * 2 * kBM];
+    if (v.y > 0.f) M = fmaxf(M, v.x);
+  }
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  float L = 0.f;
+  for (int k = 0; k < splits; ++k) {
+    const long long ts = ts0 + (long long)k * 2 * kBM;
+    const float2 v = ml[ts];
+    if (v.y <= 0.f) continue;
+    const float w = ex2(v.x - M);
+    L += w * v.y;
+    const float4* src = reinterpret_cast<const float4*>(ws + ts * kD + lane * 8);
+    const float4 a = src[0], c = src[1];
+    acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
+    acc[4] += w * c.x; acc[5] += w * c.y; acc[6] += w * c.z; acc[7] += w * c.w;
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  uint4 pk;
+  pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  pk.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  pk.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  const long long grow = (long long)b * rows_per_b + row;
+  *reinterpret_cast<uint4*>(out + grow * kD + lane * 8) = pk;
+  if (lse != nullptr && lane == 0)
+    lse[grow] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
 // Dynamic shared memory for S code tokens: the layout plus up to 1 KB to
@@ -1064,15 +1142,44 @@ cudaError_t launch_tc_pair(const TcParams& p, bool suffix_mode, const DevCtl& ct
                            cudaStream_t st) {
   const int rows = p.Sq * p.Hq;
   const int n_pairs = (rows + 2 * kBM - 1) / (2 * kBM);
-  const int n_units = p.B * n_pairs * p.n_splits;
+  const int n_whole = p.B * n_pairs * p.n_splits;
+  const int n_slots = max(sm_count() / 2, 1);
+  TcParams q = p;
+  q.n_main = n_whole;
+  q.tail_splits = 1;
+  // Prefill with a batch-shared mask and scratch: when the last round of
+  // whole units would leave at least half the SM pairs idle, run full rounds
+  // whole and split each remaining unit over several pairs.  A piece pays a
+  // unit's fixed costs (its Q load, a partial write, the merge: about two
+  // tiles' time), so it must keep at least 6 key tiles: short sequences (pi0,
+  // pi0.5) are left whole, where splitting measured slower.
+  if (!suffix_mode && p.mask_bs == 0 && p.ws != nullptr && p.n_splits == 1) {
+    const int full = n_whole / n_slots, rem = n_whole % n_slots;
+    const int max_splits = ((p.Sq + kBN - 1) / kBN) / 6;
+    const int splits = rem >= 1 ? min(min(n_slots / rem, 8), max_splits) : 0;
+    if (full >= 1 && splits >= 2) {
+      q.n_main = full * n_slots;
+      q.tail_splits = splits;
+    }
+  }
+  const int n_units = q.n_main + (n_whole - q.n_main) * q.tail_splits;
   // A batch-shared mask lets one cluster per SM pair walk many units;
   // per-batch masks get one cluster per unit (each scans its own row).
-  const int n_clusters = p.mask_bs == 0 ? min(n_units, max(sm_count() / 2, 1)) : n_units;
+  const int n_clusters = p.mask_bs == 0 ? min(n_units, n_slots) : n_units;
   dim3 grid(2 * n_clusters, 1);
   const bool short_s = p.Sq <= LayoutShort::kMaxTok;
-  cudaError_t e = short_s ? launch_mode<LayoutShort>(p, suffix_mode, ctl, grid, st)
-                          : launch_mode<LayoutLong>(p, suffix_mode, ctl, grid, st);
-  if (e != cudaSuccess || p.n_splits <= 1) return e;
+  cudaError_t e = short_s ? launch_mode<LayoutShort>(q, suffix_mode, ctl, grid, st)
+                          : launch_mode<LayoutLong>(q, suffix_mode, ctl, grid, st);
+  if (e != cudaSuccess) return e;
+  if (q.tail_splits > 1) {
+    const int n_tail = n_whole - q.n_main;
+    const long long n_rows = (long long)n_tail * 2 * kBM;
+    return launch_pdl(tail_combine_kernel, dim3((unsigned)((n_rows + 7) / 8)), dim3(256), 0, st,
+                      static_cast<const float*>(p.ws),
+                      reinterpret_cast<__nv_bfloat16*>(p.out_ptr), p.lse, q.n_main, n_tail,
+                      q.tail_splits, n_pairs, rows);
+  }
+  if (p.n_splits <= 1) return e;
   const long long n_rows = (long long)p.B * rows;
   return launch_pdl(combine_kernel, dim3((unsigned)((n_rows + 7) / 8)), dim3(256), 0, st,
                     static_cast<const float*>(p.ws), reinterpret_cast<__nv_bfloat16*>(p.out_ptr),
@@ -1096,6 +1203,12 @@ int tc_suffix_splits(int B, int Sq, int P, int Hq) {
   s = min(s, tiles / 2);
   s = min(s, 8);
   return max(s, 1);
+}
+
+size_t tc_prefill_tail_bytes() {
+  // At most one round of pieces, one per SM pair, of 256 rows.
+  const size_t pieces = (size_t)max(sm_count() / 2, 1);
+  return pieces * 2 * kBM * (kD + 2) * sizeof(float);
 }
 
 size_t tc_suffix_workspace_bytes(int B, int Sq, int P, int Hq) {
