@@ -164,6 +164,10 @@ int pi_attn_prefill(const pi_attn_desc* desc, const void* q, const void* k, cons
  * enqueued.
  */
 size_t pi_attn_prefill_workspace_bytes(const pi_attn_desc* desc);
+/* Pieces per last-round query tile that pi_attn_prefill_ws would split into on
+ * the current device (1: no split; the call then launches one kernel, else
+ * two).  Host only. */
+int pi_attn_prefill_tail_splits(const pi_attn_desc* desc);
 int pi_attn_prefill_ws(const pi_attn_desc* desc, const void* q, const void* k, const void* v,
                        const uint8_t* ar_mask, const int32_t* segment_ids, void* out, float* lse,
                        void* workspace, size_t ws_bytes, pi_stream_t stream);

@@ -83,6 +83,9 @@ def test_tail_split_random_layouts(B, S, Hq, want):
     if n_slots == 74:
         assert _tail_splits(B, S, Hq, n_slots) == want
     rng = np.random.default_rng(5000 + S + Hq + B)
+    dummy = torch.empty((B, S, Hq, 256), dtype=torch.bfloat16, device="cuda")
+    assert _b().pi_attn_prefill_tail_splits(dummy, dummy[:, :, :1], torch.ones(
+        S, dtype=torch.uint8, device="cuda")) == _tail_splits(B, S, Hq, n_slots)
     ar, seg = W.random_layout(S, rng, with_seg=True)
     seg[rng.random(S) < 0.05] = -1
     s = 256 ** -0.25

@@ -42,6 +42,7 @@ EXPORTED = (
     "pi_attn_debug_tiles",
     "pi_attn_prefill_ws",
     "pi_attn_prefill_workspace_bytes",
+    "pi_attn_prefill_tail_splits",
 )
 
 
@@ -99,6 +100,8 @@ def lib() -> ctypes.CDLL:
         L.pi_attn_prefill_ws.restype = i32
         L.pi_attn_prefill_workspace_bytes.argtypes = [dp]
         L.pi_attn_prefill_workspace_bytes.restype = sz
+        L.pi_attn_prefill_tail_splits.argtypes = [dp]
+        L.pi_attn_prefill_tail_splits.restype = i32
         L.pi_attn_suffix.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.pi_attn_suffix.restype = i32
         L.pi_attn_suffix_workspace_bytes.argtypes = [dp]
@@ -185,6 +188,15 @@ def pi_attn_prefill_workspace_bytes(q, k, ar_mask, softmax_scale=1.0):
     desc = PiAttnDesc(B, S, 0, Hq, k.shape[2], d, _dtype_code(q), float(softmax_scale),
                       _mask_stride(ar_mask, B, S))
     return int(lib().pi_attn_prefill_workspace_bytes(ctypes.byref(desc)))
+
+
+def pi_attn_prefill_tail_splits(q, k, ar_mask, softmax_scale=1.0):
+    """Pieces per last-round query tile a call with a workspace splits into on
+    this device (1: none, one kernel launch per call; else two)."""
+    B, S, Hq, d = q.shape
+    desc = PiAttnDesc(B, S, 0, Hq, k.shape[2], d, _dtype_code(q), float(softmax_scale),
+                      _mask_stride(ar_mask, B, S))
+    return int(lib().pi_attn_prefill_tail_splits(ctypes.byref(desc)))
 
 
 def pi_attn_prefill(q, k, v, ar_mask, segment_ids=None, out=None, lse=None,

@@ -238,6 +238,12 @@ size_t pi_attn_prefill_workspace_bytes(const pi_attn_desc* d) {
   return tc_prefill_tail_bytes();
 }
 
+int pi_attn_prefill_tail_splits(const pi_attn_desc* d) {
+  if (check_desc(d, false) != PI_OK || !tail_split_applies(d) || d->B == 0 || d->Sq == 0)
+    return 1;
+  return tc_prefill_tail_splits(d->B, d->Sq, d->Hq);
+}
+
 int pi_attn_prefill_ws(const pi_attn_desc* d, const void* q, const void* k, const void* v,
                        const uint8_t* ar_mask, const int32_t* segment_ids, void* out, float* lse,
                        void* workspace, size_t ws_bytes, pi_stream_t stream) {

@@ -180,6 +180,8 @@ size_t tc_suffix_workspace_bytes(int B, int Sq, int P, int Hq);
 // Scratch of the prefill tail split on the current device: at most one round
 // of pieces (one per SM pair) of 256 rows, fp32 O and (m, l).
 size_t tc_prefill_tail_bytes();
+// Pieces per tail unit the prefill splits its last round into (1: none).
+int tc_prefill_tail_splits(int B, int Sq, int Hq);
 int tc_suffix_splits(int B, int Sq, int P, int Hq);
 
 // Merges split partials (unnormalised O [splits][rows][256] fp32, then (m, l)

@@ -1147,20 +1147,9 @@ cudaError_t launch_tc_pair(const TcParams& p, bool suffix_mode, const DevCtl& ct
   TcParams q = p;
   q.n_main = n_whole;
   q.tail_splits = 1;
-  // Prefill with a batch-shared mask and scratch: when the last round of
-  // whole units would leave at least half the SM pairs idle, run full rounds
-  // whole and split each remaining unit over several pairs.  A piece pays a
-  // unit's fixed costs (its Q load, a partial write, the merge: about two
-  // tiles' time), so it must keep at least 6 key tiles: short sequences (pi0,
-  // pi0.5) are left whole, where splitting measured slower.
   if (!suffix_mode && p.mask_bs == 0 && p.ws != nullptr && p.n_splits == 1) {
-    const int full = n_whole / n_slots, rem = n_whole % n_slots;
-    const int max_splits = ((p.Sq + kBN - 1) / kBN) / 6;
-    const int splits = rem >= 1 ? min(min(n_slots / rem, 8), max_splits) : 0;
-    if (full >= 1 && splits >= 2) {
-      q.n_main = full * n_slots;
-      q.tail_splits = splits;
-    }
+    q.tail_splits = tc_prefill_tail_splits(p.B, p.Sq, p.Hq);
+    if (q.tail_splits > 1) q.n_main = n_whole / n_slots * n_slots;
   }
   const int n_units = q.n_main + (n_whole - q.n_main) * q.tail_splits;
   // A batch-shared mask lets one cluster per SM pair walk many units;
@@ -1203,6 +1192,21 @@ int tc_suffix_splits(int B, int Sq, int P, int Hq) {
   s = min(s, tiles / 2);
   s = min(s, 8);
   return max(s, 1);
+}
+
+int tc_prefill_tail_splits(int B, int Sq, int Hq) {
+  // When the last round of whole units would leave at least half the SM
+  // pairs idle, the full rounds run whole and each remaining unit is split
+  // over several pairs.  A piece pays a unit's fixed costs (its Q load, a
+  // partial write, the merge: about two tiles' time), so it must keep at
+  // least 6 key tiles: short sequences (pi0, pi0.5) are left whole, where
+  // splitting measured slower.
+  const int n_slots = max(sm_count() / 2, 1);
+  const int n_whole = B * ((Sq * Hq + 2 * kBM - 1) / (2 * kBM));
+  const int full = n_whole / n_slots, rem = n_whole % n_slots;
+  if (full < 1 || rem < 1) return 1;
+  const int splits = min(min(n_slots / rem, 8), ((Sq + kBN - 1) / kBN) / 6);
+  return splits >= 2 ? splits : 1;
 }
 
 size_t tc_prefill_tail_bytes() {
