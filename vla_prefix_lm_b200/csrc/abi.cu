@@ -297,12 +297,12 @@ int pi_attn_suffix_masked(const pi_attn_desc* d, const void* q_suf, const void* 
     // element and merged on chip (no workspace).
     DecodeParams p;
     std::memset(&p, 0, sizeof(p));
-    if (!encode_rows(&p.map_k, k_suf, d->Sq, d->B, 32) ||
-        !encode_rows(&p.map_v, v_suf, d->Sq, d->B, 32))
+    if (!encode_rows(&p.map_k, k_suf, d->Sq, d->B, kDecodeTileKeys) ||
+        !encode_rows(&p.map_v, v_suf, d->Sq, d->B, kDecodeTileKeys))
       return PI_ERR_CUDA;
     if (d->P > 0) {
-      if (!encode_rows(&p.map_kc, k_cache, d->P, d->B, 32) ||
-          !encode_rows(&p.map_vc, v_cache, d->P, d->B, 32))
+      if (!encode_rows(&p.map_kc, k_cache, d->P, d->B, kDecodeTileKeys) ||
+          !encode_rows(&p.map_vc, v_cache, d->P, d->B, kDecodeTileKeys))
         return PI_ERR_CUDA;
     } else {
       p.map_kc = p.map_k;

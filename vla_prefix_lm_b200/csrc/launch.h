@@ -191,7 +191,8 @@ cudaError_t launch_combine(const float* ws, __nv_bfloat16* out, int n_splits, lo
 
 // Suffix pass with at most 8 query rows per batch element (decode.cu): bf16,
 // one KV head, d = 256.  Needs no workspace.  Cache and suffix K/V as 4-D
-// views, box (64, 32, 4, 1).
+// views, box (64, kDecodeTileKeys, 4, 1).
+constexpr int kDecodeTileKeys = 16;
 struct DecodeParams {
   CUtensorMap map_kc;
   CUtensorMap map_vc;
