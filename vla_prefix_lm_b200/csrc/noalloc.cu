@@ -3,11 +3,11 @@
 // cannot allocate device memory.  The method itself has no such call: it is
 // plumbing around pi_attn_suffix, which it calls unchanged.
 //
-// The buffer is a file-scope __device__ array (one copy per device, created
-// with the module).  Its address is looked up once per device with
-// cudaGetSymbolAddress and cached; no call here allocates or frees memory.
-#include <mutex>
-
+// The buffer is a file-scope __device__ array (one copy per device context,
+// created with the module).  Its address is looked up on every call with
+// cudaGetSymbolAddress (a host-side table lookup), so it stays right after
+// the context is reset and the module reloaded; no call here allocates or
+// frees memory.
 #include "../../include/pi_attn.h"
 
 namespace {
@@ -20,18 +20,8 @@ constexpr size_t kStaticWsBytes = size_t(16) << 20;
 __device__ __align__(256) unsigned char g_suffix_ws[kStaticWsBytes];
 
 void* static_ws_ptr() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-  static std::mutex mu;
-  static void* ptrs[64] = {nullptr};
-  if (dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_suffix_ws) != cudaSuccess) return nullptr;
-    ptrs[dev] = p;
-  }
-  return ptrs[dev];
+  void* p = nullptr;
+  return cudaGetSymbolAddress(&p, g_suffix_ws) == cudaSuccess ? p : nullptr;
 }
 
 }  // namespace
