@@ -299,7 +299,12 @@ const char* pi_attn_status_string(int status);
  * pi_attn_set_wait_limit -- bound, in SM clock cycles, on every device-side
  * spin wait (mbarrier phase waits) in kernels launched after this call.
  * 0 restores the default (2^31 cycles, about a second).  Returns the previous
- * value.  Process-wide.
+ * value.  Process-wide.  The value in force when the library is loaded is the
+ * environment variable PIATTN_WATCHDOG_CYCLES (a positive decimal integer)
+ * if set, else the default.
+ *
+ * Every entry point that enqueues work opens an NVTX range named after itself
+ * for its host-side duration (inert unless a profiler is attached).
  */
 uint64_t pi_attn_set_wait_limit(uint64_t cycles);
 

@@ -120,6 +120,23 @@ def test_status_strings_and_wait_limit():
     assert b.pi_attn_set_wait_limit(prev) == 1 << 31
 
 
+@pytest.mark.parametrize("value,expect", [("777", 777), ("abc", 1 << 31), ("0", 1 << 31)])
+def test_watchdog_env_sets_the_initial_wait_limit(value, expect):
+    """PIATTN_WATCHDOG_CYCLES (a positive integer) is the wait bound in force
+    when the library loads; anything else leaves the default."""
+    import subprocess
+    import sys
+    _lib()   # built
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "from vla_prefix_lm_b200 import binding\n"
+            "print(binding.pi_attn_set_wait_limit(5))\n" % ROOT)
+    env = dict(os.environ, PIATTN_WATCHDOG_CYCLES=value)
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert int(r.stdout.strip().splitlines()[-1]) == expect
+
+
 def test_debug_mask_argument_errors():
     b, L = _lib()
     d = _desc(b)

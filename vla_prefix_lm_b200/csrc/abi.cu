@@ -5,11 +5,12 @@
 // Validation happens entirely on the host, before anything is enqueued: an
 // entry point that returns an error has launched nothing.
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
-#include <mutex>
 
 #include "../../include/pi_attn.h"
 #include "launch.h"
@@ -20,24 +21,37 @@ namespace {
 using namespace piattn;
 
 constexpr unsigned long long kDefaultWaitLimit = 1ull << 31;
-std::atomic<unsigned long long> g_wait_limit{kDefaultWaitLimit};
 
-// The device status word (one per device the library runs on).
+// The bound on every device-side wait, in SM cycles: PIATTN_WATCHDOG_CYCLES
+// when set (a positive integer) at load time, else 2^31 (about a second).
+unsigned long long initial_wait_limit() {
+  const char* e = std::getenv("PIATTN_WATCHDOG_CYCLES");
+  if (e && *e) {
+    char* end = nullptr;
+    const unsigned long long v = std::strtoull(e, &end, 10);
+    if (end && *end == '\0' && v > 0) return v;
+  }
+  return kDefaultWaitLimit;
+}
+std::atomic<unsigned long long> g_wait_limit{initial_wait_limit()};
+
+// An NVTX range around each entry point that enqueues work (free unless a
+// profiler is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
+// The device status word (one per device context).  Its address is looked up
+// on every call (a host-side table lookup), so it stays right after the
+// context is reset and the module reloaded.
 __device__ int g_status;
 
 int* status_ptr() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-  static std::mutex mu;
-  static int* ptrs[64] = {nullptr};
-  if (dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
-    ptrs[dev] = static_cast<int*>(p);
-  }
-  return ptrs[dev];
+  void* p = nullptr;
+  return cudaGetSymbolAddress(&p, g_status) == cudaSuccess ? static_cast<int*>(p) : nullptr;
 }
 
 bool make_ctl(DevCtl* ctl) {
@@ -230,6 +244,7 @@ int prefill_impl(const pi_attn_desc* d, const void* q, const void* k, const void
 int pi_attn_prefill(const pi_attn_desc* d, const void* q, const void* k, const void* v,
                     const uint8_t* ar_mask, const int32_t* segment_ids, void* out, float* lse,
                     pi_stream_t stream) {
+  NvtxRange range("pi_attn_prefill");
   return prefill_impl(d, q, k, v, ar_mask, segment_ids, out, lse, nullptr, 0, stream);
 }
 
@@ -247,6 +262,7 @@ int pi_attn_prefill_tail_splits(const pi_attn_desc* d) {
 int pi_attn_prefill_ws(const pi_attn_desc* d, const void* q, const void* k, const void* v,
                        const uint8_t* ar_mask, const int32_t* segment_ids, void* out, float* lse,
                        void* workspace, size_t ws_bytes, pi_stream_t stream) {
+  NvtxRange range("pi_attn_prefill_ws");
   return prefill_impl(d, q, k, v, ar_mask, segment_ids, out, lse, workspace, ws_bytes, stream);
 }
 
@@ -262,6 +278,7 @@ int pi_attn_suffix_masked(const pi_attn_desc* d, const void* q_suf, const void* 
                           const uint8_t* ar_mask_suf, const int32_t* segment_ids_suf,
                           const uint8_t* cache_valid, void* out, void* workspace,
                           size_t ws_bytes, pi_stream_t stream) {
+  NvtxRange range("pi_attn_suffix_masked");
   int rc = check_desc(d, true);
   if (rc != PI_OK) return rc;
   if (d->B == 0 || d->Sq == 0) return PI_OK;
@@ -358,12 +375,14 @@ int pi_attn_suffix(const pi_attn_desc* d, const void* q_suf, const void* k_suf,
                    const void* v_suf, const void* k_cache, const void* v_cache,
                    const uint8_t* ar_mask_suf, void* out, void* workspace, size_t ws_bytes,
                    pi_stream_t stream) {
+  NvtxRange range("pi_attn_suffix");
   return pi_attn_suffix_masked(d, q_suf, k_suf, v_suf, k_cache, v_cache, ar_mask_suf, nullptr,
                                nullptr, out, workspace, ws_bytes, stream);
 }
 
 int pi_rope_inplace(const pi_rope_desc* d, void* q, void* k, const uint8_t* token_mask,
                     const uint8_t* prefix_mask, int32_t* positions_out, pi_stream_t stream) {
+  NvtxRange range("pi_rope_inplace");
   if (!d) return PI_ERR_ARG;
   if (d->B < 0 || d->S < 0 || d->P < 0 || d->Hq <= 0 || d->Hkv <= 0 || d->d <= 0)
     return PI_ERR_ARG;
@@ -401,6 +420,7 @@ int pi_rope_inplace(const pi_rope_desc* d, void* q, void* k, const uint8_t* toke
 
 int pi_euler_update(float* x, const void* v, int32_t v_dtype, float dt, int64_t n,
                     pi_stream_t stream) {
+  NvtxRange range("pi_euler_update");
   if (n < 0 || !std::isfinite(dt)) return PI_ERR_ARG;
   if (v_dtype != PI_BF16 && v_dtype != PI_F32) return PI_ERR_UNSUPPORTED;
   if (n == 0) return PI_OK;
@@ -419,6 +439,7 @@ int pi_attn_prefill_backward(const pi_attn_desc* d, const void* q, const void* k
                              const uint8_t* ar_mask, const int32_t* segment_ids, const void* out,
                              const float* lse, const void* dout, float* dq, float* dk, float* dv,
                              void* workspace, size_t ws_bytes, pi_stream_t stream) {
+  NvtxRange range("pi_attn_prefill_backward");
   const int rc = check_backward_desc(d);
   if (rc != PI_OK) return rc;
   if (d->B == 0 || d->Sq == 0) return PI_OK;
