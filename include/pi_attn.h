@@ -42,11 +42,11 @@
  * work.  Calls on different streams may run concurrently; the global state is
  * the device status word read by pi_attn_read_status, the wait bound set by
  * pi_attn_set_wait_limit, and the fixed scratch of pi_attn_suffix_noalloc.
- * The device addresses of the status word and of that scratch, and each
- * device's SM count, are looked up on the first call that needs them on that
- * device and kept for the life of the process: a device reset
- * (cudaDeviceReset) after the first call invalidates them, so do not reset a
- * device this library has run on.
+ * The device addresses of the status word and of that scratch are looked up
+ * on every call (cudaGetSymbolAddress, a host-side lookup that is allowed
+ * during stream capture), so they stay right after a device reset
+ * (cudaDeviceReset) reloads the module; each device's SM count is looked up
+ * once and kept.
  *
  * Errors: every entry point returns PI_OK or a PI_ERR_* code.  Argument
  * errors are detected on the host before anything is enqueued (nothing is
@@ -326,9 +326,8 @@ int pi_attn_selftest_wait(pi_stream_t stream);
  * pi_attn_suffix_noalloc_capacity() = 16 MiB).
  *
  *  - Allocates nothing: no cudaMalloc/cudaFree, no allocating library call.
- *  - The first call on each device looks up the buffer's address
- *    (cudaGetSymbolAddress) and caches it; make that first call before any
- *    stream capture begins.
+ *  - Each call looks up the buffer's address (cudaGetSymbolAddress) on the
+ *    current device; the lookup also works during stream capture.
  *  - Nothing in the buffer needs to start at zero: every call writes each
  *    partial it later reads.
  *  - Two calls that may overlap on the GPU (different streams of one device)
