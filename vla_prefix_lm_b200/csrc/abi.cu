@@ -467,10 +467,8 @@ int pi_attn_prefill_backward(const pi_attn_desc* d, const void* q, const void* k
     t.P = reinterpret_cast<__nv_bfloat16*>(w + plan.off_P);
     t.dS = reinterpret_cast<__nv_bfloat16*>(w + plan.off_dS);
     t.part = plan.n_chunks > 1 ? reinterpret_cast<float*>(w + plan.off_part) : nullptr;
-    if (!encode_rows(&t.map_q, q, rows, d->B, 128) ||
-        !encode_rows(&t.map_do, dout, rows, d->B, 128) ||
-        !encode_rows(&t.map_k32, k, d->Sq, d->B, 32) ||
-        !encode_rows(&t.map_v32, v, d->Sq, d->B, 32) ||
+    if (!encode_rows(&t.map_k64, k, d->Sq, d->B, 64) ||
+        !encode_rows(&t.map_v64, v, d->Sq, d->B, 64) ||
         !encode_rows(&t.map_kh, k, d->Sq, d->B, 64, 2) ||
         !encode_rows(&t.map_qh, q, rows, d->B, 64, 2) ||
         !encode_rows(&t.map_doh, dout, rows, d->B, 64, 2) ||
@@ -481,11 +479,11 @@ int pi_attn_prefill_backward(const pi_attn_desc* d, const void* q, const void* k
         !encode_rows64b(&t.map_dsw, t.dS, plan.Skp, rows, d->B, pitch))
       return PI_ERR_CUDA;
     t.ar = ar_mask; t.seg = segment_ids; t.mask_bs = d->mask_batch_stride;
-    t.out = out; t.dout = dout; t.lse = lse;
+    t.q = q; t.out = out; t.dout = dout; t.lse = lse;
     t.dq = dq; t.dk = dk; t.dv = dv;
     t.B = d->B; t.S = d->Sq; t.Hq = d->Hq; t.Skp = plan.Skp;
     t.n_chunks = plan.n_chunks; t.pairs_per_chunk = plan.pairs_per_chunk;
-    t.ns1 = plan.ns1; t.clusters = plan.clusters;
+    t.clusters = plan.clusters;
     t.scale = d->softmax_scale;
     t.scale_log2 = d->softmax_scale * 1.4426950408889634f;
     return launched(launch_backward_tc(t, ctl, static_cast<cudaStream_t>(stream)));

@@ -17,12 +17,16 @@
 // once each, every one on tcgen05 pair MMAs (cta_group::2, M = 256 rows over a
 // cluster of two CTAs):
 //
-//   score pass  query-major: S = Q K^T and dP = dO V^T on 64-key tiles into
-//               TMEM; one thread per row forms P and dS in fp32 and writes
-//               both as bf16 to the caller's workspace [B, rows, Skp] (Skp = S
-//               rounded up to 64).  Persistent: each SM pair takes an equal,
-//               contiguous run of the (batch, 256-row tile, key tile) sequence
-//               and reloads Q and dO only when the row tile changes.
+//   score pass  query-major: S = Q K^T and dP = dO V^T on 128-key tiles into
+//               TMEM (N = 128 pair MMAs in TS form: the row tile's Q and dO
+//               sit in TMEM as the A operand, 256 of the 512 columns, copied
+//               in by the row warps when the row tile changes; S and dP take
+//               the other 256, one buffer); one thread per row and 32 keys
+//               forms P and dS in fp32 and writes both as bf16 to the
+//               caller's workspace [B, rows, Skp] (Skp = S rounded up to 64).
+//               Persistent: each SM pair takes an equal, contiguous run of the
+//               (batch, 256-row tile, key tile) sequence; shared memory holds
+//               a two-stage K/V ring and the P/dS store stages.
 //   dK/dV pass  key-major, per 256-key group: dV += P^T dO and dK += dS^T Q
 //               over 64-row steps, P^T and dS^T read MN-major from the
 //               workspace; small problems split the rows into chunks whose
@@ -33,7 +37,7 @@
 //
 // Tiles are skipped by the forward's rule: a 256-key group is visited by a
 // 256-row tile unless no row of it sees any key of the group (block index,
-// expert <- FAST, padding).  The score pass writes all four 64-key tiles of a
+// expert <- FAST, padding).  The score pass writes both 128-key tiles of a
 // visited group (exact zeros where masked), so the dK/dV pass, which reads
 // whole groups, never reads an unwritten block.  Rows go to global memory
 // through a per-warp shared-memory transpose, so every store instruction
@@ -49,7 +53,7 @@ namespace piattn {
 namespace {
 
 constexpr int kT = 192;          // warp 0 TMA, warp 1 TMEM + MMA issue, warps 2..5 rows
-constexpr int kT1 = 320;         // score pass: warps 2..9 rows, two per TMEM lane quarter
+constexpr int kT1 = 576;         // score pass: warps 2..17 rows, four per TMEM lane quarter
 constexpr int kRows = 128;       // rows per CTA (256 per pair)
 constexpr int kD = 256;
 constexpr int kKT = 64;          // keys per score tile (32 per CTA)
@@ -59,31 +63,32 @@ constexpr int kMaxTiles128 = (kMaxTokens + 127) / 128 + 1;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Shared-memory operand sizes (bf16, 128-byte swizzled [rows x 64] blocks).
-constexpr int kRowTile = kRows * kD * 2;       // [128 x 256]   64 KB (Q, dO in the score pass)
-constexpr int kItem32 = 32 * kD * 2;           // [32 x 256]    16 KB (this CTA's keys of a score tile)
+constexpr int kKT1 = 128;        // keys per score-pass tile (64 per CTA)
+constexpr int kItem64 = 64 * kD * 2;           // [64 x 256]    32 KB (this CTA's keys of a score tile)
 constexpr int kHalf64 = 64 * 128 * 2;          // [64 x 128]    16 KB (64 rows/keys x this CTA's d-half)
 constexpr int kDsTile = kRows * 64 * 2;        // [128 x 64]    16 KB (dS rows of a 64-key tile)
 constexpr int kWarpStage = 32 * 128;           // 4 KB per row warp: 32 rows x 128 B transpose
 
 constexpr int kNS2 = 3, kNS3 = 4;              // ring stages of the dK/dV and dQ passes
-constexpr int kStage1 = 2 * kItem32;           // K, V items
+constexpr int kStage1 = 2 * kItem64;           // K, V items
+constexpr int kNS1 = 2;                        // ring stages of the score pass
+constexpr int kBox1 = 32 * 64;                 // 2 KB per score row warp: one 32 x 32 bf16 box
 constexpr int kStage2 = 4 * kHalf64;           // P^T, dS^T, dO half, Q half
 constexpr int kStage3 = kDsTile + kHalf64;     // dS tile, K half
-__host__ __device__ constexpr int ops1(int ns) { return 2 * kRowTile + ns * kStage1 + 4 * kWarpStage; }
+constexpr int kOps1 = kNS1 * kStage1 + 16 * kBox1;             // 160 KB
 constexpr int kOps2 = kNS2 * kStage2;                        // 192 KB
 constexpr int kOps3 = kNS3 * kStage3 + 4 * kWarpStage;       // 144 KB
 
-constexpr uint32_t kIdescScore = idesc_bf16_f32(2 * kRows, kKT, false, false);
+constexpr uint32_t kIdescScore = idesc_bf16_f32(2 * kRows, kKT1, false, false);
 constexpr uint32_t kIdescKV = idesc_bf16_f32(2 * kRows, kD, true, true);
 constexpr uint32_t kIdescQ = idesc_bf16_f32(2 * kRows, kD, false, true);
 
 struct __align__(8) Ctl {
   uint64_t full[4];       // leader: a ring stage of both CTAs landed
   uint64_t empty[4];      // each CTA: its stage may be refilled
-  uint64_t qd_full;       // leader (score pass): Q and dO of both CTAs landed
-  uint64_t qd_empty;      // each CTA (score pass): the row tile's last MMA read them
-  uint64_t s_full[2];     // each CTA (score pass): S and dP of a tile in TMEM
-  uint64_t s_free[2];     // leader (score pass): the pair's 16 row warps read them
+  uint64_t qd_full;       // leader (score pass): the pair's 32 row warps put Q and dO in TMEM
+  uint64_t s_full;        // each CTA (score pass): S and dP of a tile in TMEM
+  uint64_t s_free;        // leader (score pass): the pair's 32 row warps read them
   uint64_t done[2];       // each CTA: an accumulator is final
   uint64_t acc_free[2];   // leader (dQ pass): the pair's 8 row warps read an accumulator
   uint64_t drain;         // leader: every MMA issued has completed
@@ -238,7 +243,20 @@ __device__ __forceinline__ uint8_t* bwd_smem(uint8_t* raw, int need, int smem_by
 
 // ---------------------------------------------------------------- score pass
 
-// Position in a cluster's run of the (batch, row tile, visited key tile)
+// The score pass's visited 128-key tiles of a row tile, in order (two per
+// 256-key group).
+__device__ __forceinline__ int next_tile128(const Ctl& c, uint32_t csq1, bool all_e, int kt,
+                                            int S, int n_kt) {
+  int t = kt + 1;
+  while (t < n_kt) {
+    if ((t & 1) != 0) return t;                 // the second tile of a visited group
+    if (group_visible(c, csq1, all_e, t >> 1, S)) return t;
+    t += 2;
+  }
+  return -1;
+}
+
+// Position in a cluster's run of the (batch, row tile, visited 128-key tile)
 // sequence.  Every role walks the same run with its own copy.
 struct TileWalk {
   int b, pair, kt, left;
@@ -253,7 +271,7 @@ __device__ __forceinline__ void walk_enter(TileWalk& w, const Ctl& c, const int*
   w.csq1 = codes[tq1] >> 2;
   w.all_e = ((pinfo[w.pair] >> 30) & 1) != 0;
   w.kt = -1;
-  for (int i = 0; i <= j; ++i) w.kt = next_tile(c, w.csq1, w.all_e, w.kt, S, n_kt);
+  for (int i = 0; i <= j; ++i) w.kt = next_tile128(c, w.csq1, w.all_e, w.kt, S, n_kt);
 }
 
 // Moves to the next tile of the run; returns true if the row tile changed.
@@ -261,7 +279,7 @@ __device__ __forceinline__ bool walk_next(TileWalk& w, const Ctl& c, const int* 
                                           const uint16_t* codes, int S, int n_kt, int n_pairs,
                                           int tok_per_pair) {
   if (--w.left <= 0) return false;
-  const int nk = next_tile(c, w.csq1, w.all_e, w.kt, S, n_kt);
+  const int nk = next_tile128(c, w.csq1, w.all_e, w.kt, S, n_kt);
   if (nk >= 0) {
     w.kt = nk;
     return false;
@@ -276,22 +294,101 @@ __device__ __forceinline__ bool walk_next(TileWalk& w, const Ctl& c, const int* 
   return true;
 }
 
+// Score pass, at a row tile (b, pair): this row warp's share of its Q (parts
+// 0, 1) or dO (parts 2, 3), a 256-byte slice of each of the warp's 32 rows,
+// into TMEM lane quarter * 32 + row, 64 columns of bf16 pairs (the MMA's A
+// layout).  Coalesced loads (8 rows x 64 B per instruction) become one row
+// per lane through the warp's 2 KB stage (16-byte chunk j of row r at
+// j ^ ((r / 2) % 4)); then the warp arrives on the leader's qd_full and warms
+// L2 with the following row tile's rows (its Q / dO, lse, D).  Called only at
+// row-tile switches, so it is kept out of line.
+__device__ __noinline__ void score_copy_rows(const BwdTcParams& p, int b, int pair, uint32_t rank,
+                                             int quarter, int part, uint32_t tmem,
+                                             uint8_t* wstage, bool store_pending,
+                                             const int* pinfo, int n_pairs, uint32_t qd_full_l) {
+  const int lane = threadIdx.x & 31;
+  const int rows_per_b = p.S * p.Hq;
+  const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+  const int r0 = pair * 2 * kRows + (int)rank * kRows + quarter * 32;
+  const long long g0 = (long long)b * rows_per_b + r0;
+  const uint8_t* gsrc = static_cast<const uint8_t*>(part < 2 ? p.q : p.dout) +
+                        g0 * (long long)(kD * 2) + 256 * (part & 1);
+  const uint32_t tdst = tmem + lane_off + 256 + 128 * (part >> 1) + 64 * (part & 1);
+  if (store_pending) {   // the last P / dS box has been read out of the stage
+    if (lane == 0) tma_store_wait_read();
+    __syncwarp();
+  }
+#pragma unroll 1
+  for (int h2 = 0; h2 < 2; ++h2) {
+    uint4 qv[2][4];
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int rr = 8 * i + (lane >> 2);
+        qv[c2][i] = r0 + rr < rows_per_b
+                        ? *reinterpret_cast<const uint4*>(gsrc + rr * (kD * 2) + 128 * h2 +
+                                                          64 * c2 + 16 * (lane & 3))
+                        : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+    for (int c2 = 0; c2 < 2; ++c2) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int rr = 8 * i + (lane >> 2);
+        *reinterpret_cast<uint4*>(wstage + rr * 64 + (((lane & 3) ^ ((rr >> 1) & 3)) << 4)) =
+            qv[c2][i];
+      }
+      __syncwarp();
+      uint32_t r16[16];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 t4 =
+            *reinterpret_cast<const uint4*>(wstage + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4));
+        r16[4 * j] = t4.x; r16[4 * j + 1] = t4.y;
+        r16[4 * j + 2] = t4.z; r16[4 * j + 3] = t4.w;
+      }
+      __syncwarp();
+      tmem_st16(tdst + 32 * h2 + 16 * c2, r16);
+    }
+  }
+  tmem_st_wait();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive_remote(qd_full_l);
+  if (p.mask_bs == 0 && (part & 1) == 0) {
+    int nb = b, npair = pair;
+    do {
+      if (++npair == n_pairs) {
+        npair = 0;
+        ++nb;
+      }
+    } while (nb < p.B && (pinfo[npair] & 0x3FFFFFFF) == 0);
+    const int nr0 = npair * 2 * kRows + (int)rank * kRows + quarter * 32;
+    const int nrows = min(32, rows_per_b - nr0);
+    if (nb < p.B && nrows > 0) {
+      const long long ng0 = (long long)nb * rows_per_b + nr0;
+      if (lane == 0)
+        bulk_prefetch_l2(static_cast<const uint8_t*>(part < 2 ? p.q : p.dout) + ng0 * (kD * 2),
+                         (uint32_t)nrows * (kD * 2));
+      if (lane < nrows) prefetch_l2(part < 2 ? p.lse + ng0 + lane : p.D + ng0 + lane);
+    }
+  }
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
     bwd_score_kernel(const __grid_constant__ BwdTcParams p, const DevCtl ctl, int smem_bytes) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const int S = p.S, Hq = p.Hq, ns = p.ns1;
+  const int S = p.S, Hq = p.Hq;
   const int rows_per_b = S * Hq;
   const int n_pairs = (rows_per_b + 2 * kRows - 1) / (2 * kRows);
-  const int ops = ops1(ns);
-  uint8_t* smem = bwd_smem(smem_raw, smem_need(ops, S, n_pairs * 4), smem_bytes, ctl, S);
+  uint8_t* smem = bwd_smem(smem_raw, smem_need(kOps1, S, n_pairs * 4), smem_bytes, ctl, S);
   if (smem == nullptr) return;
-  Ctl& c = *reinterpret_cast<Ctl*>(smem + ops);
-  int* pinfo = reinterpret_cast<int*>(smem + ops + ctl_bytes());
-  uint16_t* codes = reinterpret_cast<uint16_t*>(smem + ops + ctl_bytes() + pad128(n_pairs * 4));
-  uint8_t* sQ = smem;
-  uint8_t* sdO = smem + kRowTile;
-  uint8_t* ring = smem + 2 * kRowTile;
-  uint8_t* stage = ring + ns * kStage1;
+  Ctl& c = *reinterpret_cast<Ctl*>(smem + kOps1);
+  int* pinfo = reinterpret_cast<int*>(smem + kOps1 + ctl_bytes());
+  uint16_t* codes = reinterpret_cast<uint16_t*>(smem + kOps1 + ctl_bytes() + pad128(n_pairs * 4));
+  uint8_t* ring = smem;
+  uint8_t* stage = ring + kNS1 * kStage1;
 
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -299,7 +396,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
   const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
   const int tok_per_pair = 2 * kRows / Hq;
   const int n_sup = (S + kSup - 1) / kSup;
-  const int n_kt = (S + kKT - 1) / kKT;
+  const int n_kt = (S + kKT1 - 1) / kKT1;
   // A batch-shared mask: the clusters split the whole run evenly.  Per-batch
   // masks: one cluster per (batch, row tile), scanning its own batch row.
   const bool per_batch = p.mask_bs != 0;
@@ -309,29 +406,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
   const int32_t* seg_b = p.seg ? p.seg + (long long)b_mask * p.mask_bs : nullptr;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < ns; ++s) {
+    for (int s = 0; s < kNS1; ++s) {
       mbar_init(&c.full[s], 1);
       mbar_init(&c.empty[s], 1);
     }
-    mbar_init(&c.qd_full, 1);
-    mbar_init(&c.qd_empty, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&c.s_full[s], 1);
-      mbar_init(&c.s_free[s], 16);
-    }
+    mbar_init(&c.qd_full, 32);
+    mbar_init(&c.s_full, 1);
+    mbar_init(&c.s_free, 32);
     mbar_init(&c.drain, 1);
     c.abort = 0;
     fence_barrier_init();
-    tma_prefetch_desc(&p.map_q);
-    tma_prefetch_desc(&p.map_do);
-    tma_prefetch_desc(&p.map_k32);
-    tma_prefetch_desc(&p.map_v32);
+    tma_prefetch_desc(&p.map_k64);
+    tma_prefetch_desc(&p.map_v64);
     tma_prefetch_desc(&p.map_pw);
     tma_prefetch_desc(&p.map_dsw);
   }
   cluster_sync();
   if (warp == 1) {
-    tmem_alloc_pair(&c.tmem_base, 256);
+    tmem_alloc_pair(&c.tmem_base, 512);
     tmem_relinquish_pair();
   }
   // Nothing above touched global memory (it may overlap the previous kernel);
@@ -349,7 +441,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
     const uint32_t csq1 = codes[tq1] >> 2;
     int cnt = 0;
     for (int ks = 0; ks < n_sup; ++ks)
-      if (group_visible(c, csq1, all_e, ks, S)) cnt += min(4 * ks + 4, n_kt) - 4 * ks;
+      if (group_visible(c, csq1, all_e, ks, S)) cnt += min(2 * ks + 2, n_kt) - 2 * ks;
     pinfo[pr] = cnt | (all_e ? (1 << 30) : 0);
   }
   tc_fence_before();
@@ -386,49 +478,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
+    // (Q and dO of each row tile reach TMEM through the row warps.)
     TileWalk w = w0;
-    uint32_t n = 0, np = 0;
-    bool new_pair = true, ok = true;
-    const uint32_t qd_full_l = mapa_shared(smem_u32(&c.qd_full), 0);
+    uint32_t n = 0;
+    bool ok = true;
     // K and V are read by every row tile: keep them in L2 against the P and dS
     // stream this pass writes.
     const uint64_t keep = l2_policy_evict_last();
     while (w.left > 0 && ok) {
-      if (new_pair) {
-        // Q and dO of the row tile; the previous tile's last MMA read them.
-        if (np > 0 && !warp_wait(&c.qd_empty, (np - 1) & 1, c, ctl)) break;
-        if (lane == 0) {
-          if (leader) mbar_arrive_expect_tx(&c.qd_full, 4 * kRowTile);
-          const int row0 = w.pair * 2 * kRows + (int)rank * kRows;
-          tma_load_4d_pair(sQ, &p.map_q, qd_full_l, 0, row0, 0, w.b);
-          tma_load_4d_pair(sdO, &p.map_do, qd_full_l, 0, row0, 0, w.b);
-        }
-        __syncwarp();
-        ++np;
-      }
-      const int s = (int)(n % ns);
-      const uint32_t rel = n / ns;
+      const int s = (int)(n % kNS1);
+      const uint32_t rel = n / kNS1;
       if (rel > 0 && !warp_wait(&c.empty[s], (rel - 1) & 1, c, ctl)) break;
       if (lane == 0) {
         const uint32_t full_l = mapa_shared(smem_u32(&c.full[s]), 0);
         if (leader) mbar_arrive_expect_tx(&c.full[s], 2 * kStage1);
         uint8_t* st = ring + s * kStage1;
-        // this CTA's 32 keys of the tile, all 256 columns, of K and of V
-        tma_load_4d_pair_hint(st, &p.map_k32, full_l, 0, w.kt * kKT + 32 * (int)rank, 0, w.b,
-                              keep);
-        tma_load_4d_pair_hint(st + kItem32, &p.map_v32, full_l, 0, w.kt * kKT + 32 * (int)rank,
-                              0, w.b, keep);
+        // this CTA's 64 keys of the tile, all 256 columns, of K and of V
+        const int key0 = w.kt * kKT1 + 64 * (int)rank;
+        tma_load_4d_pair_hint(st, &p.map_k64, full_l, 0, key0, 0, w.b, keep);
+        tma_load_4d_pair_hint(st + kItem64, &p.map_v64, full_l, 0, key0, 0, w.b, keep);
       }
       __syncwarp();
       ++n;
-      new_pair = walk_next(w, c, pinfo, codes, S, n_kt, n_pairs, tok_per_pair);
+      (void)walk_next(w, c, pinfo, codes, S, n_kt, n_pairs, tok_per_pair);
     }
     // Loads complete on the leader's barriers: wait there (bounded) for the
     // last phase of each, so no copy is in flight when the cluster leaves.
     if (leader && lane == 0) {
-      if (np > 0) (void)mbar_wait(&c.qd_full, (np - 1) & 1, ctl);
-      for (int s = 0; s < ns; ++s) {
-        const uint32_t n_s = n > (uint32_t)s ? (n - (uint32_t)s + ns - 1) / ns : 0;
+      for (int s = 0; s < kNS1; ++s) {
+        const uint32_t n_s = n > (uint32_t)s ? (n - (uint32_t)s + kNS1 - 1) / kNS1 : 0;
         if (n_s > 0) (void)mbar_wait(&c.full[s], (n_s - 1) & 1, ctl);
       }
     }
@@ -436,48 +514,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
   } else if (warp == 1) {
     // ------------------------------------------- MMA issue (leader CTA only)
     if (leader) {
-      const uint64_t qdesc = sdesc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t dodesc = sdesc_sw128(smem_u32(sdO), 16, 1024);
       const uint64_t rdesc = sdesc_sw128(smem_u32(ring), 16, 1024);
+      const uint32_t tS = tmem, tP = tmem + 128, tQ = tmem + 256, tdO = tmem + 384;
       TileWalk w = w0;
       uint32_t n = 0, np = 0;
       bool new_pair = true, ok = true;
       while (w.left > 0 && ok) {
+        // A new row tile: the row warps have put its Q and dO in TMEM.
         if (new_pair) {
-          // Every MMA so far read the previous row tile's Q and dO.
-          if (np > 0 && lane == 0) commit_both(&c.qd_empty);
-          __syncwarp();
           if (!warp_wait(&c.qd_full, np & 1, c, ctl)) break;
           ++np;
         }
-        const int s = (int)(n % ns);
-        if (!warp_wait(&c.full[s], (n / ns) & 1, c, ctl)) break;
-        // S/dP buffer n % 2 was last read by the row warps at tile n - 2.
-        if (n >= 2 && !warp_wait(&c.s_free[n & 1], ((n - 2) >> 1) & 1, c, ctl)) break;
+        const int s = (int)(n % kNS1);
+        if (!warp_wait(&c.full[s], (n / kNS1) & 1, c, ctl)) break;
+        // S and dP of tile n - 1 have been read out of TMEM.
+        if (n >= 1 && !warp_wait(&c.s_free, (n - 1) & 1, c, ctl)) break;
         tc_fence_after();
         if (lane == 0) {
           const uint64_t kd = rdesc + (uint64_t)((s * kStage1) >> 4);
-          const uint64_t vd = rdesc + (uint64_t)((s * kStage1 + kItem32) >> 4);
-          const uint32_t tS = tmem + 64 * (n & 1), tP = tmem + 128 + 64 * (n & 1);
+          const uint64_t vd = rdesc + (uint64_t)((s * kStage1 + kItem64) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
-            // A: [128 rows x 16 d] of Q / dO; B: [32 keys x 16 d] of K / V; both
-            // K-major, 8-row groups 1024 B apart, a K step walks 32 B inside a
-            // 64-column block, then to the next block.
-            const uint32_t aoff = (uint32_t)((kk >> 2) * (kRows * 128) + (kk & 3) * 32);
-            const uint32_t boff = (uint32_t)((kk >> 2) * (32 * 128) + (kk & 3) * 32);
-            umma_pair_ss(tS, qdesc + (aoff >> 4), kd + (boff >> 4), kIdescScore,
-                         kk > 0 ? 1u : 0u);
+            // A: [128 rows x 16 d] of Q / dO in TMEM (a row per lane, bf16
+            // pairs per column: a K step is 8 columns); B: [64 keys x 16 d] of
+            // K / V, K-major, 8-row groups 1024 B apart, a K step walks 32 B
+            // inside a 64-column block (8 KB), then to the next block.
+            const uint32_t boff = (uint32_t)((kk >> 2) * (64 * 128) + (kk & 3) * 32);
+            umma_pair_ts(tS, tQ + 8 * kk, kd + (boff >> 4), kIdescScore, kk > 0 ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t aoff = (uint32_t)((kk >> 2) * (kRows * 128) + (kk & 3) * 32);
-            const uint32_t boff = (uint32_t)((kk >> 2) * (32 * 128) + (kk & 3) * 32);
-            umma_pair_ss(tP, dodesc + (aoff >> 4), vd + (boff >> 4), kIdescScore,
-                         kk > 0 ? 1u : 0u);
+            const uint32_t boff = (uint32_t)((kk >> 2) * (64 * 128) + (kk & 3) * 32);
+            umma_pair_ts(tP, tdO + 8 * kk, vd + (boff >> 4), kIdescScore, kk > 0 ? 1u : 0u);
           }
           commit_both(&c.empty[s]);
-          commit_both(&c.s_full[n & 1]);
+          commit_both(&c.s_full);
         }
         __syncwarp();
         ++n;
@@ -489,29 +560,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
     }
   } else {
     // ------------------------------------------ row warps (both CTAs)
-    // A warp reaches only the TMEM lanes of quarter warp % 4; two warps share
-    // each quarter's 32 rows, warp 2 + q + 4h taking keys [32h, 32h + 32) of
-    // every tile.  P = exp2(S c - lse) needs no running maximum, so the halves
-    // never exchange anything.
+    // A warp reaches only the TMEM lanes of quarter warp % 4; four warps share
+    // each quarter's 32 rows, warp 2 + q + 4 h taking keys [32 h, 32 h + 32)
+    // of every tile.  P = exp2(S c - lse) needs no running maximum, so the
+    // warps never exchange anything.
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int part = (warp - 2) >> 2;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float cs = p.scale_log2;
-    const uint32_t s_free_l0 = mapa_shared(smem_u32(&c.s_free[0]), 0);
-    const uint32_t s_free_l1 = mapa_shared(smem_u32(&c.s_free[1]), 0);
+    const uint32_t s_free_l = mapa_shared(smem_u32(&c.s_free), 0);
+    const uint32_t qd_full_l = mapa_shared(smem_u32(&c.qd_full), 0);
     // The warp's 32 x 32 P and dS boxes leave by TMA bulk stores from a 2 KB
-    // stage, laid out as the tensor map's 64-byte swizzle expects.
-    uint8_t* wstage = stage + (warp - 2) * (kWarpStage / 2);
+    // stage laid out as the tensor map's 64-byte swizzle expects; the same
+    // stage turns the row tile's Q / dO slabs into rows on their way to TMEM.
+    uint8_t* wstage = stage + (warp - 2) * kBox1;
     const uint64_t stream = l2_policy_evict_first();
+    bool store_pending = false;   // lane 0's bulk stores may still read the stage
+    bool ok = true;
+
     TileWalk w = w0;
     uint32_t n = 0;
-    bool new_pair = true, ok = true;
-    bool store_pending = false;   // lane 0's bulk stores may still read the stage
+    bool new_pair = true;
     // Per row tile: this thread's row.
     uint32_t csq = 0;
     bool row_expert = false, row_live = false;
     float lse2 = 0.f, Dv = 0.f;
     int rho0 = 0;                                           // the warp's row 0 in its batch element
+    if (w.left > 0)
+      score_copy_rows(p, w.b, w.pair, rank, quarter, part, tmem, wstage, store_pending, pinfo,
+                      n_pairs, qd_full_l);
     while (w.left > 0 && ok) {
       if (new_pair) {
         rho0 = w.pair * 2 * kRows + (int)rank * kRows + quarter * 32;
@@ -526,35 +603,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
         lse2 = row_live ? p.lse[g0 + lane] * kLog2e : 0.f;
         Dv = row_live ? p.D[g0 + lane] : 0.f;
       }
-      const int bs = (int)(n & 1);
-      const int k0 = w.kt * kKT;
-      const int kh = k0 + 32 * half;                        // this warp's first key
+      const int k0 = w.kt * kKT1;
+      const int kh = k0 + 32 * part;                        // this warp's first key
       // Keys of this tile the row sees: a prefix (block index is
       // non-decreasing), minus FAST keys for expert rows and padding keys.
       // The tile's last key visible means every key is (most tiles).
-      int e = kKT;
-      if ((uint32_t)(codes[min(k0 + kKT, S) - 1] >> 2) > csq) {
+      int e = kKT1;
+      if ((uint32_t)(codes[min(k0 + kKT1, S) - 1] >> 2) > csq) {
         e = 0;
 #pragma unroll
-        for (int step = kKT; step >= 1; step >>= 1) {
+        for (int step = kKT1; step >= 1; step >>= 1) {
           const int probe = e + step;
-          if (probe <= kKT && (uint32_t)(codes[k0 + probe - 1] >> 2) <= csq) e = probe;
+          if (probe <= kKT1 && (uint32_t)(codes[k0 + probe - 1] >> 2) <= csq) e = probe;
         }
       }
-      e = row_live ? min(e, S - k0) - 32 * half : 0;       // visible keys of this half
-      const uint32_t tf = c.flags[w.kt >> 1];
+      e = row_live ? min(e, S - k0) - 32 * part : 0;       // visible keys of this warp's 32
+      const uint32_t tf = c.flags[w.kt];
       const bool hole = ((tf & 1u) && row_expert) || (tf & 4u);
-      if (!warp_wait(&c.s_full[bs], (n >> 1) & 1, c, ctl)) break;
+      if (!warp_wait(&c.s_full, n & 1, c, ctl)) break;
       tc_fence_after();
+      // The next tile; when it starts a new row tile, its Q and dO go to TMEM
+      // now (every MMA that read the old ones has completed: S is here), so
+      // that its MMAs overlap this tile's P and dS (they wait for the copy
+      // anyway, so reading S after it costs nothing).
+      TileWalk nw = w;
+      const bool next_new = walk_next(nw, c, pinfo, codes, S, n_kt, n_pairs, tok_per_pair);
+      if (next_new) {
+        score_copy_rows(p, nw.b, nw.pair, rank, quarter, part, tmem, wstage, store_pending,
+                        pinfo, n_pairs, qd_full_l);
+        store_pending = false;   // the copy waited for the stage
+      }
       uint32_t s0[32], d0[32];
-      tmem_ld32(tmem + lane_off + 64 * bs + 32 * half, s0);
-      tmem_ld32(tmem + lane_off + 128 + 64 * bs + 32 * half, d0);
+      tmem_ld32(tmem + lane_off + 32 * part, s0);
+      tmem_ld32(tmem + lane_off + 128 + 32 * part, d0);
       tmem_ld_wait();
       reg_fence(s0);
       reg_fence(d0);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(bs ? s_free_l1 : s_free_l0);
+      if (lane == 0) mbar_arrive_remote(s_free_l);
       uint32_t hid = 0u;               // bit j: key kh + j hidden by the hole rule
       if (hole) {
         const uint4* kc = reinterpret_cast<const uint4*>(codes + kh);
@@ -581,7 +668,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
         dk[j >> 1] = cvt_bf16x2(p0 * (__uint_as_float(d0[j]) - Dv),
                                 p1 * (__uint_as_float(d0[j + 1]) - Dv));
       }
-      if (rho0 < rows_per_b) {
+      if (rho0 < rows_per_b && kh < p.Skp) {
         // Row `lane` of each box: its 16-byte chunk j at j ^ ((lane / 2) % 4).
         // Rows past the batch element's end are clipped by the tensor map.
         uint8_t* const line = wstage + lane * 64;
@@ -607,7 +694,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
         }
       }
       ++n;
-      new_pair = walk_next(w, c, pinfo, codes, S, n_kt, n_pairs, tok_per_pair);
+      w = nw;
+      new_pair = next_new;
     }
     if (store_pending && lane == 0) tma_store_wait_all();
     __syncwarp();
@@ -619,7 +707,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
   cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem, 256);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -1082,8 +1170,6 @@ BwdTcPlan bwd_tc_plan(int B, int S, int Hq, int sms) {
   pl.n_sup = (S + kSup - 1) / kSup;
   pl.Skp = (S + kKT - 1) / kKT * kKT;
   pl.clusters = max(sms / 2, 1);
-  // Two K/V stages in the score pass when they fit beside the codes.
-  pl.ns1 = smem_need(ops1(2), S, pl.n_pairs * 4) + 1024 <= kSmemLimit ? 2 : 1;
   // Row chunks of the dK/dV pass: the fewest that keep the SM pairs as busy
   // as any larger count would (whole waves of clusters).
   const long long units = (long long)B * pl.n_sup;
@@ -1127,7 +1213,7 @@ cudaError_t launch_backward_tc(const BwdTcParams& p, const DevCtl& ctl, cudaStre
   const int units = p.B * n_pairs;
   const int persistent = p.mask_bs == 0 ? min(units, p.clusters) : units;
   e = launch_cluster_kernel(bwd_score_kernel, persistent,
-                            smem_need(ops1(p.ns1), p.S, n_pairs * 4), p, ctl, st, kT1);
+                            smem_need(kOps1, p.S, n_pairs * 4), p, ctl, st, kT1);
   if (e != cudaSuccess) return e;
   e = launch_cluster_kernel(bwd_dkdv_tc_kernel, p.B * n_sup * p.n_chunks,
                             smem_need(kOps2, p.S, 0), p, ctl, st);

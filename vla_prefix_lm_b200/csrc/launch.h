@@ -91,10 +91,8 @@ cudaError_t launch_backward(const BwdParams& p, cudaStream_t st);
 // Gradient of the prefill on tensor cores (bwd_tc.cu): bf16, Hkv = 1, d = 256.
 // Tensor maps are 4-D views (64, rows, column blocks, B) as for TcParams.
 struct BwdTcParams {
-  CUtensorMap map_q;    // q rows [B, S*Hq, 256], box (64, 128, 4, 1)
-  CUtensorMap map_do;   // dout rows, box (64, 128, 4, 1)
-  CUtensorMap map_k32;  // keys [B, S, 256], box (64, 32, 4, 1)
-  CUtensorMap map_v32;  // values, box (64, 32, 4, 1)
+  CUtensorMap map_k64;  // keys [B, S, 256], box (64, 64, 4, 1): the score pass's K item
+  CUtensorMap map_v64;  // values, box (64, 64, 4, 1)
   CUtensorMap map_kh;   // keys, box (64, 64, 2, 1): 64 keys x 128 columns
   CUtensorMap map_qh;   // q rows, box (64, 64, 2, 1)
   CUtensorMap map_doh;  // dout rows, box (64, 64, 2, 1)
@@ -106,6 +104,7 @@ struct BwdTcParams {
   const uint8_t* ar;
   const int32_t* seg;
   long long mask_bs;
+  const void* q;        // q rows (bf16), for the score pass's TMEM copy
   const void* out;      // forward output (bf16), for D
   const void* dout;
   const float* lse;     // [B, S*Hq] natural log
@@ -117,7 +116,6 @@ struct BwdTcParams {
   float* dk;
   float* dv;
   int B, S, Hq, Skp, n_chunks, pairs_per_chunk;
-  int ns1;              // K/V stages of the score pass (1 or 2, by shared memory)
   int clusters;         // SM pairs the persistent passes use
   float scale, scale_log2;
 };
@@ -126,7 +124,7 @@ struct BwdTcParams {
 // padded key count of the P / dS workspace, the dK/dV row chunks, and the
 // workspace layout (byte offsets, total).
 struct BwdTcPlan {
-  int n_pairs, n_sup, Skp, n_chunks, pairs_per_chunk, ns1, clusters;
+  int n_pairs, n_sup, Skp, n_chunks, pairs_per_chunk, clusters;
   size_t off_D, off_P, off_dS, off_part, bytes;
 };
 BwdTcPlan bwd_tc_plan(int B, int S, int Hq, int sms);
