@@ -63,8 +63,12 @@ __device__ __forceinline__ uint4 pack(const float (&f)[4], float*) {
                     __float_as_uint(f[3]));
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kRopeThreads)
+// kU heads' loads are in flight together per thread; kMinBlocks CTAs of the
+// kernel fit on an SM.  A grid that fills the GPU several times over keeps
+// four heads in flight and five CTAs per SM; a grid of at most two CTAs per
+// SM takes all nine heads of the pi0 shapes at once, four CTAs per SM.
+template <typename T, int kU, int kMinBlocks>
+__global__ void __launch_bounds__(kRopeThreads, kMinBlocks)
     rope_kernel(T* q, T* k, const uint8_t* tmask, long long tmask_bs, const uint8_t* pmask,
                 long long pmask_bs, int S, int P, int Hq, int Hkv, int d, int tok,
                 double log2_base, int32_t* pos_out) {
@@ -128,7 +132,6 @@ __global__ void __launch_bounds__(kRopeThreads)
   }
   T* gq = q + bt * Hq * d + vi * N;
   T* gk = k ? k + bt * Hkv * d + vi * N : nullptr;
-  constexpr int kU = 4;                          // heads whose loads are in flight together
   for (int h0 = 0; h0 < Hq + Hk; h0 += kU) {
     uint4 x1[kU], x2[kU];
 #pragma unroll
@@ -211,15 +214,16 @@ cudaError_t launch_rope(const RopeParams& p, const DevCtl& ctl, cudaStream_t st)
   const int tok = rope_tokens_per_cta(p.d, p.f32);
   dim3 grid((p.S + tok - 1) / tok, p.B);
   const double log2_base = log2((double)p.base);
+  const bool small = (long long)grid.x * grid.y <= 2LL * sm_count();
   if (p.f32)
-    return launch_pdl(rope_kernel<float>, grid, dim3(kRopeThreads), 0, st,
-                      static_cast<float*>(p.q), static_cast<float*>(p.k), p.tmask, p.tmask_bs,
-                      p.pmask, p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, tok, log2_base,
-                      p.pos_out);
-  return launch_pdl(rope_kernel<__nv_bfloat16>, grid, dim3(kRopeThreads), 0, st,
-                    static_cast<__nv_bfloat16*>(p.q), static_cast<__nv_bfloat16*>(p.k), p.tmask,
-                    p.tmask_bs, p.pmask, p.pmask_bs, p.S, p.P, p.Hq, p.Hkv, p.d, tok, log2_base,
-                    p.pos_out);
+    return launch_pdl(small ? rope_kernel<float, 9, 4> : rope_kernel<float, 4, 5>, grid,
+                      dim3(kRopeThreads), 0, st, static_cast<float*>(p.q),
+                      static_cast<float*>(p.k), p.tmask, p.tmask_bs, p.pmask, p.pmask_bs, p.S,
+                      p.P, p.Hq, p.Hkv, p.d, tok, log2_base, p.pos_out);
+  return launch_pdl(small ? rope_kernel<__nv_bfloat16, 9, 4> : rope_kernel<__nv_bfloat16, 4, 5>,
+                    grid, dim3(kRopeThreads), 0, st, static_cast<__nv_bfloat16*>(p.q),
+                    static_cast<__nv_bfloat16*>(p.k), p.tmask, p.tmask_bs, p.pmask, p.pmask_bs,
+                    p.S, p.P, p.Hq, p.Hkv, p.d, tok, log2_base, p.pos_out);
 }
 
 cudaError_t launch_euler(float* x, const void* v, bool v_f32, float dt, long long n,
