@@ -984,7 +984,8 @@ def run_case(args):
                                              stream=stream)
     elif name.endswith("_prefill"):
         w = W.workload({"mmdit_prefill": 5, "pi0_prefill": 2, "pi05_prefill": 4}[name])
-        q, k, v = (W.device_draw((w.B, w.Sq, h, w.d), 7_000_000 + j, w.d, w.dtype, dev)
+        B = args.case_batch or w.B
+        q, k, v = (W.device_draw((B, w.Sq, h, w.d), 7_000_000 + j, w.d, w.dtype, dev)
                    for j, h in enumerate((w.Hq, w.Hkv, w.Hkv)))
         ar = torch.tensor(w.ar, dtype=torch.uint8, device=dev)
         seg = None if w.seg is None else torch.tensor(w.seg, dtype=torch.int32, device=dev)
@@ -1072,6 +1073,9 @@ def main():
     ap.add_argument("--case", choices=CASES,
                     help="run --launches calls of one workload on one input set (for ncu)")
     ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--case-batch", type=int, default=0,
+                    help="with a prefill --case: this batch size instead of the workload's "
+                         "(a smaller case of the same kernel for multi-pass captures)")
     ap.add_argument("--plumbing-check", action="store_true",
                     help="CPU-only multi-rank check of the timing plumbing (gloo)")
     args = ap.parse_args()
