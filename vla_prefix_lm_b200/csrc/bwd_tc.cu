@@ -658,15 +658,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
         }
       }
       uint32_t pk[16], dk[16];
+      if (__all_sync(0xffffffffu, e >= 32 && hid == 0u)) {
+        // Every row of the warp sees all 32 keys (most tiles): no predicates.
+        const float2 nD = make_float2(-Dv, -Dv);
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float2 t = ffma2(make_float2(__uint_as_float(s0[j]), __uint_as_float(s0[j + 1])),
-                               make_float2(cs, cs), make_float2(-lse2, -lse2));
-        const float p0 = (j < e && !((hid >> j) & 1u)) ? ex2(t.x) : 0.f;
-        const float p1 = (j + 1 < e && !((hid >> (j + 1)) & 1u)) ? ex2(t.y) : 0.f;
-        pk[j >> 1] = cvt_bf16x2(p0, p1);
-        dk[j >> 1] = cvt_bf16x2(p0 * (__uint_as_float(d0[j]) - Dv),
-                                p1 * (__uint_as_float(d0[j + 1]) - Dv));
+        for (int j = 0; j < 32; j += 2) {
+          const float2 t = ffma2(make_float2(__uint_as_float(s0[j]), __uint_as_float(s0[j + 1])),
+                                 make_float2(cs, cs), make_float2(-lse2, -lse2));
+          const float2 pp = make_float2(ex2(t.x), ex2(t.y));
+          const float2 dd = fadd2(make_float2(__uint_as_float(d0[j]), __uint_as_float(d0[j + 1])),
+                                  nD);
+          pk[j >> 1] = cvt_bf16x2(pp.x, pp.y);
+          dk[j >> 1] = cvt_bf16x2(pp.x * dd.x, pp.y * dd.y);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float2 t = ffma2(make_float2(__uint_as_float(s0[j]), __uint_as_float(s0[j + 1])),
+                                 make_float2(cs, cs), make_float2(-lse2, -lse2));
+          const float p0 = (j < e && !((hid >> j) & 1u)) ? ex2(t.x) : 0.f;
+          const float p1 = (j + 1 < e && !((hid >> (j + 1)) & 1u)) ? ex2(t.y) : 0.f;
+          pk[j >> 1] = cvt_bf16x2(p0, p1);
+          dk[j >> 1] = cvt_bf16x2(p0 * (__uint_as_float(d0[j]) - Dv),
+                                  p1 * (__uint_as_float(d0[j + 1]) - Dv));
+        }
       }
       if (rho0 < rows_per_b && kh < p.Skp) {
         // Row `lane` of each box: its 16-byte chunk j at j ^ ((lane / 2) % 4).
