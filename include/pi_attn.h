@@ -222,8 +222,8 @@ int pi_attn_prefill_backward(const pi_attn_desc* desc, const void* q, const void
  *   that may overlap on the GPU need distinct workspaces.
  * Two kernels serve this call.  A suffix of at most 8 query rows (Sq * Hq <=
  * 8, e.g. the single-token decode of "Pi0-FAST 模型架构", 4.1) streams the cache
- * through the CUDA cores of a cluster of 8 CTAs per batch element and merges
- * on chip: it needs no workspace.  Larger suffixes run on the tensor cores;
+ * through a cluster of 8 CTAs per batch element (warp-level mma.sync tensor
+ * instructions) and merges on chip: it needs no workspace.  Larger suffixes run on the tensor cores;
  * batches too small to fill the GPU split the cache over several CTA pairs
  * and need a workspace for the partial results.
  */
