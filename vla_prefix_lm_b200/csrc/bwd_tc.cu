@@ -21,9 +21,10 @@
 //               TMEM (N = 128 pair MMAs in TS form: the row tile's Q and dO
 //               sit in TMEM as the A operand, 256 of the 512 columns, copied
 //               in by the row warps when the row tile changes; S and dP take
-//               the other 256, one buffer); one thread per row and 32 keys
-//               forms P and dS in fp32 and writes both as bf16 to the
-//               caller's workspace [B, rows, Skp] (Skp = S rounded up to 64).
+//               the other 256, one buffer each, freed separately so that the
+//               next tile's S MMAs run while dP is read); one thread per row
+//               and 32 keys forms P and dS in fp32 and writes both as bf16 to
+//               the caller's workspace [B, rows, Skp] (Skp = S rounded up to 64).
 //               Persistent: each SM pair takes an equal, contiguous run of the
 //               (batch, 256-row tile, key tile) sequence; shared memory holds
 //               a two-stage K/V ring and the P/dS store stages.
@@ -87,8 +88,8 @@ struct __align__(8) Ctl {
   uint64_t full[4];       // leader: a ring stage of both CTAs landed
   uint64_t empty[4];      // each CTA: its stage may be refilled
   uint64_t qd_full;       // leader (score pass): the pair's 32 row warps put Q and dO in TMEM
-  uint64_t s_full;        // each CTA (score pass): S and dP of a tile in TMEM
-  uint64_t s_free;        // leader (score pass): the pair's 32 row warps read them
+  uint64_t s_full[2];     // each CTA (score pass): S [0] / dP [1] of a tile in TMEM
+  uint64_t s_free[2];     // leader (score pass): the pair's 32 row warps read S / dP
   uint64_t done[2];       // each CTA: an accumulator is final
   uint64_t acc_free[2];   // leader (dQ pass): the pair's 8 row warps read an accumulator
   uint64_t drain;         // leader: every MMA issued has completed
@@ -411,8 +412,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
       mbar_init(&c.empty[s], 1);
     }
     mbar_init(&c.qd_full, 32);
-    mbar_init(&c.s_full, 1);
-    mbar_init(&c.s_free, 32);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&c.s_full[i], 1);
+      mbar_init(&c.s_free[i], 32);
+    }
     mbar_init(&c.drain, 1);
     c.abort = 0;
     fence_barrier_init();
@@ -527,12 +530,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
         }
         const int s = (int)(n % kNS1);
         if (!warp_wait(&c.full[s], (n / kNS1) & 1, c, ctl)) break;
-        // S and dP of tile n - 1 have been read out of TMEM.
-        if (n >= 1 && !warp_wait(&c.s_free, (n - 1) & 1, c, ctl)) break;
+        // S and dP have a TMEM buffer each, freed separately: the S MMAs of
+        // tile n start once S of tile n - 1 has been read, while the row warps
+        // still read dP (and the dP MMAs follow once they have), so the
+        // tensor pipe need not idle while the row warps drain the tile.
+        if (n >= 1 && !warp_wait(&c.s_free[0], (n - 1) & 1, c, ctl)) break;
         tc_fence_after();
         if (lane == 0) {
           const uint64_t kd = rdesc + (uint64_t)((s * kStage1) >> 4);
-          const uint64_t vd = rdesc + (uint64_t)((s * kStage1 + kItem64) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
             // A: [128 rows x 16 d] of Q / dO in TMEM (a row per lane, bf16
@@ -542,13 +547,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
             const uint32_t boff = (uint32_t)((kk >> 2) * (64 * 128) + (kk & 3) * 32);
             umma_pair_ts(tS, tQ + 8 * kk, kd + (boff >> 4), kIdescScore, kk > 0 ? 1u : 0u);
           }
+          commit_both(&c.s_full[0]);
+        }
+        __syncwarp();
+        if (n >= 1 && !warp_wait(&c.s_free[1], (n - 1) & 1, c, ctl)) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint64_t vd = rdesc + (uint64_t)((s * kStage1 + kItem64) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
             const uint32_t boff = (uint32_t)((kk >> 2) * (64 * 128) + (kk & 3) * 32);
             umma_pair_ts(tP, tdO + 8 * kk, vd + (boff >> 4), kIdescScore, kk > 0 ? 1u : 0u);
           }
           commit_both(&c.empty[s]);
-          commit_both(&c.s_full);
+          commit_both(&c.s_full[1]);
         }
         __syncwarp();
         ++n;
@@ -568,7 +580,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
     const int part = (warp - 2) >> 2;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float cs = p.scale_log2;
-    const uint32_t s_free_l = mapa_shared(smem_u32(&c.s_free), 0);
+    const uint32_t sS_free_l = mapa_shared(smem_u32(&c.s_free[0]), 0);
+    const uint32_t dP_free_l = mapa_shared(smem_u32(&c.s_free[1]), 0);
     const uint32_t qd_full_l = mapa_shared(smem_u32(&c.qd_full), 0);
     // The warp's 32 x 32 P and dS boxes leave by TMA bulk stores from a 2 KB
     // stage laid out as the tensor map's 64-byte swizzle expects; the same
@@ -580,29 +593,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
 
     TileWalk w = w0;
     uint32_t n = 0;
-    bool new_pair = true;
-    // Per row tile: this thread's row.
+    // Per row tile: this thread's row.  Its lse and D are loaded when the row
+    // tile is entered (right after its Q and dO copy) and first used after the
+    // next S wait, which hides their latency.
     uint32_t csq = 0;
     bool row_expert = false, row_live = false;
-    float lse2 = 0.f, Dv = 0.f;
+    float lse = 0.f, Dv = 0.f;
     int rho0 = 0;                                           // the warp's row 0 in its batch element
-    if (w.left > 0)
-      score_copy_rows(p, w.b, w.pair, rank, quarter, part, tmem, wstage, store_pending, pinfo,
+    auto enter_row_tile = [&](const TileWalk& t) {
+      score_copy_rows(p, t.b, t.pair, rank, quarter, part, tmem, wstage, store_pending, pinfo,
                       n_pairs, qd_full_l);
+      store_pending = false;   // the copy waited for the stage
+      rho0 = t.pair * 2 * kRows + (int)rank * kRows + quarter * 32;
+      const int rho = rho0 + lane;
+      const bool row_valid = rho < rows_per_b;
+      const int tq1 = min(t.pair * tok_per_pair + tok_per_pair, S) - 1;
+      const uint32_t cq = codes[row_valid ? rho / Hq : tq1];
+      csq = cq >> 2;
+      row_expert = (cq & 2u) != 0;
+      row_live = row_valid && !is_pad(cq);
+      const long long g0 = (long long)t.b * rows_per_b + rho0;
+      lse = row_live ? p.lse[g0 + lane] : 0.f;
+      Dv = row_live ? p.D[g0 + lane] : 0.f;
+    };
+    if (w.left > 0) enter_row_tile(w);
     while (w.left > 0 && ok) {
-      if (new_pair) {
-        rho0 = w.pair * 2 * kRows + (int)rank * kRows + quarter * 32;
-        const int rho = rho0 + lane;
-        const bool row_valid = rho < rows_per_b;
-        const int tq1 = min(w.pair * tok_per_pair + tok_per_pair, S) - 1;
-        const uint32_t cq = codes[row_valid ? rho / Hq : tq1];
-        csq = cq >> 2;
-        row_expert = (cq & 2u) != 0;
-        row_live = row_valid && !is_pad(cq);
-        const long long g0 = (long long)w.b * rows_per_b + rho0;
-        lse2 = row_live ? p.lse[g0 + lane] * kLog2e : 0.f;
-        Dv = row_live ? p.D[g0 + lane] : 0.f;
-      }
       const int k0 = w.kt * kKT1;
       const int kh = k0 + 32 * part;                        // this warp's first key
       // Keys of this tile the row sees: a prefix (block index is
@@ -620,28 +635,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
       e = row_live ? min(e, S - k0) - 32 * part : 0;       // visible keys of this warp's 32
       const uint32_t tf = c.flags[w.kt];
       const bool hole = ((tf & 1u) && row_expert) || (tf & 4u);
-      if (!warp_wait(&c.s_full, n & 1, c, ctl)) break;
+      if (!warp_wait(&c.s_full[0], n & 1, c, ctl)) break;
       tc_fence_after();
-      // The next tile; when it starts a new row tile, its Q and dO go to TMEM
-      // now (every MMA that read the old ones has completed: S is here), so
-      // that its MMAs overlap this tile's P and dS (they wait for the copy
-      // anyway, so reading S after it costs nothing).
-      TileWalk nw = w;
-      const bool next_new = walk_next(nw, c, pinfo, codes, S, n_kt, n_pairs, tok_per_pair);
-      if (next_new) {
-        score_copy_rows(p, nw.b, nw.pair, rank, quarter, part, tmem, wstage, store_pending,
-                        pinfo, n_pairs, qd_full_l);
-        store_pending = false;   // the copy waited for the stage
-      }
-      uint32_t s0[32], d0[32];
+      const float lse2 = lse * kLog2e;
+      // S first: P is formed while the dP MMAs run.
+      uint32_t s0[32];
       tmem_ld32(tmem + lane_off + 32 * part, s0);
-      tmem_ld32(tmem + lane_off + 128 + 32 * part, d0);
       tmem_ld_wait();
       reg_fence(s0);
-      reg_fence(d0);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(s_free_l);
+      if (lane == 0) mbar_arrive_remote(sS_free_l);
       uint32_t hid = 0u;               // bit j: key kh + j hidden by the hole rule
       if (hole) {
         const uint4* kc = reinterpret_cast<const uint4*>(codes + kh);
@@ -657,60 +661,79 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
           }
         }
       }
+      // P in place of S (fp32; exact zeros where the key is hidden).
       uint32_t pk[16], dk[16];
       if (__all_sync(0xffffffffu, e >= 32 && hid == 0u)) {
         // Every row of the warp sees all 32 keys (most tiles): no predicates.
-        const float2 nD = make_float2(-Dv, -Dv);
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const float2 t = ffma2(make_float2(__uint_as_float(s0[j]), __uint_as_float(s0[j + 1])),
                                  make_float2(cs, cs), make_float2(-lse2, -lse2));
-          const float2 pp = make_float2(ex2(t.x), ex2(t.y));
-          const float2 dd = fadd2(make_float2(__uint_as_float(d0[j]), __uint_as_float(d0[j + 1])),
-                                  nD);
-          pk[j >> 1] = cvt_bf16x2(pp.x, pp.y);
-          dk[j >> 1] = cvt_bf16x2(pp.x * dd.x, pp.y * dd.y);
+          s0[j] = __float_as_uint(ex2(t.x));
+          s0[j + 1] = __float_as_uint(ex2(t.y));
         }
       } else {
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const float2 t = ffma2(make_float2(__uint_as_float(s0[j]), __uint_as_float(s0[j + 1])),
                                  make_float2(cs, cs), make_float2(-lse2, -lse2));
-          const float p0 = (j < e && !((hid >> j) & 1u)) ? ex2(t.x) : 0.f;
-          const float p1 = (j + 1 < e && !((hid >> (j + 1)) & 1u)) ? ex2(t.y) : 0.f;
-          pk[j >> 1] = cvt_bf16x2(p0, p1);
-          dk[j >> 1] = cvt_bf16x2(p0 * (__uint_as_float(d0[j]) - Dv),
-                                  p1 * (__uint_as_float(d0[j + 1]) - Dv));
+          s0[j] = __float_as_uint((j < e && !((hid >> j) & 1u)) ? ex2(t.x) : 0.f);
+          s0[j + 1] = __float_as_uint((j + 1 < e && !((hid >> (j + 1)) & 1u)) ? ex2(t.y) : 0.f);
         }
       }
-      if (rho0 < rows_per_b && kh < p.Skp) {
-        // Row `lane` of each box: its 16-byte chunk j at j ^ ((lane / 2) % 4).
-        // Rows past the batch element's end are clipped by the tensor map.
+#pragma unroll
+      for (int j = 0; j < 32; j += 2)
+        pk[j >> 1] = cvt_bf16x2(__uint_as_float(s0[j]), __uint_as_float(s0[j + 1]));
+      // Row `lane` of each 32 x 32 box: its 16-byte chunk j at j ^ ((lane / 2) % 4).
+      // Rows past the batch element's end are clipped by the tensor map.
+      const bool do_store = rho0 < rows_per_b && kh < p.Skp;
+      auto store_box = [&](const uint32_t* src, const CUtensorMap* map) {
         uint8_t* const line = wstage + lane * 64;
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          const uint32_t* src = m == 0 ? pk : dk;
-          if (store_pending) {   // the previous box has been read out of the stage
-            if (lane == 0) tma_store_wait_read();
-            __syncwarp();
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            *reinterpret_cast<uint4*>(line + ((j ^ ((lane >> 1) & 3)) << 4)) =
-                make_uint4(src[4 * j], src[4 * j + 1], src[4 * j + 2], src[4 * j + 3]);
-          fence_proxy_async_smem();
+        if (store_pending) {   // the previous box has been read out of the stage
+          if (lane == 0) tma_store_wait_read();
           __syncwarp();
-          if (lane == 0) {
-            tma_store_3d_hint(m == 0 ? &p.map_pw : &p.map_dsw, wstage, kh, rho0, w.b, stream);
-            tma_store_commit();
-          }
-          __syncwarp();
-          store_pending = true;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4*>(line + ((j ^ ((lane >> 1) & 3)) << 4)) =
+              make_uint4(src[4 * j], src[4 * j + 1], src[4 * j + 2], src[4 * j + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d_hint(map, wstage, kh, rho0, w.b, stream);
+          tma_store_commit();
+        }
+        __syncwarp();
+        store_pending = true;
+      };
+      if (do_store) store_box(pk, &p.map_pw);
+      if (!warp_wait(&c.s_full[1], n & 1, c, ctl)) break;
+      tc_fence_after();
+      uint32_t d0[32];
+      tmem_ld32(tmem + lane_off + 128 + 32 * part, d0);
+      tmem_ld_wait();
+      reg_fence(d0);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(dP_free_l);
+      {
+        const float2 nD = make_float2(-Dv, -Dv);
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float2 dd = fadd2(make_float2(__uint_as_float(d0[j]), __uint_as_float(d0[j + 1])),
+                                  nD);
+          dk[j >> 1] = cvt_bf16x2(__uint_as_float(s0[j]) * dd.x,
+                                  __uint_as_float(s0[j + 1]) * dd.y);
         }
       }
+      if (do_store) store_box(dk, &p.map_dsw);
+      // The next tile; when it starts a new row tile, its Q and dO go to TMEM
+      // now (every MMA that read the old ones has completed: dP is here).
+      TileWalk nw = w;
+      const bool next_new = walk_next(nw, c, pinfo, codes, S, n_kt, n_pairs, tok_per_pair);
+      if (next_new) enter_row_tile(nw);
       ++n;
       w = nw;
-      new_pair = next_new;
     }
     if (store_pending && lane == 0) tma_store_wait_all();
     __syncwarp();
