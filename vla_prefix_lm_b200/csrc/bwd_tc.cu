@@ -429,10 +429,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
     tmem_alloc_pair(&c.tmem_base, 512);
     tmem_relinquish_pair();
   }
-  // Nothing above touched global memory (it may overlap the previous kernel);
-  // its results are visible from here on.
-  pdl_wait();
-  pdl_launch_dependents();
+  // Up to the wait below this kernel may overlap the previous one.  It reads
+  // only ar_mask and the segment ids there, which no kernel of this library
+  // writes; and it starts only after the backward's first launch (the
+  // row-dot, which waits before it releases its dependents) has seen the
+  // caller's earlier work complete.
   const Flags32 flags0 = load_flags32(ar_b, seg_b, S, (int)threadIdx.x * 32);
   build_codes_x32<kT1>(ar_b, seg_b, S, pad128(S), codes, c.scan, flags0,
                       TileSums{c.cs_first, c.cs_last, c.flags});
@@ -450,6 +451,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT1, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();                 // the previous kernel's results are visible from here on
+  pdl_launch_dependents();
   const uint32_t tmem = c.tmem_base;
 
   // This cluster's run.
@@ -806,16 +809,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     tmem_alloc_pair(&c.tmem_base, 512);
     tmem_relinquish_pair();
   }
-  // Nothing above touched global memory (it may overlap the previous kernel);
-  // its results are visible from here on.
-  pdl_wait();
-  pdl_launch_dependents();
+  // Up to the wait below this kernel may overlap the previous one.  It reads
+  // only ar_mask and the segment ids there, which no kernel of this library
+  // writes; and it starts only after the backward's first launch (the
+  // row-dot, which waits before it releases its dependents) has seen the
+  // caller's earlier work complete.
   const Flags32 flags0 = load_flags32(ar_b, seg_b, S, (int)threadIdx.x * 32);
   build_codes_x32<kT>(ar_b, seg_b, S, pad128(S), codes, c.scan, flags0,
                       TileSums{c.cs_first, c.cs_last, c.flags});
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();                 // the previous kernel's results are visible from here on
+  pdl_launch_dependents();
   const uint32_t tmem = c.tmem_base;
   const uint32_t tdV = tmem, tdK = tmem + 256;
 
@@ -998,16 +1004,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kT, 1)
     tmem_alloc_pair(&c.tmem_base, 512);
     tmem_relinquish_pair();
   }
-  // Nothing above touched global memory (it may overlap the previous kernel);
-  // its results are visible from here on.
-  pdl_wait();
-  pdl_launch_dependents();
+  // Up to the wait below this kernel may overlap the previous one.  It reads
+  // only ar_mask and the segment ids there, which no kernel of this library
+  // writes; and it starts only after the backward's first launch (the
+  // row-dot, which waits before it releases its dependents) has seen the
+  // caller's earlier work complete.
   const Flags32 flags0 = load_flags32(ar_b, seg_b, S, (int)threadIdx.x * 32);
   build_codes_x32<kT>(ar_b, seg_b, S, pad128(S), codes, c.scan, flags0,
                       TileSums{c.cs_first, c.cs_last, c.flags});
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();                 // the previous kernel's results are visible from here on
+  pdl_launch_dependents();
   const uint32_t tmem = c.tmem_base;
 
   // Visited key tiles of row tile `pair`: kt = first, then next_tile.
