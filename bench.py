@@ -50,7 +50,7 @@ L2_BYTES = 126 * 2**20
 # DRAM traffic of the prefill kernel per launch on the headline workload, from
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only for
 # the kernel sources whose digest is recorded beside it.
-TRAFFIC = {"bytes": 125987840, "src_sha": "9ec1c2fe430fb24e", "workload": "mmdit"}
+TRAFFIC = {"bytes": 125614848, "src_sha": "d4a1a6103d0956fc", "workload": "mmdit"}
 KERNEL_SOURCES = ("vla_prefix_lm_b200/csrc/tc_pair.cu", "vla_prefix_lm_b200/csrc/common.cuh",
                   "vla_prefix_lm_b200/csrc/mask.cuh")
 

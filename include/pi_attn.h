@@ -45,8 +45,9 @@
  * The device addresses of the status word and of that scratch are looked up
  * on every call (cudaGetSymbolAddress, a host-side lookup that is allowed
  * during stream capture), so they stay right after a device reset
- * (cudaDeviceReset) reloads the module; each device's SM count is looked up
- * once and kept.
+ * (cudaDeviceReset) reloads the module; the kernels' shared-memory attributes
+ * are set on every call for the same reason; each device's SM count is looked
+ * up once and kept.
  *
  * Errors: every entry point returns PI_OK or a PI_ERR_* code.  Argument
  * errors are detected on the host before anything is enqueued (nothing is

@@ -432,7 +432,9 @@ __global__ void __cluster_dims__(kDecCluster, 1, 1) __launch_bounds__(kDecThread
 bool decode_applies(int Sq, int Hq) { return Sq >= 1 && Sq * Hq <= kDecRows; }
 
 cudaError_t launch_decode(const DecodeParams& p, const DevCtl& ctl, cudaStream_t st) {
-  static const cudaError_t attr = cudaFuncSetAttribute(
+  // Per call: the attribute belongs to the device (and to the module, which a
+  // device reset reloads).
+  const cudaError_t attr = cudaFuncSetAttribute(
       decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmemBytes);
   if (attr != cudaSuccess) return attr;
   dim3 grid(kDecCluster, (unsigned)p.B);

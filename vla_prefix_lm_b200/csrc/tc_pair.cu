@@ -1051,7 +1051,9 @@ int pair_smem_bytes(int n_code_tokens) {
 
 template <bool kSuffix, bool kCacheMask, class L>
 cudaError_t launch_pair(const TcParams& p, const DevCtl& ctl, dim3 grid, cudaStream_t st) {
-  static const cudaError_t attr_err = cudaFuncSetAttribute(
+  // Per call: the attribute belongs to the device (and to the module, which a
+  // device reset reloads).
+  const cudaError_t attr_err = cudaFuncSetAttribute(
       tc_pair_kernel<kSuffix, kCacheMask, L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
       kSmemLimit);
   if (attr_err != cudaSuccess) return attr_err;
@@ -1113,7 +1115,7 @@ cudaError_t launch_debug_tiles(const uint8_t* ar, const int32_t* seg, long long 
                                int S, int Hq, uint8_t* out, cudaStream_t st) {
   const int n_pairs = (S * Hq + 2 * kBM - 1) / (2 * kBM);
   const int smem = (int)((sizeof(DbgTileSmem) + 127) / 128 * 128) + pad_tokens(S) * 2;
-  static const cudaError_t attr = cudaFuncSetAttribute(
+  const cudaError_t attr = cudaFuncSetAttribute(
       debug_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
   if (attr != cudaSuccess) return attr;
   debug_tiles_kernel<<<dim3(n_pairs, B), kThreads, smem, st>>>(ar, seg, mask_bs, S, Hq, out);
