@@ -2,7 +2,8 @@
 header declares, and rejects bad arguments before touching the GPU.
 
 Nothing here launches a kernel; each call below fails validation (or is a
-B == 0 no-op) before any CUDA runtime call is made.
+B == 0 no-op) before any CUDA runtime call is made, or is a host-only size
+query (which at most asks the runtime for the device's SM count).
 """
 
 import ctypes
@@ -109,6 +110,81 @@ def test_workspace_query_is_host_only():
     assert n >= 0
     assert L.pi_attn_suffix_workspace_bytes(ctypes.byref(_desc(b, Hq=0))) == 0
     assert L.pi_attn_suffix_workspace_bytes(None) == 0
+
+
+def _sm_count():
+    """The SM count the library plans with: the device's, or 148 (a B200) with
+    no device, as the library assumes when the runtime finds none."""
+    import torch
+    if torch.cuda.is_available():
+        return torch.cuda.get_device_properties(0).multi_processor_count
+    return 148
+
+
+@pytest.mark.parametrize("B,S", [(8, 611), (16, 938), (2, 300), (1, 17), (3, 2000)])
+def test_backward_workspace_follows_its_layout(B, S):
+    """The bf16 backward's workspace is D (fp32 per row), P and dS (bf16
+    [B, rows, Skp], Skp = S rounded up to 64), each 256-byte aligned, plus the
+    dK / dV partials of 2 <= n_chunks <= (256-row tiles) row chunks when the
+    rows are split: 2 * n_chunks * B * (256-key groups) * 256 * 256 fp32."""
+    b, L = _lib()
+    Hq = 8
+    n = L.pi_attn_prefill_backward_workspace_bytes(ctypes.byref(_desc(b, B=B, Sq=S, Hq=Hq)))
+    up = lambda x: (x + 255) // 256 * 256
+    rows = S * Hq
+    skp = (S + 63) // 64 * 64
+    base = up(B * rows * 4) + 2 * up(B * rows * skp * 2)
+    assert n >= base
+    chunk = 2 * B * ((S + 255) // 256) * 256 * 256 * 4
+    extra = n - base
+    assert extra % chunk == 0, (n, base, chunk)
+    n_chunks = extra // chunk
+    assert n_chunks == 0 or 2 <= n_chunks <= (rows + 255) // 256
+    if (B, S) == (8, 611):
+        assert n == 138_011_392        # the pi0 figure the bench reports
+
+
+def test_prefill_split_workspace_and_plan():
+    """pi_attn_prefill_ws: one round of fp32 pieces (256 rows x (256 + 2)
+    floats each) per SM pair for bf16 with a batch-shared mask, nothing
+    otherwise; MM-DiT (532 units on 74 SM pairs: 14 in the last round) splits
+    5 ways, pi0 and pi0.5 stay whole."""
+    b, L = _lib()
+    pairs = _sm_count() // 2
+    q = lambda **kw: ctypes.byref(_desc(b, **kw))
+    assert L.pi_attn_prefill_workspace_bytes(q(B=4, Sq=4250)) == pairs * 256 * 258 * 4
+    assert L.pi_attn_prefill_workspace_bytes(q(B=4, Sq=4250, dtype=b.PI_F32)) == 0
+    assert L.pi_attn_prefill_workspace_bytes(q(B=4, Sq=4250, mask_batch_stride=4250)) == 0
+    assert L.pi_attn_prefill_tail_splits(q(B=8, Sq=611)) == 1
+    assert L.pi_attn_prefill_tail_splits(q(B=16, Sq=938)) == 1
+    if pairs == 74:
+        assert L.pi_attn_prefill_tail_splits(q(B=4, Sq=4250)) == 5
+
+
+def test_suffix_workspace_and_noalloc_capacity():
+    """Split-K suffix scratch is a whole number s of partial sets (B x Sq*Hq
+    rows of 256 + 2 fp32), 2 <= s <= 8, and s x (CTA pairs per element) x B
+    never exceeds the SM pairs; none when the batch fills the SMs (the pi0
+    suffix step, B = 32) or for a few-row suffix (the decode kernel).  At the
+    pi0 suffix shape every batch size and cache length fits the no-alloc
+    buffer."""
+    b, L = _lib()
+    pairs = _sm_count() // 2
+    cap = L.pi_attn_suffix_noalloc_capacity()
+    assert cap == 16 << 20
+    q = lambda **kw: ctypes.byref(_desc(b, **kw))
+    assert L.pi_attn_suffix_workspace_bytes(q(B=1, Sq=1, P=3000)) == 0
+    if pairs == 74:
+        assert L.pi_attn_suffix_workspace_bytes(q(B=32, Sq=51, P=816)) == 0
+    for Bn in list(range(1, 40)) + [64, 128]:
+        for P in (1, 128, 816, 3000, 16000):
+            n = L.pi_attn_suffix_workspace_bytes(q(B=Bn, Sq=51, P=P))
+            part = Bn * 51 * 8 * 258 * 4
+            assert n % part == 0
+            s = n // part
+            assert s == 0 or 2 <= s <= 8
+            assert s * 2 * Bn <= pairs          # two CTA pairs per element (408 rows)
+            assert n <= cap, (Bn, P, n)
 
 
 def test_status_strings_and_wait_limit():
