@@ -187,6 +187,30 @@ def test_suffix_workspace_and_noalloc_capacity():
             assert n <= cap, (Bn, P, n)
 
 
+def test_split_prefill_and_noalloc_argument_errors():
+    """Host-side rejections, before anything is enqueued: a split-prefill
+    workspace smaller than the query's size (PI_ERR_ARG) or misaligned
+    (PI_ERR_ALIGN); a no-alloc suffix whose split-K scratch would exceed the
+    fixed buffer (PI_ERR_UNSUPPORTED: B = 1, 512 tokens x 8 heads against a
+    3000-key cache needs 4 splits x 4096 rows x 1032 B = 16.1 MiB)."""
+    b, L = _lib()
+    d = _desc(b, B=4, Sq=4250)
+    need = L.pi_attn_prefill_workspace_bytes(ctypes.byref(d))
+    assert need > 0
+    args = (FAKE, FAKE, FAKE, FAKE, None, FAKE, None)
+    rc = L.pi_attn_prefill_ws(ctypes.byref(d), *args, FAKE, ctypes.c_size_t(need - 16), None)
+    assert rc == b.PI_ERR_ARG
+    rc = L.pi_attn_prefill_ws(ctypes.byref(d), *args, FAKE_MIS, ctypes.c_size_t(need), None)
+    assert rc == b.PI_ERR_ALIGN
+    big = _desc(b, B=1, Sq=512, P=3000)
+    if _sm_count() != 148:
+        return                      # the split count (and so the size) follows the SM count
+    assert L.pi_attn_suffix_workspace_bytes(ctypes.byref(big)) > L.pi_attn_suffix_noalloc_capacity()
+    rc = L.pi_attn_suffix_noalloc(ctypes.byref(big), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                  None)
+    assert rc == b.PI_ERR_UNSUPPORTED
+
+
 def test_status_strings_and_wait_limit():
     b, L = _lib()
     for code in range(6):
