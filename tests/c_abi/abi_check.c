@@ -36,6 +36,13 @@ int main(void) {
   /* workspace queries are host-only */
   /* bf16, one KV head, d = 256: D (fp32 per row) and the bf16 P / dS tiles */
   CHECK(pi_attn_prefill_backward_workspace_bytes(&d) == 2 * 128 * 4 + 2 * (2 * 128 * 64 * 2));
+  /* the split prefill: scratch for bf16 with a batch-shared mask only */
+  CHECK(pi_attn_prefill_tail_splits(&d) >= 1);
+  d.dtype = PI_F32;
+  CHECK(pi_attn_prefill_workspace_bytes(&d) == 0);
+  d.dtype = PI_BF16;
+  CHECK(pi_attn_prefill_ws(&d, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL) ==
+        PI_ERR_ARG);
   d.P = 816; d.Sq = 51; d.B = 1;
   (void)pi_attn_suffix_workspace_bytes(&d);
   CHECK(pi_attn_suffix_noalloc_capacity() > 0);
